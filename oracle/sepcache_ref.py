@@ -1,0 +1,105 @@
+"""SepCache streaming-decode oracle (test infrastructure): cache state machine + fp64 decode.
+
+[BD] "SepLLM's Architecture: Composing Efficiency" splits the streaming KV cache into an
+Initial Cache (first tokens), a Local Window Cache of capacity w, a Past Window Cache and a
+Separator Cache that keeps only separator KV of older tokens, with total capacity c. [SP]
+"Limitations & Caveats" and [AS] "Measured effects" (removing positional-encoding shifting)
+say positions are taken inside the cache, not in the original text.
+
+Readings where the pages are silent (listed again in the design doc):
+* Fixed partitions c = a + s + w; the Past Window Cache has size 0, so compression happens
+  one token at a time: when the window overflows, its oldest token moves to the separator
+  cache if it is a separator and is evicted otherwise; when the separator cache overflows,
+  its oldest entry is evicted. The first a tokens go to the initial cache whatever their flag.
+* Per step: the update happens first, then the new token's query attends to every retained
+  slot, itself included.
+* Positional-encoding shifting: the position of a retained key is its rank in the logical
+  order [initial | separators oldest first | window oldest first]; the query's position is
+  its own rank (occupied - 1). Keys are kept un-rotated and rotated afresh at every step.
+* RoPE convention: rotate-half pairs (k, k + d/2) with angle p * theta^(-2k/d).
+"""
+
+from __future__ import annotations
+
+from collections import deque
+
+import numpy as np
+
+
+class SepCacheSim:
+    """Integer state machine of one SepCache sequence: which original tokens are retained.
+
+    Holds original token positions only; the K/V content is looked up by position.
+    """
+
+    def __init__(self, a, s, w):
+        assert a >= 0 and s >= 0 and w >= 1
+        self.a, self.s, self.w = a, s, w
+        self.initial = []
+        self.seps = deque()
+        self.window = deque()
+        self.t = 0
+
+    def append(self, is_sep):
+        """Add the next token (original position self.t) and compress if over capacity."""
+        tok = self.t
+        self.t += 1
+        if tok < self.a:
+            self.initial.append(tok)
+            return
+        self.window.append((tok, bool(is_sep)))
+        if len(self.window) > self.w:
+            old, old_sep = self.window.popleft()
+            if old_sep:
+                self.seps.append(old)
+                if len(self.seps) > self.s:
+                    self.seps.popleft()
+
+    def order(self):
+        """Retained original positions in logical order; a key's rank is its in-cache position."""
+        return list(self.initial) + list(self.seps) + [p for p, _ in self.window]
+
+
+def rope_rotate(x, pos, theta):
+    """Rotate-half RoPE of vectors x [..., d] at integer positions pos (broadcast on [...]).
+
+    out[k] = x[k] cos(p w_k) - x[k + d/2] sin(p w_k), out[k + d/2] = x[k + d/2] cos(p w_k)
+    + x[k] sin(p w_k), w_k = theta^(-2k/d), in fp64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    h = d // 2
+    w = theta ** (-2.0 * np.arange(h) / d)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * w
+    c, s = np.cos(ang), np.sin(ang)
+    x1, x2 = x[..., :h], x[..., h:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def decode_attention(q, k_ret, v_ret, theta, scale):
+    """Single-query attention of one step over the retained keys, with in-cache positions.
+
+    q [Hq, d] is the new token's query (un-rotated); k_ret/v_ret [n_ret, Hkv, d] are the
+    retained keys/values in logical order (un-rotated keys). Key r sits at position r, the
+    query at position n_ret - 1. Returns o [Hq, d] and lse [Hq] (natural log), fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k_ret = np.asarray(k_ret, dtype=np.float64)
+    v_ret = np.asarray(v_ret, dtype=np.float64)
+    n_ret = k_ret.shape[0]
+    Hq, d = q.shape
+    Hkv = k_ret.shape[1]
+    G = Hq // Hkv
+    kr = rope_rotate(k_ret, np.arange(n_ret)[:, None], theta)
+    qr = rope_rotate(q, np.full((Hq,), n_ret - 1), theta)
+    o = np.zeros((Hq, d))
+    lse = np.zeros(Hq)
+    for h in range(Hq):
+        kh = h // G
+        s = scale * (kr[:, kh, :] @ qr[h])
+        mx = s.max()
+        e = np.exp(s - mx)
+        l = e.sum()
+        o[h] = (e / l) @ v_ret[:, kh, :]
+        lse[h] = mx + np.log(l)
+    return o, lse

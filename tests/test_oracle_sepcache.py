@@ -1,0 +1,113 @@
+"""Pins for the SepCache oracle (CPU only): hand-derived trajectory, invariants, RoPE forms."""
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import load_golden
+from oracle import sepattn_ref as R
+from oracle import sepcache_ref as C
+
+
+def test_golden_trajectory():
+    g = load_golden("sepcache_a1_s2_w3.txt")
+    sim = C.SepCacheSim(g["a"][0], g["s"][0], g["w"][0])
+    seps = set(g["sep"])
+    for t in sorted(g["step"]):
+        sim.append(t in seps)
+        assert sim.order() == g["step"][t], t
+
+
+@pytest.mark.parametrize("a,s,w,p", [(4, 64, 732, 0.1), (0, 3, 5, 0.3), (2, 0, 4, 0.5),
+                                     (1, 2, 1, 0.9), (3, 1, 2, 0.0)])
+def test_invariants(a, s, w, p):
+    rng = np.random.default_rng(a * 100 + s)
+    steps = 3000
+    flags = rng.random(steps) < p
+    sim = C.SepCacheSim(a, s, w)
+    for t in range(steps):
+        sim.append(flags[t])
+        order = sim.order()
+        assert len(order) <= a + s + w
+        assert order == sorted(order) and len(set(order)) == len(order)
+        assert order[-1] == t                     # the new token is retained
+        n_init = min(t + 1, a)
+        assert order[:n_init] == list(range(n_init))
+        n_win = min(t + 1 - n_init, w)
+        assert order[len(order) - n_win:] == list(range(t + 1 - n_win, t + 1))
+        middle = order[n_init:len(order) - n_win]
+        assert len(middle) <= s
+        assert all(flags[j] for j in middle)
+        # every separator that left the window is retained unless s newer ones displaced it
+        left = [j for j in range(n_init, t + 1 - n_win) if flags[j]]
+        assert middle == left[max(0, len(left) - s):]
+
+
+def test_unbounded_separator_cache_equals_prefill_mask():
+    """With s >= #separators and w = n the retained set is the kept set K(t) of the mask."""
+    rng = np.random.default_rng(11)
+    a, n, steps = 3, 7, 400
+    sep = (rng.random(steps) < 0.2).astype(np.uint8)
+    sim = C.SepCacheSim(a, steps, n)
+    f = R.anchor_flags(sep, a)
+    for t in range(steps):
+        sim.append(bool(sep[t]))
+        assert sim.order() == R.kept_index_set(f, t, n).tolist()
+
+
+def test_no_separator_cache_is_streaming_llm():
+    sim = C.SepCacheSim(4, 0, 10)
+    for t in range(100):
+        sim.append(True)
+        order = sim.order()
+        assert order == list(range(min(t + 1, 4))) + list(range(max(4, t - 9), t + 1))
+
+
+def test_rope_matches_complex_multiplication():
+    rng = np.random.default_rng(12)
+    d, theta = 16, 500000.0
+    x = rng.standard_normal((5, d))
+    pos = np.array([0, 1, 7, 799, 12345])
+    y = C.rope_rotate(x, pos, theta)
+    w = theta ** (-np.arange(d // 2) * 2.0 / d)
+    z = (x[:, : d // 2] + 1j * x[:, d // 2:]) * np.exp(1j * pos[:, None] * w)
+    np.testing.assert_allclose(y, np.concatenate([z.real, z.imag], axis=1), atol=1e-12)
+    np.testing.assert_allclose(C.rope_rotate(x, np.zeros(5), theta), x, atol=0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+
+
+def test_rope_small_worked_example():
+    # d = 4, theta = 100: frequencies 1 and 0.1; e_0 at position 1 -> (cos 1, 0, sin 1, 0)
+    y = C.rope_rotate(np.array([1.0, 0, 0, 0]), np.array(1), 100.0)
+    np.testing.assert_allclose(y, [np.cos(1.0), 0.0, np.sin(1.0), 0.0], atol=1e-15)
+
+
+def test_rope_relative_invariance():
+    rng = np.random.default_rng(13)
+    d = 32
+    q, k = rng.standard_normal(d), rng.standard_normal((6, d))
+    pk = np.array([0, 3, 4, 9, 10, 11])
+    s1 = C.rope_rotate(k, pk, 1e4) @ C.rope_rotate(q, np.array(11), 1e4)
+    s2 = C.rope_rotate(k, pk + 500, 1e4) @ C.rope_rotate(q, np.array(511), 1e4)
+    np.testing.assert_allclose(s1, s2, atol=1e-10)
+
+
+def test_decode_without_eviction_is_causal_rope_attention():
+    """Before any eviction the in-cache rank is the original position: ordinary RoPE decode."""
+    rng = np.random.default_rng(14)
+    Hq, Hkv, d, theta, t = 4, 2, 8, 1e4, 9
+    k = rng.standard_normal((t + 1, Hkv, d))
+    v = rng.standard_normal((t + 1, Hkv, d))
+    q = rng.standard_normal((Hq, d))
+    o, lse = C.decode_attention(q, k, v, theta, 0.3)
+    # library reference: rotate at original positions, SDPA over all keys (last query sees all)
+    kr = C.rope_rotate(k, np.arange(t + 1)[:, None], theta)
+    qr = C.rope_rotate(q, np.full(Hq, t), theta)
+    G = Hq // Hkv
+    qt = torch.from_numpy(qr)[:, None, :]
+    kt = torch.from_numpy(np.repeat(kr, G, axis=1)).permute(1, 0, 2)
+    vt = torch.from_numpy(np.repeat(v, G, axis=1)).permute(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=0.3)[:, 0].numpy()
+    np.testing.assert_allclose(o, ref, atol=1e-12)
+    s = 0.3 * np.einsum("khd,hd->hk", np.repeat(kr, G, axis=1), qr)
+    np.testing.assert_allclose(lse, np.log(np.exp(s).sum(1)), atol=1e-12)

@@ -1,0 +1,448 @@
+// SepCache streaming decode on sm_100a: cache update (append / compress) and single-query
+// attention with positional-encoding shifting.
+//
+// Cache blocks ("How SepLLM reorchestrates the language model...", beiduofen.top, section
+// "SepLLM's Architecture: Composing Efficiency"): a initial slots, a separator FIFO of s slots,
+// a local-window FIFO of w slots. When the window overflows, its oldest token moves to the
+// separator FIFO if it is a separator and is dropped otherwise; the separator FIFO drops its
+// oldest entry when full. Positions are ranks inside the cache (SepLLM project card,
+// "Limitations & Caveats": streaming needs positional-encoding shifting), so a key is rotated
+// by RoPE(rank) at every step and the query by RoPE(occupied - 1).
+//
+// Slot storage per (sequence, KV head) is [c][d] with c = a + s + w: slots 0..a-1 initial,
+// a..a+s-1 separator ring, a+s..c-1 window ring. Keys are stored without rotation.
+//
+// Decode: one thread-block cluster of kSplit CTAs per (sequence, KV head). Each CTA streams a
+// contiguous range of ranks with 16 half-warps (one key per half-warp per step, 8 elements of
+// the row per lane, coalesced loads), rotates keys in registers (cos/sin advanced by a complex
+// recurrence from the table row of the first rank), keeps an online softmax per query head,
+// and combines: half-warps through shared memory, CTAs of the cluster through distributed
+// shared memory. No global scratch is used.
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+
+#include "sep_common.cuh"
+#include "sep_launch.h"
+
+namespace cg = cooperative_groups;
+
+namespace sep {
+
+constexpr int kSplit = 4;          // CTAs per cluster (per sequence and KV head)
+constexpr int kDecThreads = 256;   // 16 half-warps
+constexpr int kHalfWarps = kDecThreads / 16;
+
+// ------------------------------------------------------------------ init
+__global__ void sepcache_init_kernel(int S, int c, int d, double theta, int32_t* meta,
+                                     int32_t* slot_pos, uint8_t* slot_sep, float* rope_cs) {
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nthr = gridDim.x * blockDim.x;
+  for (int e = tid; e < S * SEPCACHE_META; e += nthr) meta[e] = 0;
+  for (int e = tid; e < S * c; e += nthr) {
+    slot_pos[e] = -1;
+    slot_sep[e] = 0;
+  }
+  const int h = d / 2;
+  for (int e = tid; e < c * h; e += nthr) {
+    const int p = e / h, k = e % h;
+    const double ang = (double)p * pow(theta, -2.0 * (double)k / (double)d);
+    double sn, cs;
+    sincos(ang, &sn, &cs);
+    rope_cs[2 * e] = (float)cs;
+    rope_cs[2 * e + 1] = (float)sn;
+  }
+}
+
+// ------------------------------------------------------------------ update
+// One CTA per sequence. Thread 0 plans the move, all threads copy rows (16-byte vectors).
+__global__ void __launch_bounds__(128) sepcache_update_kernel(
+    int Hkv, int d, int a, int s, int w, uint4* __restrict__ k_slots, uint4* __restrict__ v_slots,
+    int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep, int32_t* __restrict__ meta,
+    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+    const uint8_t* __restrict__ sep_new) {
+  const int seq = blockIdx.x;
+  const int c = a + s + w;
+  int32_t* m = meta + (size_t)seq * SEPCACHE_META;
+  __shared__ int plan[4];  // slot_new, move_from, move_to, t
+  if (threadIdx.x == 0) {
+    const int t = m[SEPCACHE_META_T];
+    int slot_new, move_from = -1, move_to = -1;
+    if (t < a) {
+      slot_new = t;
+      m[SEPCACHE_META_NINIT] = t + 1;
+    } else {
+      int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
+      if (win_cnt < w) {
+        slot_new = a + s + (win_head + win_cnt) % w;
+        m[SEPCACHE_META_WIN_CNT] = win_cnt + 1;
+      } else {
+        // window full: its oldest token leaves and the new token takes its slot
+        const int old_slot = a + s + win_head;
+        if (slot_sep[(size_t)seq * c + old_slot] && s > 0) {
+          int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
+          int to;
+          if (sep_cnt < s) {
+            to = a + (sep_head + sep_cnt) % s;
+            m[SEPCACHE_META_SEP_CNT] = sep_cnt + 1;
+          } else {  // separator FIFO full: the oldest separator is dropped
+            to = a + sep_head;
+            m[SEPCACHE_META_SEP_HEAD] = (sep_head + 1) % s;
+          }
+          move_from = old_slot;
+          move_to = to;
+        }
+        slot_new = old_slot;
+        m[SEPCACHE_META_WIN_HEAD] = (win_head + 1) % w;
+      }
+    }
+    m[SEPCACHE_META_T] = t + 1;
+    plan[0] = slot_new;
+    plan[1] = move_from;
+    plan[2] = move_to;
+    plan[3] = t;
+  }
+  __syncthreads();
+  const int slot_new = plan[0], move_from = plan[1], move_to = plan[2], t = plan[3];
+  const int vec = d / 8;  // 16-byte vectors per row
+  const size_t seq_rows = (size_t)seq * Hkv * c;
+  if (move_from >= 0) {
+    for (int e = threadIdx.x; e < Hkv * vec; e += blockDim.x) {
+      const int hh = e / vec, q = e % vec;
+      const size_t src = (seq_rows + (size_t)hh * c + move_from) * vec + q;
+      const size_t dst = (seq_rows + (size_t)hh * c + move_to) * vec + q;
+      k_slots[dst] = k_slots[src];
+      v_slots[dst] = v_slots[src];
+    }
+    if (threadIdx.x == 0) {
+      slot_pos[(size_t)seq * c + move_to] = slot_pos[(size_t)seq * c + move_from];
+      slot_sep[(size_t)seq * c + move_to] = 1;
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < Hkv * vec; e += blockDim.x) {
+    const int hh = e / vec, q = e % vec;
+    const size_t dst = (seq_rows + (size_t)hh * c + slot_new) * vec + q;
+    const size_t src = ((size_t)seq * Hkv + hh) * vec + q;
+    k_slots[dst] = k_new[src];
+    v_slots[dst] = v_new[src];
+  }
+  if (threadIdx.x == 0) {
+    slot_pos[(size_t)seq * c + slot_new] = t;
+    slot_sep[(size_t)seq * c + slot_new] = sep_new[seq] != 0;
+  }
+}
+
+// Slot holding logical rank r (r < occupied).
+__device__ __forceinline__ int rank_to_slot(int r, int ninit, int sep_head, int sep_cnt,
+                                            int win_head, int a, int s, int w) {
+  if (r < ninit) return r;
+  r -= ninit;
+  if (r < sep_cnt) return a + (sep_head + r) % s;
+  r -= sep_cnt;
+  return a + s + (win_head + r) % w;
+}
+
+// N consecutive bf16 (N = 2 or 4, 4- or 8-byte aligned) to fp32.
+template <int N>
+__device__ __forceinline__ void load_bf16_vec(const __nv_bfloat16* p, float (&out)[N]) {
+  if constexpr (N == 4) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    out[0] = __low2float(x); out[1] = __high2float(x);
+    out[2] = __low2float(y); out[3] = __high2float(y);
+  } else {
+    static_assert(N == 2, "two or four elements per lane");
+    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u);
+    out[0] = __low2float(x); out[1] = __high2float(x);
+  }
+}
+
+// ------------------------------------------------------------------ decode
+// EPL = elements of a key row per lane (d / 16): the lane owns EPL/2 rotation pairs
+// (k, k + d/2), k = lane16 * EPL/2 + e.
+template <int D, int G>
+__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
+    sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int w,
+                           const __nv_bfloat16* __restrict__ k_slots,
+                           const __nv_bfloat16* __restrict__ v_slots,
+                           const int32_t* __restrict__ meta, const float2* __restrict__ rope_cs,
+                           const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ o,
+                           float* __restrict__ lse, float scale_log2) {
+  constexpr int HP = D / 32;       // rotation pairs per lane
+  constexpr int HALF = D / 2;
+  const int split = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int c = a + s + w;
+  const int tid = threadIdx.x, lane16 = tid & 15, hw = tid >> 4;
+  cg::cluster_group cluster = cg::this_cluster();
+
+  const int32_t* m = meta + (size_t)seq * SEPCACHE_META;
+  const int ninit = m[SEPCACHE_META_NINIT];
+  const int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
+  const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
+  const int occ = ninit + sep_cnt + win_cnt;
+  const int mq = occ - 1;  // the query's own rank
+  const int chunk = (occ + kSplit - 1) / kSplit;
+  const int r0 = split * chunk, r1 = min(occ, r0 + chunk);
+
+  // query heads of this KV head, rotated by RoPE(mq) and scaled by scale*log2(e)
+  float qr[G][2 * HP];
+  {
+    const float2* cs = rope_cs + (size_t)max(mq, 0) * HALF;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const __nv_bfloat16* qh = q + ((size_t)seq * Hq + kvh * G + g) * D;
+#pragma unroll
+      for (int e = 0; e < HP; ++e) {
+        const int k = lane16 * HP + e;
+        const float x1 = __bfloat162float(qh[k]), x2 = __bfloat162float(qh[k + HALF]);
+        const float2 r = cs[k];
+        qr[g][e] = (x1 * r.x - x2 * r.y) * scale_log2;
+        qr[g][HP + e] = (x2 * r.x + x1 * r.y) * scale_log2;
+      }
+    }
+  }
+
+  float mrun[G], lrun[G], acc[G][2 * HP];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    mrun[g] = -INFINITY;
+    lrun[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 2 * HP; ++e) acc[g][e] = 0.f;
+  }
+
+  // this half-warp's ranks: r0 + hw, r0 + hw + 16, ...; cos/sin by recurrence with step 16
+  int r = r0 + hw;
+  float cr[HP], sr[HP], cd[HP], sd[HP];
+  if (r < r1) {
+#pragma unroll
+    for (int e = 0; e < HP; ++e) {
+      const int k = lane16 * HP + e;
+      const float2 v0 = rope_cs[(size_t)r * HALF + k];
+      cr[e] = v0.x;
+      sr[e] = v0.y;
+      const float2 st = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
+      cd[e] = st.x;
+      sd[e] = st.y;
+    }
+  }
+  const size_t row_base = ((size_t)seq * Hkv + kvh) * c;
+  for (; r < r1; r += kHalfWarps) {
+    const int slot = rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w);
+    const __nv_bfloat16* kr = k_slots + (row_base + slot) * D + lane16 * HP;
+    const __nv_bfloat16* vr = v_slots + (row_base + slot) * D + lane16 * HP;
+    float k1[HP], k2[HP], v1[HP], v2[HP];
+    load_bf16_vec<HP>(kr, k1);
+    load_bf16_vec<HP>(kr + HALF, k2);
+    load_bf16_vec<HP>(vr, v1);
+    load_bf16_vec<HP>(vr + HALF, v2);
+    // rotate the key by RoPE(r) and dot with every query head
+    float part[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) part[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < HP; ++e) {
+      const float y1 = k1[e] * cr[e] - k2[e] * sr[e];
+      const float y2 = k2[e] * cr[e] + k1[e] * sr[e];
+#pragma unroll
+      for (int g = 0; g < G; ++g) part[g] = fmaf(qr[g][e], y1, fmaf(qr[g][HP + e], y2, part[g]));
+    }
+    // advance cos/sin by kHalfWarps positions
+#pragma unroll
+    for (int e = 0; e < HP; ++e) {
+      const float cn = cr[e] * cd[e] - sr[e] * sd[e];
+      const float sn = sr[e] * cd[e] + cr[e] * sd[e];
+      cr[e] = cn;
+      sr[e] = sn;
+    }
+    // reduce over the 16 lanes of the half-warp
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
+    }
+    // online softmax per head (lazy rescale: only when the max grows by more than 2^8)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float sc = part[g];
+      if (sc > mrun[g] + 8.0f) {
+        const float alpha = ex2(mrun[g] - sc);
+        lrun[g] *= alpha;
+#pragma unroll
+        for (int e = 0; e < 2 * HP; ++e) acc[g][e] *= alpha;
+        mrun[g] = sc;
+      }
+      const float pg = ex2(sc - mrun[g]);
+      lrun[g] += pg;
+#pragma unroll
+      for (int e = 0; e < HP; ++e) {
+        acc[g][e] = fmaf(pg, v1[e], acc[g][e]);
+        acc[g][HP + e] = fmaf(pg, v2[e], acc[g][HP + e]);
+      }
+    }
+  }
+
+  // ---- combine the two half-warps of each warp (lanes l and l^16 hold the same columns)
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float mo = __shfl_xor_sync(0xffffffffu, mrun[g], 16);
+    const float lo = __shfl_xor_sync(0xffffffffu, lrun[g], 16);
+    const float M = fmaxf(mrun[g], mo);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    const float fs = ex2(mrun[g] - Mu), fo = ex2(mo - Mu);
+#pragma unroll
+    for (int e = 0; e < 2 * HP; ++e) {
+      const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], 16);
+      acc[g][e] = acc[g][e] * fs + ao * fo;
+    }
+    lrun[g] = lrun[g] * fs + lo * fo;
+    mrun[g] = M;
+  }
+  // ---- combine the warps of this CTA through shared memory
+  constexpr int kWarps = kDecThreads / 32;
+  __shared__ float s_m[kWarps][G], s_l[kWarps][G];
+  __shared__ float s_acc[kWarps][G][D];
+  __shared__ float s_res[G][D + 2];  // this CTA's combined (acc..., m, l) per head
+  const int warp = tid >> 5;
+  if ((tid & 31) < 16) {
+    if (lane16 == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        s_m[warp][g] = mrun[g];
+        s_l[warp][g] = lrun[g];
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+#pragma unroll
+      for (int e = 0; e < HP; ++e) {
+        s_acc[warp][g][lane16 * HP + e] = acc[g][e];
+        s_acc[warp][g][HALF + lane16 * HP + e] = acc[g][HP + e];
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < G * D; e += kDecThreads) {
+    const int g = e / D, col = e % D;
+    float M = -INFINITY;
+    for (int x = 0; x < kWarps; ++x) M = fmaxf(M, s_m[x][g]);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float sum = 0.f, lsum = 0.f;
+    for (int x = 0; x < kWarps; ++x) {
+      const float f = ex2(s_m[x][g] - Mu);
+      sum += s_acc[x][g][col] * f;
+      lsum += s_l[x][g] * f;
+    }
+    s_res[g][col] = sum;
+    if (col == 0) {
+      s_res[g][D] = M;
+      s_res[g][D + 1] = lsum;
+    }
+  }
+  cluster.sync();
+  // ---- CTA 0 of the cluster combines the kSplit partial results through DSMEM
+  if (cluster.block_rank() == 0) {
+    for (int e = tid; e < G * D; e += kDecThreads) {
+      const int g = e / D, col = e % D;
+      float mm[kSplit], ll[kSplit], aa[kSplit];
+      float M = -INFINITY;
+#pragma unroll
+      for (int x = 0; x < kSplit; ++x) {
+        const float* rr = cluster.map_shared_rank(&s_res[0][0], x);
+        mm[x] = rr[g * (D + 2) + D];
+        ll[x] = rr[g * (D + 2) + D + 1];
+        aa[x] = rr[g * (D + 2) + col];
+        M = fmaxf(M, mm[x]);
+      }
+      const float Mu = (M == -INFINITY) ? 0.f : M;
+      float sum = 0.f, lsum = 0.f;
+#pragma unroll
+      for (int x = 0; x < kSplit; ++x) {
+        const float f = ex2(mm[x] - Mu);
+        sum += aa[x] * f;
+        lsum += ll[x] * f;
+      }
+      const int hq = kvh * G + g;
+      o[((size_t)seq * Hq + hq) * D + col] = __float2bfloat16(sum / lsum);
+      if (col == 0 && lse)
+        lse[(size_t)seq * Hq + hq] = (M + __log2f(lsum)) * 0.69314718055994531f;
+    }
+  }
+  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 has read it
+}
+
+// ------------------------------------------------------------------ export order
+__global__ void sepcache_export_kernel(int a, int s, int w, const int32_t* __restrict__ meta,
+                                       const int32_t* __restrict__ slot_pos,
+                                       int32_t* __restrict__ pos_out, int32_t* __restrict__ count) {
+  const int seq = blockIdx.x;
+  const int c = a + s + w;
+  const int32_t* m = meta + (size_t)seq * SEPCACHE_META;
+  const int ninit = m[SEPCACHE_META_NINIT];
+  const int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
+  const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
+  const int occ = ninit + sep_cnt + win_cnt;
+  for (int r = threadIdx.x; r < c; r += blockDim.x) {
+    pos_out[(size_t)seq * c + r] =
+        r < occ ? slot_pos[(size_t)seq * c +
+                           rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w)]
+                : -1;
+  }
+  if (threadIdx.x == 0) count[seq] = occ;
+}
+
+cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream) {
+  const int c = st.a + st.s + st.w;
+  sepcache_init_kernel<<<64, 256, 0, stream>>>(st.S, c, st.d, (double)st.rope_theta, st.meta,
+                                               st.slot_pos, st.slot_sep, st.rope_cs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new, const void* v_new,
+                                   const uint8_t* sep_new, cudaStream_t stream) {
+  sepcache_update_kernel<<<st.S, 128, 0, stream>>>(
+      st.Hkv, st.d, st.a, st.s, st.w, reinterpret_cast<uint4*>(st.k_slots),
+      reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta,
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), sep_new);
+  return cudaGetLastError();
+}
+
+template <int D, int G>
+static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void* o, float* lse,
+                                   float scale, cudaStream_t stream) {
+  dim3 grid(kSplit, st.Hkv, st.S);
+  sepcache_decode_kernel<D, G><<<grid, kDecThreads, 0, stream>>>(
+      st.Hq, st.Hkv, st.a, st.s, st.w, reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
+      reinterpret_cast<const __nv_bfloat16*>(st.v_slots), st.meta,
+      reinterpret_cast<const float2*>(st.rope_cs), static_cast<const __nv_bfloat16*>(q),
+      static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sepcache_decode(const SepCacheState& st, const void* q, void* o, float* lse,
+                                   float scale, cudaStream_t stream) {
+  const int G = st.Hq / st.Hkv;
+#define SEP_DEC_CASE(DD, GG) \
+  if (st.d == DD && G == GG) return launch_decode_t<DD, GG>(st, q, o, lse, scale, stream);
+  SEP_DEC_CASE(128, 1)
+  SEP_DEC_CASE(128, 2)
+  SEP_DEC_CASE(128, 4)
+  SEP_DEC_CASE(128, 8)
+  SEP_DEC_CASE(64, 1)
+  SEP_DEC_CASE(64, 2)
+  SEP_DEC_CASE(64, 4)
+  SEP_DEC_CASE(64, 8)
+#undef SEP_DEC_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_sepcache_export(const SepCacheState& st, int32_t* pos_out, int32_t* count,
+                                   cudaStream_t stream) {
+  sepcache_export_kernel<<<st.S, 256, 0, stream>>>(st.a, st.s, st.w, st.meta, st.slot_pos,
+                                                   pos_out, count);
+  return cudaGetLastError();
+}
+
+}  // namespace sep

@@ -1,0 +1,56 @@
+// Host-side interface between the C-ABI layer (api.cpp) and the kernel launchers (*.cu).
+// Plain C++ types only; every pointer is a device pointer owned by the caller.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sepattn.h"
+
+namespace sep {
+
+// Device address of the sticky error word on the current device (nullptr on failure).
+unsigned* device_error_word();
+
+cudaError_t launch_mask_build(const uint8_t* sep, int B, int L, int a, int n, int bm, int bn,
+                              int32_t* anchor_idx, int32_t* anchor_cnt, int32_t* gather_end,
+                              int8_t* tile_map, int64_t* kept, cudaStream_t stream);
+
+// Copies the K/V rows of every anchor to rows 0..anchor_cnt[b]-1 of kc/vc ([B, L, Hkv, d]).
+cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* anchor_idx,
+                                   const int32_t* anchor_cnt, int B, int L, int Hkv, int d,
+                                   void* kc, void* vc, cudaStream_t stream);
+
+struct AttnMaps {
+  CUtensorMap q, k, v, kc, vc;  // 4-D {d, H, L, B}, box {64, 1, 128, 1}, 128-byte swizzle
+  CUtensorMap o, dout;          // used by the backward kernels
+};
+
+struct AttnShape {
+  int B, L, Hq, Hkv, d, a, n;
+  float scale;
+};
+
+cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint8_t* sep,
+                            const int32_t* gather_end, const int8_t* tile_map, void* o,
+                            float* lse, cudaStream_t stream);
+
+cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint8_t* sep,
+                            const int32_t* anchor_idx, const int32_t* anchor_cnt,
+                            const int32_t* gather_end, const int8_t* tile_map, const void* o,
+                            const float* lse, const void* dout, const void* q, const void* k,
+                            const void* v, void* dq, void* dk, void* dv, void* kc, void* vc,
+                            float* delta, float* dka, float* dva, cudaStream_t stream);
+
+cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream);
+cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new,
+                                   const void* v_new, const uint8_t* sep_new,
+                                   cudaStream_t stream);
+cudaError_t launch_sepcache_decode(const SepCacheState& st, const void* q, void* o, float* lse,
+                                   float scale, cudaStream_t stream);
+cudaError_t launch_sepcache_export(const SepCacheState& st, int32_t* pos_out, int32_t* count,
+                                   cudaStream_t stream);
+
+}  // namespace sep

@@ -1,0 +1,64 @@
+// Tile schedule and keep-mask helpers shared by the forward and backward attention kernels.
+//
+// keep(i, j) = j <= i && (i - j < n || f[j]) with f[j] = (j < a) || sep[j] (SepLLM, atlas.scime.ai
+// summary, section "Approach"). Query tile t (rows 128t..128t+127) reads whole key tiles
+// lo(t)..t, lo(t) = max(0, 128t - n + 1) / 128, and the anchors left of tile lo(t) (the first
+// gather_end[t] entries of the sorted anchor list), which every row of the tile keeps.
+#pragma once
+
+#include <stdint.h>
+
+namespace sep {
+
+__host__ __device__ __forceinline__ int window_lo_tile(int t, int n) {
+  const long long k = (long long)t * 128 - n + 1;
+  return k > 0 ? (int)(k / 128) : 0;
+}
+
+// Bits of one 32-column word (columns 32w..32w+31 of a 128-column tile) that lie in [lo, hi].
+__device__ __forceinline__ uint32_t range_word(long long lo, long long hi, int w) {
+  const long long l = lo - 32 * w, h = hi - 32 * w;
+  if (h < 0 || l > 31 || h < l) return 0u;
+  const uint32_t le = (h >= 31) ? 0xffffffffu : ((2u << h) - 1u);
+  const uint32_t ge = (l <= 0) ? 0xffffffffu : ~((1u << l) - 1u);
+  return le & ge;
+}
+
+// Keep bits of one 32-column word of key tile k0..k0+127 for query row i (row-major view: the
+// thread owns a query row, the columns are keys). fbits = anchor flags of the word's keys.
+__device__ __forceinline__ uint32_t window_keep_word(int w, long long i, long long k0, int n,
+                                                     int L, uint32_t fbits) {
+  const long long hi = (i < (long long)L - 1 ? i : (long long)L - 1) - k0;  // causal, in bounds
+  const long long lo = i - n + 1 - k0;                                     // inside the band
+  return range_word(lo > 0 ? lo : 0, hi, w) | (fbits & range_word(0, hi, w));
+}
+
+// Anchor flags of keys base..base+31 as a bit word (sep[j] != 0 or j < a); keys >= L read as 0.
+__device__ __forceinline__ uint32_t anchor_bits32(const uint8_t* __restrict__ sep_row,
+                                                  long long base, int L, int a) {
+  uint32_t bits = 0;
+  if (base + 32 <= L && ((reinterpret_cast<uintptr_t>(sep_row + base) & 15) == 0)) {
+    const uint4* p = reinterpret_cast<const uint4*>(sep_row + base);
+    const uint4 x0 = __ldg(p), x1 = __ldg(p + 1);
+    const uint32_t wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t v = wv[q];
+      const uint32_t nib = (uint32_t)((v & 0xffu) != 0) | ((uint32_t)(((v >> 8) & 0xffu) != 0) << 1) |
+                           ((uint32_t)(((v >> 16) & 0xffu) != 0) << 2) |
+                           ((uint32_t)(((v >> 24) & 0xffu) != 0) << 3);
+      bits |= nib << (4 * q);
+    }
+  } else {
+    for (int c = 0; c < 32; ++c) {
+      const long long j = base + c;
+      if (j < L && sep_row[j] != 0) bits |= 1u << c;
+    }
+  }
+  const long long na = (long long)a - base;  // keys j < a are anchors
+  if (na > 0) bits |= (na >= 32) ? 0xffffffffu : ((1u << na) - 1u);
+  if (base + 32 > L) bits &= range_word(0, (long long)L - 1 - base, 0);
+  return bits;
+}
+
+}  // namespace sep

@@ -1,0 +1,228 @@
+"""Thin ctypes binding of libsepattn.so: same names as the C ABI, argument marshalling only.
+
+Every computation runs in the library's CUDA kernels; this module allocates outputs and scratch
+with torch (device memory), passes raw pointers and the current CUDA stream, and turns status
+codes into exceptions. There is no CPU path: importing this module without the built library
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsepattn.so")
+
+SEP_OK = 0
+TILE = 128
+META = 8
+
+
+class SepError(RuntimeError):
+    pass
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with `python -m kv_cache_compression_sep_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "sep_mask_build": (I, [P, I, I, I, I, I, I, P, P, P, P, P, P]),
+        "sep_attn_fwd_workspace_size": (Z, [I, I, I, I]),
+        "sep_attn_fwd": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
+        "sep_attn_bwd_workspace_size": (Z, [I, I, I, I, I]),
+        "sep_attn_bwd": (I, [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, P, Z, P]),
+        "sepcache_state_init": (I, [P, P]),
+        "sepcache_update": (I, [P, P, P, P, P]),
+        "sepcache_decode": (I, [P, P, P, P, F, P]),
+        "sepcache_export_order": (I, [P, P, P, P]),
+        "sep_last_device_error": (I, []),
+        "sep_status_string": (ctypes.c_char_p, [I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+class _SepMask(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("L", ctypes.c_int), ("a", ctypes.c_int), ("n", ctypes.c_int),
+                ("sep", ctypes.c_void_p), ("anchor_idx", ctypes.c_void_p),
+                ("anchor_cnt", ctypes.c_void_p), ("gather_end", ctypes.c_void_p),
+                ("tile_map", ctypes.c_void_p)]
+
+
+class _SepCacheState(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("a", ctypes.c_int32), ("s", ctypes.c_int32),
+                ("w", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
+                ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
+                ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]
+
+
+def _check(status: int, what: str):
+    if status != SEP_OK:
+        raise SepError(f"{what}: {_lib.sep_status_string(status).decode()} ({status})")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _cuda(t, dtype, name):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise SepError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def sep_last_device_error() -> int:
+    return int(_lib.sep_last_device_error())
+
+
+@dataclasses.dataclass
+class SepMask:
+    """Outputs of sep_mask_build (device tensors) plus the flags and parameters used."""
+    sep: torch.Tensor
+    anchor_idx: torch.Tensor
+    anchor_cnt: torch.Tensor
+    gather_end: torch.Tensor
+    tile_map: torch.Tensor
+    kept: torch.Tensor
+    a: int
+    n: int
+
+    def _c(self):
+        B, L = self.sep.shape
+        return _SepMask(B, L, self.a, self.n, self.sep.data_ptr(), self.anchor_idx.data_ptr(),
+                        self.anchor_cnt.data_ptr(), self.gather_end.data_ptr(),
+                        self.tile_map.data_ptr())
+
+
+def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = TILE) -> SepMask:
+    _cuda(sep, torch.uint8, "sep")
+    B, L = sep.shape
+    T, U = -(-L // bm), -(-L // bn)
+    dev = sep.device
+    out = SepMask(sep=sep,
+                  anchor_idx=torch.empty(B, L, dtype=torch.int32, device=dev),
+                  anchor_cnt=torch.empty(B, dtype=torch.int32, device=dev),
+                  gather_end=torch.empty(B, T, dtype=torch.int32, device=dev),
+                  tile_map=torch.empty(B, T, U, dtype=torch.int8, device=dev),
+                  kept=torch.empty(B, dtype=torch.int64, device=dev), a=a, n=n)
+    _check(_lib.sep_mask_build(_ptr(sep), B, L, a, n, bm, bn, _ptr(out.anchor_idx),
+                               _ptr(out.anchor_cnt), _ptr(out.gather_end), _ptr(out.tile_map),
+                               _ptr(out.kept), _stream()), "sep_mask_build")
+    return out
+
+
+def sep_attn_fwd_workspace_size(B, L, Hkv, d) -> int:
+    return int(_lib.sep_attn_fwd_workspace_size(B, L, Hkv, d))
+
+
+def sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d) -> int:
+    return int(_lib.sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d))
+
+
+def _workspace(nbytes, device, ws):
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+    return ws
+
+
+def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspace=None):
+    """O, LSE of separator-sparse attention. q [B,L,Hq,d], k/v [B,L,Hkv,d] bf16 CUDA."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, torch.bfloat16, name)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = d ** -0.5 if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device) if lse is None else lse
+    nbytes = sep_attn_fwd_workspace_size(B, L, Hkv, d)
+    ws = _workspace(nbytes, q.device, workspace)
+    mc = mask._c()
+    _check(_lib.sep_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale), mask.a,
+                             mask.n, ctypes.byref(mc), _ptr(o), _ptr(lse), _ptr(ws),
+                             ws.numel(), _stream()), "sep_attn_fwd")
+    return o, lse
+
+
+def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=None, grads=None):
+    """dQ, dK, dV of sum(O * dout) for sep_attn_fwd."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _cuda(t, torch.bfloat16, name)
+    _cuda(lse, torch.float32, "lse")
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = d ** -0.5 if scale is None else scale
+    if grads is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = grads
+    nbytes = sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d)
+    ws = _workspace(nbytes, q.device, workspace)
+    mc = mask._c()
+    _check(_lib.sep_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), B, L, Hq,
+                             Hkv, d, float(scale), mask.a, mask.n, ctypes.byref(mc), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream()), "sep_attn_bwd")
+    return dq, dk, dv
+
+
+class SepCache:
+    """SepCache state for S sequences, held in torch-allocated device memory.
+
+    Capacities: a initial slots, s separator slots, w window slots (c = a + s + w).
+    Methods map one-to-one to sepcache_update / sepcache_decode / sepcache_export_order.
+    """
+
+    def __init__(self, S, Hq, Hkv, d, a, s, w, rope_theta, device="cuda"):
+        self.S, self.Hq, self.Hkv, self.d, self.a, self.s, self.w = S, Hq, Hkv, d, a, s, w
+        self.c = a + s + w
+        self.rope_theta = float(rope_theta)
+        dev = torch.device(device)
+        self.k_slots = torch.zeros(S, Hkv, self.c, d, dtype=torch.bfloat16, device=dev)
+        self.v_slots = torch.zeros(S, Hkv, self.c, d, dtype=torch.bfloat16, device=dev)
+        self.slot_pos = torch.empty(S, self.c, dtype=torch.int32, device=dev)
+        self.slot_sep = torch.empty(S, self.c, dtype=torch.uint8, device=dev)
+        self.meta = torch.empty(S, META, dtype=torch.int32, device=dev)
+        self.rope_cs = torch.empty(self.c, d, dtype=torch.float32, device=dev)
+        self._st = _SepCacheState(S, Hq, Hkv, d, a, s, w, self.rope_theta,
+                                  self.k_slots.data_ptr(), self.v_slots.data_ptr(),
+                                  self.slot_pos.data_ptr(), self.slot_sep.data_ptr(),
+                                  self.meta.data_ptr(), self.rope_cs.data_ptr())
+        _check(_lib.sepcache_state_init(ctypes.byref(self._st), _stream()), "sepcache_state_init")
+
+    def sepcache_update(self, k_new, v_new, sep_new):
+        _cuda(k_new, torch.bfloat16, "k_new")
+        _cuda(v_new, torch.bfloat16, "v_new")
+        _cuda(sep_new, torch.uint8, "sep_new")
+        _check(_lib.sepcache_update(ctypes.byref(self._st), _ptr(k_new), _ptr(v_new),
+                                    _ptr(sep_new), _stream()), "sepcache_update")
+
+    def sepcache_decode(self, q, scale=None, out=None, lse=None):
+        _cuda(q, torch.bfloat16, "q")
+        scale = self.d ** -0.5 if scale is None else scale
+        o = torch.empty_like(q) if out is None else out
+        _check(_lib.sepcache_decode(ctypes.byref(self._st), _ptr(q), _ptr(o), _ptr(lse),
+                                    float(scale), _stream()), "sepcache_decode")
+        return o
+
+    def sepcache_export_order(self):
+        pos = torch.empty(self.S, self.c, dtype=torch.int32, device=self.k_slots.device)
+        cnt = torch.empty(self.S, dtype=torch.int32, device=self.k_slots.device)
+        _check(_lib.sepcache_export_order(ctypes.byref(self._st), _ptr(pos), _ptr(cnt),
+                                          _stream()), "sepcache_export_order")
+        return pos, cnt

@@ -27,6 +27,8 @@ finite differences). No function here is "parity unpinned".
 from .sepattn_ref import (  # noqa: F401
     anchor_flags,
     keep_mask,
+    keep_block,
+    tile_class,
     kept_pairs,
     kept_pairs_closed_form,
     mask_build,

@@ -48,6 +48,24 @@ def keep_mask(sep_row, a, n):
     return (j <= i) & (((i - j) < n) | f[None, :])
 
 
+def keep_block(sep_row, a, n, r0, r1, c0, c1):
+    """Rows r0..r1-1 x columns c0..c1-1 of M_b, from the same rule as keep_mask.
+
+    For long sequences, where the full L x L mask does not fit in memory.
+    """
+    f = anchor_flags(sep_row, a)
+    i = np.arange(r0, r1)[:, None]
+    j = np.arange(c0, c1)[None, :]
+    return (j <= i) & (((i - j) < n) | f[c0:c1][None, :])
+
+
+def tile_class(sep_row, a, n, bm, bn, t, u):
+    """SKIP / PARTIAL / FULL of block (t, u) of M_b (in-bounds pairs only)."""
+    L = len(sep_row)
+    blk = keep_block(sep_row, a, n, t * bm, min(L, (t + 1) * bm), u * bn, min(L, (u + 1) * bn))
+    return SKIP if not blk.any() else (FULL if blk.all() else PARTIAL)
+
+
 def kept_pairs(sep, a, n):
     """Number of kept (query, key) pairs per batch element, counted on the mask."""
     sep = np.atleast_2d(sep)
@@ -201,29 +219,33 @@ def attn_fwd_rows(q, k, v, sep, a, n, scale, b, rows, heads=None):
 
     Second form of the same definition: for each query row i of batch b, gather K(i)
     and run ordinary softmax attention on it. Never builds the L x L mask, so it serves
-    long sequences at sampled rows. Returns O [len(rows), H, d] and LSE [len(rows), H]
+    long sequences at sampled rows (inputs may be float32 or bf16-valued arrays; only the
+    gathered rows are widened to fp64). Returns O [len(rows), H, d] and LSE [len(rows), H]
     for the heads asked for (all query heads by default).
     """
-    q_b = _f64(q[b])
-    k_b = _f64(k[b])
-    v_b = _f64(v[b])
     f = anchor_flags(np.asarray(sep)[b], a)
-    L, Hq, d = q_b.shape
-    Hkv = k_b.shape[1]
+    L, Hq, d = q.shape[1:]
+    Hkv = k.shape[2]
     G = Hq // Hkv
     heads = list(range(Hq)) if heads is None else list(heads)
     O = np.zeros((len(rows), len(heads), d))
     LSE = np.zeros((len(rows), len(heads)))
     for r, i in enumerate(rows):
-        idx = kept_index_set(f, int(i), n)
-        for c, h in enumerate(heads):
-            kh = h // G
-            s = scale * (k_b[idx, kh, :] @ q_b[i, h, :])
-            mx = s.max()
-            e = np.exp(s - mx)
-            l = e.sum()
-            O[r, c, :] = (e / l) @ v_b[idx, kh, :]
-            LSE[r, c] = mx + np.log(l)
+        i = int(i)
+        idx = kept_index_set(f, i, n)
+        qi = _f64(q[b, i])
+        for kh in sorted({h // G for h in heads}):
+            K = _f64(k[b, idx, kh, :])
+            V = _f64(v[b, idx, kh, :])
+            for c, h in enumerate(heads):
+                if h // G != kh:
+                    continue
+                s = scale * (K @ qi[h])
+                mx = s.max()
+                e = np.exp(s - mx)
+                l = e.sum()
+                O[r, c, :] = (e / l) @ V
+                LSE[r, c] = mx + np.log(l)
     return O, LSE
 
 
@@ -237,42 +259,41 @@ def attn_bwd_sampled(q, k, v, do, sep, a, n, scale, b, q_rows, k_rows, kv_heads=
     summed over the query heads of the KV head. P_ij and Delta_i come from each query's own
     gathered forward. Returns dq [len(q_rows), Hq, d], dk/dv [len(k_rows), Hkv', d].
     """
-    q_b = _f64(q[b])
-    k_b = _f64(k[b])
-    v_b = _f64(v[b])
-    do_b = _f64(do[b])
     f = anchor_flags(np.asarray(sep)[b], a)
-    L, Hq, d = q_b.shape
-    Hkv = k_b.shape[1]
+    L, Hq, d = q.shape[1:]
+    Hkv = k.shape[2]
     G = Hq // Hkv
     kv_heads = list(range(Hkv)) if kv_heads is None else list(kv_heads)
 
     row_cache = {}
 
     def row_stats(i):
-        # P row over K(i), and Delta_i, for every query head
+        # P row over K(i), dP row and Delta_i, for every query head
         if i not in row_cache:
             idx = kept_index_set(f, i, n)
             P = np.zeros((Hq, len(idx)))
+            dP = np.zeros((Hq, len(idx)))
             Delta = np.zeros(Hq)
-            for h in range(Hq):
-                kh = h // G
-                s = scale * (k_b[idx, kh, :] @ q_b[i, h, :])
-                e = np.exp(s - s.max())
-                P[h] = e / e.sum()
-                o = P[h] @ v_b[idx, kh, :]
-                Delta[h] = float(do_b[i, h, :] @ o)
-            row_cache[i] = (idx, P, Delta)
+            qi, doi = _f64(q[b, i]), _f64(do[b, i])
+            for kh in range(Hkv):
+                K = _f64(k[b, idx, kh, :])
+                V = _f64(v[b, idx, kh, :])
+                for h in range(kh * G, (kh + 1) * G):
+                    s = scale * (K @ qi[h])
+                    e = np.exp(s - s.max())
+                    P[h] = e / e.sum()
+                    Delta[h] = float(doi[h] @ (P[h] @ V))
+                    dP[h] = V @ doi[h]
+            row_cache[i] = (idx, P, dP, Delta)
         return row_cache[i]
 
     dq = np.zeros((len(q_rows), Hq, d))
     for r, i in enumerate(q_rows):
-        idx, P, Delta = row_stats(int(i))
+        i = int(i)
+        idx, P, dP, Delta = row_stats(i)
         for h in range(Hq):
-            kh = h // G
-            dP = v_b[idx, kh, :] @ do_b[i, h, :]
-            dS = P[h] * (dP - Delta[h])
-            dq[r, h, :] = scale * (dS @ k_b[idx, kh, :])
+            dS = P[h] * (dP[h] - Delta[h])
+            dq[r, h, :] = scale * (dS @ _f64(k[b, idx, h // G, :]))
 
     dk = np.zeros((len(k_rows), len(kv_heads), d))
     dv = np.zeros((len(k_rows), len(kv_heads), d))
@@ -282,14 +303,14 @@ def attn_bwd_sampled(q, k, v, do, sep, a, n, scale, b, q_rows, k_rows, kv_heads=
         if f[j]:
             rows += list(range(j + n, L))
         for i in rows:
-            idx, P, Delta = row_stats(i)
+            idx, P, dP, Delta = row_stats(i)
             pos = int(np.searchsorted(idx, j))
             assert idx[pos] == j
+            qi, doi = _f64(q[b, i]), _f64(do[b, i])
             for c, kh in enumerate(kv_heads):
                 for h in range(kh * G, (kh + 1) * G):
                     p = P[h, pos]
-                    dp = float(do_b[i, h, :] @ v_b[j, kh, :])
-                    ds = p * (dp - Delta[h])
-                    dk[r, c, :] += scale * ds * q_b[i, h, :]
-                    dv[r, c, :] += p * do_b[i, h, :]
+                    ds = p * (dP[h, pos] - Delta[h])
+                    dk[r, c, :] += scale * ds * qi[h]
+                    dv[r, c, :] += p * doi[h]
     return dq, dk, dv

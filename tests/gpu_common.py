@@ -1,0 +1,38 @@
+"""Helpers for the GPU parity tests: tolerances and comparisons against the oracle."""
+
+import numpy as np
+
+# Forward outputs (and decode outputs): max-abs and mean-abs error against fp64.
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+# log-sum-exp (fp32 accumulation of up to ~10^4 terms): absolute error.
+LSE_ABS = 2e-3
+# Gradients: relative L2 error against fp64.
+GRAD_REL_L2 = 1e-2
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def check_out(got, ref, what=""):
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    assert err.max() <= O_MAX_ABS, f"{what}: max-abs {err.max():.3e}"
+    assert err.mean() <= O_MEAN_ABS, f"{what}: mean-abs {err.mean():.3e}"
+
+
+def check_lse(got, ref, what=""):
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite lse"
+    assert err.max() <= LSE_ABS, f"{what}: lse max-abs {err.max():.3e}"
+
+
+def rel_l2(got, ref):
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def check_grad(got, ref, what=""):
+    assert np.isfinite(got).all(), f"{what}: non-finite gradient"
+    r = rel_l2(got, ref)
+    assert r <= GRAD_REL_L2, f"{what}: rel-L2 {r:.3e}"

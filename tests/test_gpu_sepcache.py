@@ -1,0 +1,132 @@
+"""GPU parity of sepcache_update / sepcache_decode against the SepCache oracle.
+
+The retained-position trajectory (logical order of original positions) is compared bit-exactly;
+decode outputs are compared with the fp64 oracle at the forward tolerances.
+"""
+
+import numpy as np
+import pytest
+
+from gpu_common import check_out, f64
+from oracle import sepcache_ref as C
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def S():
+    import torch
+    assert torch.cuda.is_available()
+    from kv_cache_compression_sep_b200 import sepattn
+    return sepattn
+
+
+@pytest.mark.parametrize("Sq,Hq,Hkv,d,a,s,w,steps,p", [
+    (3, 8, 2, 128, 4, 6, 20, 120, 0.2),
+    (2, 4, 4, 64, 0, 3, 7, 60, 0.5),
+    (2, 8, 1, 128, 2, 0, 9, 50, 0.3),     # s = 0: StreamingLLM with shifting
+    (1, 16, 2, 64, 1, 2, 1, 30, 0.6),     # window of one slot
+    (2, 32, 8, 128, 4, 64, 300, 500, 0.1),
+])
+def test_small_every_step(S, Sq, Hq, Hkv, d, a, s, w, steps, p):
+    import torch
+    theta = 500000.0
+    g = torch.Generator().manual_seed(Sq * 1000 + w)
+    cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, theta)
+    sims = [C.SepCacheSim(a, s, w) for _ in range(Sq)]
+    K, V = [], []
+    for t in range(steps):
+        kn = torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16)
+        vn = torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16)
+        qn = torch.randn(Sq, Hq, d, generator=g).to(torch.bfloat16)
+        sn = (torch.rand(Sq, generator=g) < p).to(torch.uint8)
+        K.append(f64(kn))
+        V.append(f64(vn))
+        cache.sepcache_update(kn.cuda(), vn.cuda(), sn.cuda())
+        lse = torch.empty(Sq, Hq, dtype=torch.float32, device="cuda")
+        o = cache.sepcache_decode(qn.cuda(), lse=lse)
+        pos, cnt = cache.sepcache_export_order()
+        pos, cnt = pos.cpu().numpy(), cnt.cpu().numpy()
+        for sq in range(Sq):
+            sims[sq].append(bool(sn[sq]))
+            order = sims[sq].order()
+            assert int(cnt[sq]) == len(order)
+            assert pos[sq, : len(order)].tolist() == order, (t, sq)
+            assert (pos[sq, len(order):] == -1).all()
+            kr = np.stack([K[j][sq] for j in order])
+            vr = np.stack([V[j][sq] for j in order])
+            ro, rl = C.decode_attention(f64(qn[sq]), kr, vr, theta, d ** -0.5)
+            check_out(f64(o[sq]), ro, f"step {t} seq {sq}")
+            assert np.abs(f64(lse[sq]) - rl).max() < 2e-3
+    assert S.sep_last_device_error() == 0
+
+
+def test_sepcache_decode_config_full(S):
+    """64 sequences x 65536 steps, c = 800 = 4 + 64 + 732, theta = 5e5.
+
+    Trajectory: all 64 sequences at steps 0..2047 and every 256th step after, bit-exact.
+    Outputs: 4 sequences at steps 0..1023 and every 64th step to 2047; every 8th sequence at
+    every 1024th step (the retained tokens' K/V regenerated from their chunk seeds).
+    """
+    import torch
+    import workloads
+    cfg = workloads.SEPCACHE_DECODE
+    dev = "cuda"
+    CH = 256
+    cache = S.SepCache(cfg.S, cfg.Hq, cfg.Hkv, cfg.d, cfg.a, cfg.s, cfg.w, cfg.theta)
+    sims = [C.SepCacheSim(cfg.a, cfg.s, cfg.w) for _ in range(cfg.S)]
+    track = [0, 17, 40, 63]
+    early_k, early_v = [], []   # host K/V of every sequence, steps < 2048
+
+    def gather(pairs):
+        """K/V (fp64) of (sequence, original position) pairs, regenerated chunk by chunk."""
+        out = {}
+        by_chunk = {}
+        for sq, j in pairs:
+            by_chunk.setdefault(j // CH, []).append((sq, j))
+        for ci, lst in by_chunk.items():
+            chk = workloads.decode_chunk(cfg, ci * CH, CH, device=dev)
+            st = torch.tensor([j % CH for _, j in lst], device=dev)
+            sq = torch.tensor([q for q, _ in lst], device=dev)
+            kk = f64(chk["k"][st, sq])
+            vv = f64(chk["v"][st, sq])
+            for z, key in enumerate(lst):
+                out[key] = (kk[z], vv[z])
+        return out
+
+    def check(t, o, q, seqs, kv):
+        for sq in seqs:
+            order = sims[sq].order()
+            kr = np.stack([kv[(sq, j)][0] for j in order])
+            vr = np.stack([kv[(sq, j)][1] for j in order])
+            ro, _ = C.decode_attention(q[sq], kr, vr, cfg.theta, cfg.scale)
+            check_out(f64(o[sq]), ro, f"step {t} seq {sq}")
+
+    for t in range(cfg.steps):
+        if t % CH == 0:
+            chunk = workloads.decode_chunk(cfg, t, CH, device=dev)
+            sep_host = chunk["sep"].cpu().numpy()
+        lt = t % CH
+        kn, vn, qn = chunk["k"][lt], chunk["v"][lt], chunk["q"][lt]
+        cache.sepcache_update(kn, vn, chunk["sep"][lt])
+        o = cache.sepcache_decode(qn)
+        for sq in range(cfg.S):
+            sims[sq].append(bool(sep_host[lt, sq]))
+        if t < 2048:
+            early_k.append(f64(kn))
+            early_v.append(f64(vn))
+        if t < 2048 or t % 256 == 0:
+            pos, cnt = cache.sepcache_export_order()
+            pos, cnt = pos.cpu().numpy(), cnt.cpu().numpy()
+            for sq in range(cfg.S):
+                assert pos[sq, : int(cnt[sq])].tolist() == sims[sq].order(), (t, sq)
+        if t < 1024 or (t < 2048 and t % 64 == 0):
+            kv = {(sq, j): (early_k[j][sq], early_v[j][sq])
+                  for sq in track for j in sims[sq].order()}
+            check(t, o, f64(qn), track, kv)
+        if t % 1024 == 1023:
+            seqs = list(range(0, cfg.S, 8))
+            kv = gather([(sq, j) for sq in seqs for j in sims[sq].order()])
+            check(t, o, f64(qn), seqs, kv)
+    torch.cuda.synchronize()
+    assert S.sep_last_device_error() == 0

@@ -122,3 +122,15 @@ def test_gather_split_covers_mask_once(L, a, n, bm, bn, p):
         for i in range(t * bm, min(L, (t + 1) * bm)):
             window_part = [j for j in range(lo_tile * bn, i + 1) if M[i, j]]
             assert sorted(gathered + window_part) == np.nonzero(M[i])[0].tolist()
+
+
+def test_block_form_matches_full_mask():
+    rng = np.random.default_rng(21)
+    L, a, n = 90, 3, 11
+    sep = (rng.random(L) < 0.15).astype(np.uint8)
+    M = R.keep_mask(sep, a, n)
+    np.testing.assert_array_equal(R.keep_block(sep, a, n, 17, 63, 5, 80), M[17:63, 5:80])
+    tm = R.mask_build(sep[None], a, n, 16, 16)["tile_map"][0]
+    for t in range(tm.shape[0]):
+        for u in range(tm.shape[1]):
+            assert R.tile_class(sep, a, n, 16, 16, t, u) == tm[t, u]

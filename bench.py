@@ -1,0 +1,567 @@
+#!/usr/bin/env python
+"""Throughput of the separator-sparse attention hot path on B200; prints one JSON line.
+
+A step is one pass of every hot-path row over one batch of synthetic input:
+  sep_mask_build -> sep_attn_fwd -> sep_attn_bwd on the Pythia-160m training attention shape
+  (B=8, H=12/12, L=2048, d=64, a=4, n=64, Geometric(mean 10) separator segments), then
+  sepcache_update -> sepcache_decode for one new token of 64 SepCache sequences
+  (Hq=32, Hkv=8, d=128, c=800 = 4+64+732, theta=5e5) held at full occupancy.
+Each step is one CUDA-graph replay. The metric is kept-pair attention TFLOP/s: FLOPs are
+counted on kept (query, key) pairs only (4*d per pair forward, 2.5x that backward, 4*d per
+retained slot and query head in decode), summed over the step and divided by its device time.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
+--workload picks a single-row run instead (llama-prefill, long-context, long-context-dense,
+decode) for the other configurations.
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no data-path collective);
+time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "kept-pair attention TFLOP/s fwd/bwd + SepCache decode GB/s, % of B200 roofline"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in self.rows for k in range(4) if r[5 + k] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ---------------------------------------------------------------------------- native arm
+class TrainDecodeStep:
+    """Buffers and one CUDA graph for the default step (training attention + decode)."""
+
+    def __init__(self, S, dev, rank):
+        self.S = S
+        cfg = workloads.PYTHIA160M
+        self.cfg = cfg
+        inp = workloads.attn_inputs(dataclasses.replace(cfg, seed=cfg.seed + 1000 * rank))
+        self.host = {k: inp[k].pin_memory() for k in ("sep", "q", "k", "v", "do")}
+        self.dev = {k: v.to(dev) for k, v in inp.items() if v is not None}
+        d = self.dev
+        self.mask = S.sep_mask_build(d["sep"], cfg.a, cfg.n)
+        self.o, self.lse = S.sep_attn_fwd(d["q"], d["k"], d["v"], self.mask)
+        self.ws_f = torch.empty(S.sep_attn_fwd_workspace_size(cfg.B, cfg.L, cfg.Hkv, cfg.d),
+                                dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(S.sep_attn_bwd_workspace_size(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.d),
+                                dtype=torch.uint8, device=dev)
+        self.grads = tuple(torch.empty_like(d[x]) for x in ("q", "k", "v"))
+        # decode: cache held at full occupancy; a pool of step inputs cycled through
+        dc = workloads.SEPCACHE_DECODE
+        self.dc = dc
+        self.cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, dc.s, dc.w, dc.theta, device=dev)
+        fill = dc.c + 100
+        ch = workloads.decode_chunk(dc, 0, fill, device=dev)
+        for t in range(fill):
+            self.cache.sepcache_update(ch["k"][t], ch["v"][t], ch["sep"][t])
+        self.pool = workloads.decode_chunk(dc, fill, 64, device=dev)
+        self.host_dec = {k: v[0].cpu().pin_memory() for k, v in self.pool.items()}
+        self.step_in = {k: v[0].clone() for k, v in self.pool.items()}
+        self.o_dec = torch.empty_like(self.step_in["q"])
+        torch.cuda.synchronize()
+        kept = int(self.mask.kept.sum())
+        self.kept = kept
+        self.flops_fwd = 4.0 * cfg.d * kept * cfg.Hq
+        self.flops_bwd = 2.5 * self.flops_fwd
+        occ = dc.c
+        self.flops_dec = 4.0 * dc.d * occ * dc.Hq * dc.S
+        # decode bytes: retained K and V rows, the query and output, the new slot written
+        self.bytes_dec = (occ * dc.Hkv * dc.d * 2 * 2 + 2 * dc.Hq * dc.d * 2 + dc.Hkv * dc.d * 2 * 2) * dc.S
+        self.flops = self.flops_fwd + self.flops_bwd + self.flops_dec
+        self.launches = 12  # mask 2, fwd 2, bwd 6, update 1, decode 1
+
+    def run(self):
+        S, d, cfg = self.S, self.dev, self.cfg
+        S.sep_mask_build(d["sep"], cfg.a, cfg.n, out=self.mask)
+        S.sep_attn_fwd(d["q"], d["k"], d["v"], self.mask, out=self.o, lse=self.lse,
+                       workspace=self.ws_f)
+        S.sep_attn_bwd(d["q"], d["k"], d["v"], self.o, self.lse, d["do"], self.mask,
+                       workspace=self.ws_b, grads=self.grads)
+        x = self.step_in
+        self.cache.sepcache_update(x["k"], x["v"], x["sep"])
+        self.cache.sepcache_decode(x["q"], out=self.o_dec)
+
+    def next_inputs(self, i):
+        for k in self.step_in:
+            self.step_in[k].copy_(self.pool[k][i % self.pool[k].shape[0]])
+
+    # one-pass components, for the per-kernel breakdown
+    def components(self):
+        S, d, cfg = self.S, self.dev, self.cfg
+        x = self.step_in
+        return {
+            "mask_build": lambda: S.sep_mask_build(d["sep"], cfg.a, cfg.n, out=self.mask),
+            "fwd_compact": lambda: S.sep_attn_fwd(d["q"], d["k"], d["v"], self.mask, out=self.o,
+                                                  lse=self.lse, workspace=self.ws_f, stage=0),
+            "fwd_kernel": lambda: S.sep_attn_fwd(d["q"], d["k"], d["v"], self.mask, out=self.o,
+                                                 lse=self.lse, workspace=self.ws_f, stage=1),
+            "bwd_prep": lambda: S.sep_attn_bwd(d["q"], d["k"], d["v"], self.o, self.lse, d["do"],
+                                               self.mask, workspace=self.ws_b, grads=self.grads,
+                                               stage=0),
+            "bwd_dq": lambda: S.sep_attn_bwd(d["q"], d["k"], d["v"], self.o, self.lse, d["do"],
+                                             self.mask, workspace=self.ws_b, grads=self.grads,
+                                             stage=1),
+            "bwd_dkdv": lambda: S.sep_attn_bwd(d["q"], d["k"], d["v"], self.o, self.lse, d["do"],
+                                               self.mask, workspace=self.ws_b, grads=self.grads,
+                                               stage=2),
+            "decode_update": lambda: self.cache.sepcache_update(x["k"], x["v"], x["sep"]),
+            "decode_attention": lambda: self.cache.sepcache_decode(x["q"], out=self.o_dec),
+        }
+
+
+def capture(fn, reps=1):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the launch path outside the capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def flush_l2(buf):
+    buf.add_(1)  # writes a buffer larger than L2
+
+
+def time_graph(g, iters, flush):
+    """Average device time of one replay (CUDA events on the replay stream), L2 flushed between."""
+    times = []
+    st = torch.cuda.current_stream()
+    for _ in range(iters):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        g.replay()
+        e1.record(st)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.mean(times)
+
+
+def native(args, rank, world, dev):
+    from kv_cache_compression_sep_b200 import sepattn as S
+    peaks, peak_src = load_peaks()
+    flush = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    step = TrainDecodeStep(S, dev, rank)
+    graph = capture(step.run)
+    assert S.sep_last_device_error() == 0
+
+    for i in range(args.warmup):
+        flush_l2(flush)
+        graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush_l2(flush)
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_ms = float(t.item())
+    value = step.flops * world * args.steps / (max_ms * 1e-3) / 1e12
+    assert S.sep_last_device_error() == 0
+
+    # ---- end to end through the public API: host inputs in pinned memory, copies timed
+    e2e = e2e_run(step, args, dev, world)
+
+    # ---- per-kernel breakdown (each pass alone, CUDA-graph replays of 20 launches)
+    comps = {}
+    for name, fn in step.components().items():
+        g = capture(fn, reps=20)
+        comps[name] = time_graph(g, 5, flush) / 20.0
+        del g
+    # the decode row needs the cache at full occupancy: update/decode advance it, which is fine
+    fwd_tf = step.flops_fwd / (comps["fwd_kernel"] * 1e-3) / 1e12
+    dq_flops = step.flops_fwd * 1.5 / 1.0  # S, dP, dQ products (3 of the 5 backward GEMMs x 2 / 2)
+    comp_out = {
+        "mask_build_us": comps["mask_build"] * 1e3,
+        "fwd": {"us": (comps["fwd_compact"] + comps["fwd_kernel"]) * 1e3,
+                "kernel_us": comps["fwd_kernel"] * 1e3, "tflops": fwd_tf,
+                "frac_bf16_peak": fwd_tf / peaks["bf16_tflops"]},
+        "bwd": {"us": (comps["bwd_prep"] + comps["bwd_dq"] + comps["bwd_dkdv"]) * 1e3,
+                "prep_us": comps["bwd_prep"] * 1e3, "dq_us": comps["bwd_dq"] * 1e3,
+                "dkdv_us": comps["bwd_dkdv"] * 1e3,
+                "tflops": step.flops_bwd / ((comps["bwd_prep"] + comps["bwd_dq"] + comps["bwd_dkdv"]) * 1e-3) / 1e12},
+        "decode": {"update_us": comps["decode_update"] * 1e3,
+                   "attention_us": comps["decode_attention"] * 1e3,
+                   "gbs": step.bytes_dec / (comps["decode_attention"] * 1e-3) / 1e9,
+                   "frac_hbm": step.bytes_dec / (comps["decode_attention"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "kept_pairs": step.kept,
+        "kept_over_dense_causal": step.kept / (step.cfg.B * step.cfg.L * (step.cfg.L + 1) / 2),
+    }
+    comp_out["bwd"]["frac_bf16_peak"] = comp_out["bwd"]["tflops"] / peaks["bf16_tflops"]
+    # dominant kernel of the step by device time
+    shares = {"fwd_kernel": comps["fwd_kernel"], "bwd_dq": comps["bwd_dq"],
+              "bwd_dkdv": comps["bwd_dkdv"], "decode_attention": comps["decode_attention"]}
+    dom = max(shares, key=shares.get)
+    roof = roofline_for(dom, comps, step, peaks, peak_src)
+    del dq_flops
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, separator flags as configured)",
+        "config": {"workload": "pythia160m-train-attention + sepcache-decode step",
+                   "train": {"B": 8, "Hq": 12, "Hkv": 12, "L": 2048, "d": 64, "a": 4, "n": 64,
+                             "flags": "geometric(mean 10) segments"},
+                   "decode": {"S": 64, "Hq": 32, "Hkv": 8, "d": 128, "c": 800, "a": 4, "s": 64,
+                              "w": 732, "theta": 5e5, "occupancy": 800},
+                   "global_batch": 8 * world, "seq_len": 2048, "parallelism": f"dp{world}",
+                   "l2": "flushed between timed steps (256 MiB write)",
+                   "step": "one CUDA graph: mask build, fwd, bwd, cache update, decode"},
+        "roofline": roof,
+        "components": comp_out,
+        "e2e": e2e,
+        "gpu_launches": step.launches * args.steps,
+        "clocks": clk.summary(),
+        "peaks": {"source": peak_src, **peaks},
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+def roofline_for(name, comps, step, peaks, peak_src):
+    ms = comps[name]
+    traffic = load_traffic(name)
+    if name == "decode_attention":
+        ach = step.bytes_dec / (ms * 1e-3) / 1e9
+        return {"kernel": "sepcache_decode_kernel", "bound": "hbm", "achieved": ach,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                "traffic": traffic, "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": step.bytes_dec}
+    flops = {"fwd_kernel": step.flops_fwd, "bwd_dq": 1.5 * step.flops_fwd,
+             "bwd_dkdv": 2.0 * step.flops_fwd}[name]
+    kname = {"fwd_kernel": "sep_attn_fwd_kernel", "bwd_dq": "sep_attn_bwd_dq_kernel",
+             "bwd_dkdv": "sep_attn_bwd_dkv_kernel"}[name]
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"kernel": kname, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
+            "peak_source": peak_src, "algorithmic_flops_per_launch": flops}
+
+
+def load_traffic(name):
+    """DRAM bytes per launch from the committed ncu summary, if one covers this kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return json.load(fh).get(name)
+    return None
+
+
+def e2e_run(step, args, dev, world):
+    """Same step through the public API with host buffers: H2D of the step's inputs, D2H of
+    its results (dQ, dK, dV and the decode output), all inside the timed region."""
+    S = step.S
+    h, d = step.host, step.dev
+    hd = step.host_dec
+    outs = {"dq": torch.empty_like(step.grads[0], device="cpu").pin_memory(),
+            "dk": torch.empty_like(step.grads[1], device="cpu").pin_memory(),
+            "dv": torch.empty_like(step.grads[2], device="cpu").pin_memory(),
+            "o_dec": torch.empty_like(step.o_dec, device="cpu").pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in list(h.values()) + list(hd.values()))
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    n = max(3, min(args.steps, 20))
+
+    def one():
+        for k in h:
+            d[k].copy_(h[k], non_blocking=True)
+        for k in hd:
+            step.step_in[k].copy_(hd[k], non_blocking=True)
+        step.run()
+        outs["dq"].copy_(step.grads[0], non_blocking=True)
+        outs["dk"].copy_(step.grads[1], non_blocking=True)
+        outs["dv"].copy_(step.grads[2], non_blocking=True)
+        outs["o_dec"].copy_(step.o_dec, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(n):
+        one()
+    e1.record(st)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": step.flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n}
+
+
+# ---------------------------------------------------------------------------- oracle arm
+def oracle_sample(H=4, ndec=4):
+    """One bounded sample of the workload on the oracle; returns (kept-pair FLOPs, seconds).
+
+    Sample: forward + backward of query heads 0..H-1 of batch 0 of the Pythia-160m shape (full
+    L=2048 masked oracle) and ndec decode steps of one SepCache sequence at full occupancy.
+    """
+    import numpy as np
+    import oracle
+    cfg = workloads.PYTHIA160M
+    inp = workloads.attn_inputs(cfg)
+    q = inp["q"][:1, :, :H].float().numpy()
+    k = inp["k"][:1, :, :H].float().numpy()
+    v = inp["v"][:1, :, :H].float().numpy()
+    do = inp["do"][:1, :, :H].float().numpy()
+    sep = inp["sep"][:1].numpy()
+    kept = int(oracle.kept_pairs_closed_form(sep, cfg.a, cfg.n)[0])
+    dc = workloads.SEPCACHE_DECODE
+    rng = np.random.default_rng(0)
+    kr = rng.standard_normal((dc.c, dc.Hkv, dc.d))
+    vr = rng.standard_normal((dc.c, dc.Hkv, dc.d))
+    qd = rng.standard_normal((dc.Hq, dc.d))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, sep, cfg.a, cfg.n, cfg.scale)
+    oracle.attn_bwd(q, k, v, do, sep, cfg.a, cfg.n, cfg.scale)
+    for _ in range(ndec):
+        oracle.decode_attention(qd, kr, vr, dc.theta, dc.scale)
+    dt = time.perf_counter() - t0
+    flops = 3.5 * 4.0 * cfg.d * kept * H + ndec * 4.0 * dc.d * dc.c * dc.Hq
+    return flops, dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((x.get("num_threads", 1) for x in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(seconds):
+    flops, dt = 0.0, 0.0
+    n = 0
+    while dt < seconds or n == 0:
+        f, t = oracle_sample()
+        flops += f
+        dt += t
+        n += 1
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": (f"{n} x [fwd+bwd of 4 query heads of batch 0, "
+                                          "Pythia-160m shape, full fp64 masked oracle; 4 decode "
+                                          "steps of one 800-slot SepCache sequence]"),
+            "seconds": dt}
+
+
+def reference(args, rank, world):
+    if rank != 0:
+        return None
+    # sample per step sized so that warm-up + steps stay within a few minutes
+    H = max(1, min(4, 120 // max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(H, 1)
+    flops, dt = 0.0, 0.0
+    for _ in range(args.steps):
+        f, t = oracle_sample(H, 1)
+        flops += f
+        dt += t
+    value = flops / dt / 1e12
+    cores = blas_threads()
+    sample = (f"per step: fwd+bwd of {H} query head(s) of batch 0 (Pythia-160m shape, fp64 "
+              "masked oracle) + 1 decode step of one 800-slot SepCache sequence")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "pythia160m-train-attention + sepcache-decode step (sample)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------- single rows
+def single_row(args, dev):
+    """Other configurations, one row at a time (fwd/bwd TFLOP/s or decode GB/s)."""
+    from kv_cache_compression_sep_b200 import sepattn as S
+    peaks, peak_src = load_peaks()
+    flush = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    out = {"workload": args.workload, "peaks": peaks, "peak_source": peak_src}
+    if args.workload == "decode":
+        step = TrainDecodeStep.__new__(TrainDecodeStep)
+        dc = workloads.SEPCACHE_DECODE
+        cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, dc.s, dc.w, dc.theta, device=dev)
+        pool = workloads.decode_chunk(dc, 0, 1024, device=dev)
+        o = torch.empty_like(pool["q"][0])
+        for t in range(1024):
+            cache.sepcache_update(pool["k"][t], pool["v"][t], pool["sep"][t])
+        x = {k: v[0].clone() for k, v in pool.items()}
+        g = capture(lambda: (cache.sepcache_update(x["k"], x["v"], x["sep"]),
+                             cache.sepcache_decode(x["q"], out=o)), reps=50)
+        ms = time_graph(g, args.steps, flush) / 50
+        occ = dc.c
+        byts = (occ * dc.Hkv * dc.d * 4 + 4 * dc.Hq * dc.d + 4 * dc.Hkv * dc.d) * dc.S
+        out.update({"us_per_step": ms * 1e3, "tokens_per_s": dc.S / (ms * 1e-3),
+                    "gbs_update_plus_decode": byts / (ms * 1e-3) / 1e9})
+        del step
+        return out
+    cfg = {"llama-prefill": workloads.LLAMA3_8B_PREFILL, "long-context": workloads.LONG_CONTEXT,
+           "long-context-dense": workloads.LONG_CONTEXT}[args.workload]
+    n = cfg.L if args.workload == "long-context-dense" else cfg.n
+    inp = workloads.attn_inputs(cfg, with_do=args.workload != "llama-prefill")
+    d = {k: v.to(dev) for k, v in inp.items() if v is not None}
+    mask = S.sep_mask_build(d["sep"], cfg.a, n)
+    o, lse = S.sep_attn_fwd(d["q"], d["k"], d["v"], mask)
+    torch.cuda.synchronize()
+    kept = int(mask.kept.sum())
+    fl = 4.0 * cfg.d * kept * cfg.Hq
+    ws = torch.empty(S.sep_attn_fwd_workspace_size(cfg.B, cfg.L, cfg.Hkv, cfg.d), dtype=torch.uint8, device=dev)
+    g = capture(lambda: S.sep_attn_fwd(d["q"], d["k"], d["v"], mask, out=o, lse=lse, workspace=ws))
+    ms = time_graph(g, args.steps, flush)
+    out.update({"kept_pairs": kept, "kept_over_dense": kept / (cfg.B * cfg.L * (cfg.L + 1) / 2),
+                "fwd_ms": ms, "fwd_tflops": fl / (ms * 1e-3) / 1e12})
+    out["fwd_frac"] = out["fwd_tflops"] / peaks["bf16_tflops"]
+    if d.get("do") is not None:
+        wsb = torch.empty(S.sep_attn_bwd_workspace_size(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.d), dtype=torch.uint8, device=dev)
+        grads = tuple(torch.empty_like(d[x]) for x in ("q", "k", "v"))
+        g = capture(lambda: S.sep_attn_bwd(d["q"], d["k"], d["v"], o, lse, d["do"], mask,
+                                           workspace=wsb, grads=grads))
+        ms = time_graph(g, max(3, args.steps // 2), flush)
+        out.update({"bwd_ms": ms, "bwd_tflops": 2.5 * fl / (ms * 1e-3) / 1e12})
+        out["bwd_frac"] = out["bwd_tflops"] / peaks["bf16_tflops"]
+    assert S.sep_last_device_error() == 0
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="train-decode",
+                    choices=["train-decode", "llama-prefill", "long-context", "long-context-dense",
+                             "decode"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        if args.workload != "train-decode":
+            line = single_row(args, dev)
+        else:
+            line = native(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

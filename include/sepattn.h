@@ -128,6 +128,25 @@ int sep_attn_bwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, const 
                  void* workspace, size_t workspace_bytes, sep_stream_t stream);
 
 /*
+ * Staged forms, for timing one pass at a time: the same arguments as sep_attn_fwd /
+ * sep_attn_bwd plus a stage number. Running the stages 0, 1 (, 2) in order on one stream is
+ * exactly the one-call form; a stage reads what the earlier stages left in `workspace`.
+ *   sep_attn_fwd_stage: 0 = anchor compaction into the workspace, 1 = attention kernel.
+ *   sep_attn_bwd_stage: 0 = anchor compaction, zeroed fp32 anchor partials, Delta;
+ *                       1 = dQ pass; 2 = dK/dV pass and the anchor combine.
+ * Returns SEP_ERR_INVALID_ARG for any other stage number.
+ */
+int sep_attn_fwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const sep_bf16* v,
+                       int B, int L, int Hq, int Hkv, int d, float scale, int a, int n,
+                       const SepMask* mask, sep_bf16* o, float* lse,
+                       void* workspace, size_t workspace_bytes, sep_stream_t stream);
+int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const sep_bf16* v,
+                       const sep_bf16* o, const float* lse, const sep_bf16* dout,
+                       int B, int L, int Hq, int Hkv, int d, float scale, int a, int n,
+                       const SepMask* mask, sep_bf16* dq, sep_bf16* dk, sep_bf16* dv,
+                       void* workspace, size_t workspace_bytes, sep_stream_t stream);
+
+/*
  * SepCache: streaming KV cache of S independent sequences with capacity c = a + s + w slots
  * per sequence: a initial slots, s separator slots (FIFO), w local-window slots (FIFO)
  * ("SepLLM's Architecture: Composing Efficiency", beiduofen.top). Keys are stored without

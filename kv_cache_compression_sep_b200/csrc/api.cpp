@@ -112,9 +112,10 @@ size_t sep_attn_fwd_workspace_size(int B, int L, int Hkv, int d) {
   return fwd_ws(B, L, Hkv, d).total;
 }
 
-int sep_attn_fwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, int B, int L, int Hq,
-                 int Hkv, int d, float scale, int a, int n, const SepMask* mask, sep_bf16* o,
-                 float* lse, void* workspace, size_t workspace_bytes, sep_stream_t stream) {
+static int attn_fwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const sep_bf16* v,
+                         int B, int L, int Hq, int Hkv, int d, float scale, int a, int n,
+                         const SepMask* mask, sep_bf16* o, float* lse, void* workspace,
+                         size_t workspace_bytes, sep_stream_t stream) {
   int st = check_attn_args(q, k, v, B, L, Hq, Hkv, d, a, n, mask);
   if (st != SEP_OK) return st;
   if (!o || !lse) return SEP_ERR_INVALID_ARG;
@@ -126,19 +127,39 @@ int sep_attn_fwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, int B,
   void* kc = ws + w.kc;
   void* vc = ws + w.vc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (stages & 1) {
+    cudaError_t e = sep::launch_compact_anchors(k, v, mask->anchor_idx, mask->anchor_cnt, B, L,
+                                                Hkv, d, kc, vc, s);
+    if (e != cudaSuccess) return SEP_ERR_CUDA;
+  }
+  if (stages & 2) {
+    AttnMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!encode_map(&maps.q, q, B, L, Hq, d) || !encode_map(&maps.k, k, B, L, Hkv, d) ||
+        !encode_map(&maps.v, v, B, L, Hkv, d) || !encode_map(&maps.kc, kc, B, L, Hkv, d) ||
+        !encode_map(&maps.vc, vc, B, L, Hkv, d))
+      return SEP_ERR_CUDA;
+    AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
+    return cuda_status(
+        sep::launch_attn_fwd(maps, sh, mask->sep, mask->gather_end, mask->tile_map, o, lse, s));
+  }
+  return SEP_OK;
+}
 
-  AttnMaps maps;
-  std::memset(&maps, 0, sizeof(maps));
-  if (!encode_map(&maps.q, q, B, L, Hq, d) || !encode_map(&maps.k, k, B, L, Hkv, d) ||
-      !encode_map(&maps.v, v, B, L, Hkv, d) || !encode_map(&maps.kc, kc, B, L, Hkv, d) ||
-      !encode_map(&maps.vc, vc, B, L, Hkv, d))
-    return SEP_ERR_CUDA;
-  cudaError_t e = sep::launch_compact_anchors(k, v, mask->anchor_idx, mask->anchor_cnt, B, L, Hkv,
-                                              d, kc, vc, s);
-  if (e != cudaSuccess) return SEP_ERR_CUDA;
-  AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
-  return cuda_status(
-      sep::launch_attn_fwd(maps, sh, mask->sep, mask->gather_end, mask->tile_map, o, lse, s));
+int sep_attn_fwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, int B, int L, int Hq,
+                 int Hkv, int d, float scale, int a, int n, const SepMask* mask, sep_bf16* o,
+                 float* lse, void* workspace, size_t workspace_bytes, sep_stream_t stream) {
+  return attn_fwd_impl(3, q, k, v, B, L, Hq, Hkv, d, scale, a, n, mask, o, lse, workspace,
+                       workspace_bytes, stream);
+}
+
+int sep_attn_fwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, int B,
+                       int L, int Hq, int Hkv, int d, float scale, int a, int n,
+                       const SepMask* mask, sep_bf16* o, float* lse, void* workspace,
+                       size_t workspace_bytes, sep_stream_t stream) {
+  if (stage != 0 && stage != 1) return SEP_ERR_INVALID_ARG;
+  return attn_fwd_impl(1 << stage, q, k, v, B, L, Hq, Hkv, d, scale, a, n, mask, o, lse,
+                       workspace, workspace_bytes, stream);
 }
 
 size_t sep_attn_bwd_workspace_size(int B, int L, int Hq, int Hkv, int d) {
@@ -146,10 +167,11 @@ size_t sep_attn_bwd_workspace_size(int B, int L, int Hq, int Hkv, int d) {
   return bwd_ws(B, L, Hq, Hkv, d).total;
 }
 
-int sep_attn_bwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, const sep_bf16* o,
-                 const float* lse, const sep_bf16* dout, int B, int L, int Hq, int Hkv, int d,
-                 float scale, int a, int n, const SepMask* mask, sep_bf16* dq, sep_bf16* dk,
-                 sep_bf16* dv, void* workspace, size_t workspace_bytes, sep_stream_t stream) {
+static int attn_bwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const sep_bf16* v,
+                         const sep_bf16* o, const float* lse, const sep_bf16* dout, int B, int L,
+                         int Hq, int Hkv, int d, float scale, int a, int n, const SepMask* mask,
+                         sep_bf16* dq, sep_bf16* dk, sep_bf16* dv, void* workspace,
+                         size_t workspace_bytes, sep_stream_t stream) {
   int st = check_attn_args(q, k, v, B, L, Hq, Hkv, d, a, n, mask);
   if (st != SEP_OK) return st;
   if (!o || !lse || !dout || !dq || !dk || !dv) return SEP_ERR_INVALID_ARG;
@@ -174,7 +196,25 @@ int sep_attn_bwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, const 
   return cuda_status(sep::launch_attn_bwd(
       maps, sh, mask->sep, mask->anchor_idx, mask->anchor_cnt, mask->gather_end, mask->tile_map,
       o, lse, dout, q, k, v, dq, dk, dv, kc, vc, reinterpret_cast<float*>(ws + w.delta),
-      reinterpret_cast<float*>(ws + w.dka), reinterpret_cast<float*>(ws + w.dva), s));
+      reinterpret_cast<float*>(ws + w.dka), reinterpret_cast<float*>(ws + w.dva), stages, s));
+}
+
+int sep_attn_bwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, const sep_bf16* o,
+                 const float* lse, const sep_bf16* dout, int B, int L, int Hq, int Hkv, int d,
+                 float scale, int a, int n, const SepMask* mask, sep_bf16* dq, sep_bf16* dk,
+                 sep_bf16* dv, void* workspace, size_t workspace_bytes, sep_stream_t stream) {
+  return attn_bwd_impl(sep::kBwdAll, q, k, v, o, lse, dout, B, L, Hq, Hkv, d, scale, a, n, mask,
+                       dq, dk, dv, workspace, workspace_bytes, stream);
+}
+
+int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const sep_bf16* v,
+                       const sep_bf16* o, const float* lse, const sep_bf16* dout, int B, int L,
+                       int Hq, int Hkv, int d, float scale, int a, int n, const SepMask* mask,
+                       sep_bf16* dq, sep_bf16* dk, sep_bf16* dv, void* workspace,
+                       size_t workspace_bytes, sep_stream_t stream) {
+  if (stage < 0 || stage > 2) return SEP_ERR_INVALID_ARG;
+  return attn_bwd_impl(1 << stage, q, k, v, o, lse, dout, B, L, Hq, Hkv, d, scale, a, n, mask, dq,
+                       dk, dv, workspace, workspace_bytes, stream);
 }
 
 static int check_cache(const SepCacheState* st) {

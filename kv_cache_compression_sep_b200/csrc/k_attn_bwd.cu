@@ -754,10 +754,12 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
                             const int32_t* gather_end, const int8_t* tile_map, const void* o,
                             const float* lse, const void* dout, const void* q, const void* k,
                             const void* v, void* dq, void* dk, void* dv, void* kc, void* vc,
-                            float* delta, float* dka, float* dva, cudaStream_t stream) {
+                            float* delta, float* dka, float* dva, int stages,
+                            cudaStream_t stream) {
   (void)q;
-  cudaError_t e = launch_compact_anchors(k, v, anchor_idx, anchor_cnt, s.B, s.L, s.Hkv, s.d, kc, vc,
-                                         stream);
+  cudaError_t e = cudaSuccess;
+  if (stages & kBwdPrep) {
+  e = launch_compact_anchors(k, v, anchor_idx, anchor_cnt, s.B, s.L, s.Hkv, s.d, kc, vc, stream);
   if (e != cudaSuccess) return e;
   {
     const int rowvec = s.Hkv * s.d / 4;
@@ -780,6 +782,8 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
                                                    s.L, s.Hq, delta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  }
+  if (!(stages & (kBwdDq | kBwdDkv))) return cudaSuccess;
   BwdParams prm;
   prm.tmQ = maps.q;
   prm.tmK = maps.k;
@@ -816,30 +820,42 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   if (s.d == 128) {
     constexpr size_t smq = dq_smem_bytes<128>(), smkv = dkv_smem_bytes<128>();
     static_assert(smq <= 227 * 1024 && smkv <= 227 * 1024, "shared memory budget");
-    if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<128>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
-      return e;
-    if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<128>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
-      return e;
-    sep_attn_bwd_dq_kernel<128><<<grid_q, 192, smq, stream>>>(prm);
+    static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<128>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
+        return e;
+      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<128>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
+        return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    if (stages & kBwdDq) sep_attn_bwd_dq_kernel<128><<<grid_q, 192, smq, stream>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    sep_attn_bwd_dkv_kernel<128><<<grid_kv, 192, smkv, stream>>>(prm, nseg);
+    if (stages & kBwdDkv) sep_attn_bwd_dkv_kernel<128><<<grid_kv, 192, smkv, stream>>>(prm, nseg);
   } else {
     constexpr size_t smq = dq_smem_bytes<64>(), smkv = dkv_smem_bytes<64>();
     static_assert(smq <= 227 * 1024 && smkv <= 227 * 1024, "shared memory budget");
-    if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<64>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
-      return e;
-    if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<64>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
-      return e;
-    sep_attn_bwd_dq_kernel<64><<<grid_q, 192, smq, stream>>>(prm);
+    static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<64>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
+        return e;
+      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<64>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
+        return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    if (stages & kBwdDq) sep_attn_bwd_dq_kernel<64><<<grid_q, 192, smq, stream>>>(prm);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    sep_attn_bwd_dkv_kernel<64><<<grid_kv, 192, smkv, stream>>>(prm, nseg);
+    if (stages & kBwdDkv) sep_attn_bwd_dkv_kernel<64><<<grid_kv, 192, smkv, stream>>>(prm, nseg);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {
+  if (stages & kBwdDkv) {
     dim3 grid((s.L + 31) / 32, s.B);
     anchor_combine_kernel<<<grid, 256, 0, stream>>>(anchor_idx, anchor_cnt, s.L, s.Hkv * s.d, 32,
                                                     dka, dva, static_cast<__nv_bfloat16*>(dk),

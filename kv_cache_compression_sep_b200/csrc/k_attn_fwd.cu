@@ -422,9 +422,16 @@ template <int D>
 static cudaError_t launch_fwd_t(const FwdParams& prm, int T, int Hq, int B, cudaStream_t stream) {
   constexpr size_t smem = fwd_smem_bytes<D>();
   static_assert(smem <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(sep_attn_fwd_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(sep_attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   sep_attn_fwd_kernel<D><<<dim3(T, Hq, B), 192, smem, stream>>>(prm);
   return cudaGetLastError();
 }

@@ -213,31 +213,40 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
     for (int e = 0; e < 2 * HP; ++e) acc[g][e] = 0.f;
   }
 
-  // this half-warp's ranks: r0 + hw, r0 + hw + 16, ...; cos/sin by recurrence with step 16
+  // this half-warp's ranks: r0 + hw, r0 + hw + 16, ...; cos/sin by recurrence with step 16.
+  // Both half-warps of a warp run the same number of iterations (that of the even half-warp,
+  // which has at least as many ranks) so that every shuffle has all 32 lanes; an iteration
+  // past the half-warp's last rank loads nothing and leaves the softmax state unchanged.
   int r = r0 + hw;
+  const int n_even = r1 - r0 - (hw & ~1);
+  const int trips = n_even > 0 ? (n_even + kHalfWarps - 1) / kHalfWarps : 0;
   float cr[HP], sr[HP], cd[HP], sd[HP];
-  if (r < r1) {
 #pragma unroll
-    for (int e = 0; e < HP; ++e) {
-      const int k = lane16 * HP + e;
-      const float2 v0 = rope_cs[(size_t)r * HALF + k];
-      cr[e] = v0.x;
-      sr[e] = v0.y;
-      const float2 st = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
-      cd[e] = st.x;
-      sd[e] = st.y;
-    }
+  for (int e = 0; e < HP; ++e) {
+    const int k = lane16 * HP + e;
+    const float2 v0 = (r < r1) ? rope_cs[(size_t)r * HALF + k] : make_float2(1.f, 0.f);
+    cr[e] = v0.x;
+    sr[e] = v0.y;
+    const float2 st = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
+    cd[e] = st.x;
+    sd[e] = st.y;
   }
   const size_t row_base = ((size_t)seq * Hkv + kvh) * c;
-  for (; r < r1; r += kHalfWarps) {
-    const int slot = rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w);
-    const __nv_bfloat16* kr = k_slots + (row_base + slot) * D + lane16 * HP;
-    const __nv_bfloat16* vr = v_slots + (row_base + slot) * D + lane16 * HP;
+  for (int it = 0; it < trips; ++it, r += kHalfWarps) {
+    const bool valid = r < r1;
     float k1[HP], k2[HP], v1[HP], v2[HP];
-    load_bf16_vec<HP>(kr, k1);
-    load_bf16_vec<HP>(kr + HALF, k2);
-    load_bf16_vec<HP>(vr, v1);
-    load_bf16_vec<HP>(vr + HALF, v2);
+    if (valid) {
+      const int slot = rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w);
+      const __nv_bfloat16* kr = k_slots + (row_base + slot) * D + lane16 * HP;
+      const __nv_bfloat16* vr = v_slots + (row_base + slot) * D + lane16 * HP;
+      load_bf16_vec<HP>(kr, k1);
+      load_bf16_vec<HP>(kr + HALF, k2);
+      load_bf16_vec<HP>(vr, v1);
+      load_bf16_vec<HP>(vr + HALF, v2);
+    } else {
+#pragma unroll
+      for (int e = 0; e < HP; ++e) k1[e] = k2[e] = v1[e] = v2[e] = 0.f;
+    }
     // rotate the key by RoPE(r) and dot with every query head
     float part[G];
 #pragma unroll
@@ -257,12 +266,13 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
       cr[e] = cn;
       sr[e] = sn;
     }
-    // reduce over the 16 lanes of the half-warp
+    // reduce over the 16 lanes of the half-warp (all 32 lanes take part)
 #pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
     }
+    if (!valid) continue;
     // online softmax per head (lazy rescale: only when the max grows by more than 2^8)
 #pragma unroll
     for (int g = 0; g < G; ++g) {

@@ -18,6 +18,9 @@ cudaError_t launch_mask_build(const uint8_t* sep, int B, int L, int a, int n, in
                               int32_t* anchor_idx, int32_t* anchor_cnt, int32_t* gather_end,
                               int8_t* tile_map, int64_t* kept, cudaStream_t stream);
 
+// Stage bits of launch_attn_bwd.
+constexpr int kBwdPrep = 1, kBwdDq = 2, kBwdDkv = 4, kBwdAll = 7;
+
 // Copies the K/V rows of every anchor to rows 0..anchor_cnt[b]-1 of kc/vc ([B, L, Hkv, d]).
 cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* anchor_idx,
                                    const int32_t* anchor_cnt, int B, int L, int Hkv, int d,
@@ -42,7 +45,8 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
                             const int32_t* gather_end, const int8_t* tile_map, const void* o,
                             const float* lse, const void* dout, const void* q, const void* k,
                             const void* v, void* dq, void* dk, void* dv, void* kc, void* vc,
-                            float* delta, float* dka, float* dva, cudaStream_t stream);
+                            float* delta, float* dka, float* dva, int stages,
+                            cudaStream_t stream);
 
 cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream);
 cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new,

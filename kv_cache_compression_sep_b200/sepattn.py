@@ -35,7 +35,9 @@ def _load():
         "sep_mask_build": (I, [P, I, I, I, I, I, I, P, P, P, P, P, P]),
         "sep_attn_fwd_workspace_size": (Z, [I, I, I, I]),
         "sep_attn_fwd": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
+        "sep_attn_fwd_stage": (I, [I, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
         "sep_attn_bwd_workspace_size": (Z, [I, I, I, I, I]),
+        "sep_attn_bwd_stage": (I, [I, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, P, Z, P]),
         "sep_attn_bwd": (I, [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, P, Z, P]),
         "sepcache_state_init": (I, [P, P]),
         "sepcache_update": (I, [P, P, P, P, P]),
@@ -111,17 +113,22 @@ class SepMask:
                         self.tile_map.data_ptr())
 
 
-def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = TILE) -> SepMask:
+def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = TILE,
+                   out: SepMask | None = None) -> SepMask:
+    """Mask artefacts of `sep` [B, L] uint8; `out` reuses the buffers of an earlier result."""
     _cuda(sep, torch.uint8, "sep")
     B, L = sep.shape
     T, U = -(-L // bm), -(-L // bn)
     dev = sep.device
-    out = SepMask(sep=sep,
-                  anchor_idx=torch.empty(B, L, dtype=torch.int32, device=dev),
-                  anchor_cnt=torch.empty(B, dtype=torch.int32, device=dev),
-                  gather_end=torch.empty(B, T, dtype=torch.int32, device=dev),
-                  tile_map=torch.empty(B, T, U, dtype=torch.int8, device=dev),
-                  kept=torch.empty(B, dtype=torch.int64, device=dev), a=a, n=n)
+    if out is not None:
+        out.sep, out.a, out.n = sep, a, n
+    else:
+        out = SepMask(sep=sep,
+                      anchor_idx=torch.empty(B, L, dtype=torch.int32, device=dev),
+                      anchor_cnt=torch.empty(B, dtype=torch.int32, device=dev),
+                      gather_end=torch.empty(B, T, dtype=torch.int32, device=dev),
+                      tile_map=torch.empty(B, T, U, dtype=torch.int8, device=dev),
+                      kept=torch.empty(B, dtype=torch.int64, device=dev), a=a, n=n)
     _check(_lib.sep_mask_build(_ptr(sep), B, L, a, n, bm, bn, _ptr(out.anchor_idx),
                                _ptr(out.anchor_cnt), _ptr(out.gather_end), _ptr(out.tile_map),
                                _ptr(out.kept), _stream()), "sep_mask_build")
@@ -142,8 +149,12 @@ def _workspace(nbytes, device, ws):
     return ws
 
 
-def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspace=None):
-    """O, LSE of separator-sparse attention. q [B,L,Hq,d], k/v [B,L,Hkv,d] bf16 CUDA."""
+def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspace=None,
+                 stage=None):
+    """O, LSE of separator-sparse attention. q [B,L,Hq,d], k/v [B,L,Hkv,d] bf16 CUDA.
+
+    stage=None runs the whole call; stage=0/1 runs sep_attn_fwd_stage (timing one pass).
+    """
     for name, t in (("q", q), ("k", k), ("v", v)):
         _cuda(t, torch.bfloat16, name)
     B, L, Hq, d = q.shape
@@ -154,14 +165,21 @@ def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspa
     nbytes = sep_attn_fwd_workspace_size(B, L, Hkv, d)
     ws = _workspace(nbytes, q.device, workspace)
     mc = mask._c()
-    _check(_lib.sep_attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale), mask.a,
-                             mask.n, ctypes.byref(mc), _ptr(o), _ptr(lse), _ptr(ws),
-                             ws.numel(), _stream()), "sep_attn_fwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale), mask.a, mask.n,
+            ctypes.byref(mc), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream())
+    if stage is None:
+        _check(_lib.sep_attn_fwd(*args), "sep_attn_fwd")
+    else:
+        _check(_lib.sep_attn_fwd_stage(int(stage), *args), "sep_attn_fwd_stage")
     return o, lse
 
 
-def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=None, grads=None):
-    """dQ, dK, dV of sum(O * dout) for sep_attn_fwd."""
+def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=None, grads=None,
+                 stage=None):
+    """dQ, dK, dV of sum(O * dout) for sep_attn_fwd.
+
+    stage=None runs the whole call; stage=0/1/2 runs sep_attn_bwd_stage (timing one pass).
+    """
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
         _cuda(t, torch.bfloat16, name)
     _cuda(lse, torch.float32, "lse")
@@ -175,9 +193,13 @@ def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=Non
     nbytes = sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d)
     ws = _workspace(nbytes, q.device, workspace)
     mc = mask._c()
-    _check(_lib.sep_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), B, L, Hq,
-                             Hkv, d, float(scale), mask.a, mask.n, ctypes.byref(mc), _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(), _stream()), "sep_attn_bwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), B, L, Hq, Hkv, d,
+            float(scale), mask.a, mask.n, ctypes.byref(mc), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(ws), ws.numel(), _stream())
+    if stage is None:
+        _check(_lib.sep_attn_bwd(*args), "sep_attn_bwd")
+    else:
+        _check(_lib.sep_attn_bwd_stage(int(stage), *args), "sep_attn_bwd_stage")
     return dq, dk, dv
 
 

@@ -236,12 +236,14 @@ def native(args, rank, world, dev):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     with ClockSampler(dev.index) as clk:
+        torch.cuda.nvtx.range_push("timed")
         for i in range(args.steps):
             flush_l2(flush)
             ev[i][0].record(stream)
             graph.replay()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -254,6 +256,9 @@ def native(args, rank, world, dev):
     value = step.flops * world * args.steps / (max_ms * 1e-3) / 1e12
     assert S.sep_last_device_error() == 0
 
+    if args.quick:  # timed step only (used under ncu)
+        return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "ms_per_step": max_ms / args.steps, "quick": True}
     # ---- end to end through the public API: host inputs in pinned memory, copies timed
     e2e = e2e_run(step, args, dev, world)
 
@@ -534,6 +539,8 @@ def main():
                              "decode"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true",
+                    help="timed step only: no e2e, breakdown or CPU baseline (for ncu runs)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

@@ -49,31 +49,34 @@ __global__ void __launch_bounds__(256) zero_anchor_partials_kernel(
   }
 }
 
-// Delta[b][h][i] = sum_c dO[b,i,h,c] * O[b,i,h,c]; one warp per (b, i, h) row.
+// Delta[b][h][i] = sum_c dO[b,i,h,c] * O[b,i,h,c]; one thread per (b, i, h) row, 16-byte loads.
 template <int D>
 __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
                                                     const __nv_bfloat16* __restrict__ dout,
                                                     int B, int L, int Hq, float* __restrict__ delta) {
-  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= (long long)B * L * Hq) return;
-  const int h = (int)(row % Hq);
-  const long long bi = row / Hq;
-  const int i = (int)(bi % L), b = (int)(bi / L);
-  constexpr int EPL = D / 32;
-  const __nv_bfloat16* po = o + row * D + lane * EPL;
-  const __nv_bfloat16* pd = dout + row * D + lane * EPL;
+  // consecutive threads take consecutive positions i of one (b, h): coalesced Delta stores
+  const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (long long)B * L * Hq) return;
+  const int i = (int)(id % L);
+  const long long bh = id / L;
+  const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+  const long long row = ((long long)b * L + i) * Hq + h;
+  const uint4* po = reinterpret_cast<const uint4*>(o + row * D);
+  const uint4* pd = reinterpret_cast<const uint4*>(dout + row * D);
   float acc = 0.f;
 #pragma unroll
-  for (int e = 0; e < EPL; e += 2) {
-    const __nv_bfloat162 a2 = *reinterpret_cast<const __nv_bfloat162*>(po + e);
-    const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(pd + e);
-    acc = fmaf(__low2float(a2), __low2float(b2), acc);
-    acc = fmaf(__high2float(a2), __high2float(b2), acc);
-  }
+  for (int q = 0; q < D / 8; ++q) {
+    const uint4 x = __ldg(po + q), y = __ldg(pd + q);
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) delta[((size_t)b * Hq + h) * L + i] = acc;
+    for (int z = 0; z < 4; ++z) {
+      const __nv_bfloat162 a2 = *reinterpret_cast<const __nv_bfloat162*>(&xs[z]);
+      const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&ys[z]);
+      acc = fmaf(__low2float(a2), __low2float(b2), acc);
+      acc = fmaf(__high2float(a2), __high2float(b2), acc);
+    }
+  }
+  delta[((size_t)b * Hq + h) * L + i] = acc;
 }
 
 // ------------------------------------------------------------------ shared parameter block
@@ -771,7 +774,7 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   }
   {
     const long long rows = (long long)s.B * s.L * s.Hq;
-    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    const unsigned blocks = (unsigned)((rows + 255) / 256);
     if (s.d == 128)
       delta_kernel<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                     static_cast<const __nv_bfloat16*>(dout), s.B,

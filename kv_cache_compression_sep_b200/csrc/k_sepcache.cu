@@ -159,23 +159,58 @@ __device__ __forceinline__ void load_bf16_vec(const __nv_bfloat16* p, float (&ou
   }
 }
 
+// N consecutive bf16 from shared memory (4- or 8-byte aligned) to fp32.
+template <int N>
+__device__ __forceinline__ void load_bf16_vec_smem(const __nv_bfloat16* p, float (&out)[N]) {
+  if constexpr (N == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    out[0] = __low2float(x); out[1] = __high2float(x);
+    out[2] = __low2float(y); out[3] = __high2float(y);
+  } else {
+    static_assert(N == 2, "two or four elements per lane");
+    const uint32_t u = *reinterpret_cast<const unsigned int*>(p);
+    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u);
+    out[0] = __low2float(x); out[1] = __high2float(x);
+  }
+}
+
 // ------------------------------------------------------------------ decode
-// EPL = elements of a key row per lane (d / 16): the lane owns EPL/2 rotation pairs
-// (k, k + d/2), k = lane16 * EPL/2 + e.
+// Streaming: bulk copies bring the K and V rows of kChunk consecutive ranks (as few contiguous
+// slot segments as the rings allow) into a kStages-deep shared-memory ring. Thread 0 fills the
+// first stages; afterwards the last warp to finish reading a stage refills it with the chunk
+// kStages further on, so no thread waits to issue. Half-warp hw handles ranks r0 + hw + 16k;
+// lane16 owns HP rotation pairs (k, k + d/2), k = lane16 * HP + e, of every row it reads.
+constexpr int kChunk = 32;
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = kDecThreads / 32;
+
+template <int D>
+struct DecSmem {
+  alignas(128) __nv_bfloat16 k[kStages][kChunk][D];
+  alignas(128) __nv_bfloat16 v[kStages][kChunk][D];
+  uint64_t full[kStages];
+  int done[kStages];  // warps finished with the stage's current chunk
+  int abort_flag;
+};
+
 template <int D, int G>
-__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
+__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 2)
     sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int w,
                            const __nv_bfloat16* __restrict__ k_slots,
                            const __nv_bfloat16* __restrict__ v_slots,
                            const int32_t* __restrict__ meta, const float2* __restrict__ rope_cs,
                            const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ o,
-                           float* __restrict__ lse, float scale_log2) {
+                           float* __restrict__ lse, float scale_log2, unsigned* err) {
   constexpr int HP = D / 32;       // rotation pairs per lane
   constexpr int HALF = D / 2;
   const int split = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
   const int c = a + s + w;
-  const int tid = threadIdx.x, lane16 = tid & 15, hw = tid >> 4;
+  const int tid = threadIdx.x, lane16 = tid & 15, hw = tid >> 4, warp = tid >> 5;
   cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(128) uint8_t dsm_raw[];
+  DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
 
   const int32_t* m = meta + (size_t)seq * SEPCACHE_META;
   const int ninit = m[SEPCACHE_META_NINIT];
@@ -183,27 +218,42 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
   const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
   const int occ = ninit + sep_cnt + win_cnt;
   const int mq = occ - 1;  // the query's own rank
-  const int chunk = (occ + kSplit - 1) / kSplit;
-  const int r0 = split * chunk, r1 = min(occ, r0 + chunk);
+  const int per = (occ + kSplit - 1) / kSplit;
+  const int r0 = split * per, r1 = min(occ, r0 + per);
+  const int nchunks = r1 > r0 ? (r1 - r0 + kChunk - 1) / kChunk : 0;
+  const size_t row_base = ((size_t)seq * Hkv + kvh) * c;
+  volatile int* abort_flag = &sm.abort_flag;
 
-  // query heads of this KV head, rotated by RoPE(mq) and scaled by scale*log2(e)
-  float qr[G][2 * HP];
-  {
-    const float2* cs = rope_cs + (size_t)max(mq, 0) * HALF;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const __nv_bfloat16* qh = q + ((size_t)seq * Hq + kvh * G + g) * D;
-#pragma unroll
-      for (int e = 0; e < HP; ++e) {
-        const int k = lane16 * HP + e;
-        const float x1 = __bfloat162float(qh[k]), x2 = __bfloat162float(qh[k + HALF]);
-        const float2 r = cs[k];
-        qr[g][e] = (x1 * r.x - x2 * r.y) * scale_log2;
-        qr[g][HP + e] = (x2 * r.x + x1 * r.y) * scale_log2;
-      }
+  auto issue_chunk = [&](int ch) {  // one thread: bulk copies of chunk ch into its stage
+    const int st = ch % kStages;
+    const int c0 = r0 + ch * kChunk;
+    const int rows = min(kChunk, r1 - c0);
+    mbar_arrive_expect_tx(&sm.full[st], (uint32_t)(rows * D * 2 * 2));
+    int r = c0;
+    while (r < c0 + rows) {
+      const int slot = rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w);
+      int len = 1;  // extend while the next rank sits in the next slot
+      while (r + len < c0 + rows &&
+             rank_to_slot(r + len, ninit, sep_head, sep_cnt, win_head, a, s, w) == slot + len)
+        ++len;
+      const size_t src = (row_base + slot) * D;
+      bulk_load(&sm.k[st][r - c0][0], k_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
+      bulk_load(&sm.v[st][r - c0][0], v_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
+      r += len;
     }
+  };
+  if (tid == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&sm.full[st], 1);
+      sm.done[st] = 0;
+    }
+    sm.abort_flag = 0;
+    fence_barrier_init();
+    for (int ch = 0; ch < min(kStages, nchunks); ++ch) issue_chunk(ch);
   }
+  __syncthreads();
 
+  // per-head softmax state (consumers)
   float mrun[G], lrun[G], acc[G][2 * HP];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -213,84 +263,124 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
     for (int e = 0; e < 2 * HP; ++e) acc[g][e] = 0.f;
   }
 
-  // this half-warp's ranks: r0 + hw, r0 + hw + 16, ...; cos/sin by recurrence with step 16.
-  // Both half-warps of a warp run the same number of iterations (that of the even half-warp,
-  // which has at least as many ranks) so that every shuffle has all 32 lanes; an iteration
-  // past the half-warp's last rank loads nothing and leaves the softmax state unchanged.
-  int r = r0 + hw;
-  const int n_even = r1 - r0 - (hw & ~1);
-  const int trips = n_even > 0 ? (n_even + kHalfWarps - 1) / kHalfWarps : 0;
-  float cr[HP], sr[HP], cd[HP], sd[HP];
+  {
+    // ---------------------------------------------------------------- consumers
+    // query heads of this KV head, rotated by RoPE(mq) and scaled by scale*log2(e)
+    float qr[G][2 * HP];
+    {
+      const float2* cs = rope_cs + (size_t)max(mq, 0) * HALF;
 #pragma unroll
-  for (int e = 0; e < HP; ++e) {
-    const int k = lane16 * HP + e;
-    const float2 v0 = (r < r1) ? rope_cs[(size_t)r * HALF + k] : make_float2(1.f, 0.f);
-    cr[e] = v0.x;
-    sr[e] = v0.y;
-    const float2 st = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
-    cd[e] = st.x;
-    sd[e] = st.y;
-  }
-  const size_t row_base = ((size_t)seq * Hkv + kvh) * c;
-  for (int it = 0; it < trips; ++it, r += kHalfWarps) {
-    const bool valid = r < r1;
-    float k1[HP], k2[HP], v1[HP], v2[HP];
-    if (valid) {
-      const int slot = rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w);
-      const __nv_bfloat16* kr = k_slots + (row_base + slot) * D + lane16 * HP;
-      const __nv_bfloat16* vr = v_slots + (row_base + slot) * D + lane16 * HP;
-      load_bf16_vec<HP>(kr, k1);
-      load_bf16_vec<HP>(kr + HALF, k2);
-      load_bf16_vec<HP>(vr, v1);
-      load_bf16_vec<HP>(vr + HALF, v2);
-    } else {
+      for (int g = 0; g < G; ++g) {
+        const __nv_bfloat16* qh = q + ((size_t)seq * Hq + kvh * G + g) * D;
 #pragma unroll
-      for (int e = 0; e < HP; ++e) k1[e] = k2[e] = v1[e] = v2[e] = 0.f;
-    }
-    // rotate the key by RoPE(r) and dot with every query head
-    float part[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) part[g] = 0.f;
-#pragma unroll
-    for (int e = 0; e < HP; ++e) {
-      const float y1 = k1[e] * cr[e] - k2[e] * sr[e];
-      const float y2 = k2[e] * cr[e] + k1[e] * sr[e];
-#pragma unroll
-      for (int g = 0; g < G; ++g) part[g] = fmaf(qr[g][e], y1, fmaf(qr[g][HP + e], y2, part[g]));
-    }
-    // advance cos/sin by kHalfWarps positions
-#pragma unroll
-    for (int e = 0; e < HP; ++e) {
-      const float cn = cr[e] * cd[e] - sr[e] * sd[e];
-      const float sn = sr[e] * cd[e] + cr[e] * sd[e];
-      cr[e] = cn;
-      sr[e] = sn;
-    }
-    // reduce over the 16 lanes of the half-warp (all 32 lanes take part)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-      for (int off = 8; off > 0; off >>= 1) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
-    }
-    if (!valid) continue;
-    // online softmax per head (lazy rescale: only when the max grows by more than 2^8)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float sc = part[g];
-      if (sc > mrun[g] + 8.0f) {
-        const float alpha = ex2(mrun[g] - sc);
-        lrun[g] *= alpha;
-#pragma unroll
-        for (int e = 0; e < 2 * HP; ++e) acc[g][e] *= alpha;
-        mrun[g] = sc;
+        for (int e = 0; e < HP; ++e) {
+          const int k = lane16 * HP + e;
+          const float x1 = __bfloat162float(qh[k]), x2 = __bfloat162float(qh[k + HALF]);
+          const float2 rr = cs[k];
+          qr[g][e] = (x1 * rr.x - x2 * rr.y) * scale_log2;
+          qr[g][HP + e] = (x2 * rr.x + x1 * rr.y) * scale_log2;
+        }
       }
-      const float pg = ex2(sc - mrun[g]);
-      lrun[g] += pg;
+    }
+    // cos/sin of this half-warp's current rank, advanced by kHalfWarps per step
+    float cr[HP], sr[HP], cd[HP], sd[HP];
+    {
+      const int rf = r0 + hw;
 #pragma unroll
       for (int e = 0; e < HP; ++e) {
-        acc[g][e] = fmaf(pg, v1[e], acc[g][e]);
-        acc[g][HP + e] = fmaf(pg, v2[e], acc[g][HP + e]);
+        const int k = lane16 * HP + e;
+        const float2 v0 = (rf < r1) ? rope_cs[(size_t)rf * HALF + k] : make_float2(1.f, 0.f);
+        cr[e] = v0.x;
+        sr[e] = v0.y;
+        const float2 stp = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
+        cd[e] = stp.x;
+        sd[e] = stp.y;
       }
+    }
+    bool ok = true;
+    for (int ch = 0; ch < nchunks && ok; ++ch) {
+      const int st = ch % kStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[st], (ch / kStages) & 1, err, abort_flag))) {
+        ok = false;
+        break;
+      }
+      const int c0 = r0 + ch * kChunk;
+#pragma unroll
+      for (int sub = 0; sub < kChunk / kHalfWarps; ++sub) {
+        const int row = sub * kHalfWarps + hw;
+        const bool valid = c0 + row < r1;
+        float k1[HP], k2[HP], v1[HP], v2[HP];
+        const __nv_bfloat16* kr = &sm.k[st][row][lane16 * HP];
+        const __nv_bfloat16* vr = &sm.v[st][row][lane16 * HP];
+        if (valid) {
+          load_bf16_vec_smem<HP>(kr, k1);
+          load_bf16_vec_smem<HP>(kr + HALF, k2);
+          load_bf16_vec_smem<HP>(vr, v1);
+          load_bf16_vec_smem<HP>(vr + HALF, v2);
+        } else {
+#pragma unroll
+          for (int e = 0; e < HP; ++e) k1[e] = k2[e] = v1[e] = v2[e] = 0.f;
+        }
+        float part[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) part[g] = 0.f;
+#pragma unroll
+        for (int e = 0; e < HP; ++e) {
+          const float y1 = k1[e] * cr[e] - k2[e] * sr[e];
+          const float y2 = k2[e] * cr[e] + k1[e] * sr[e];
+#pragma unroll
+          for (int g = 0; g < G; ++g) part[g] = fmaf(qr[g][e], y1, fmaf(qr[g][HP + e], y2, part[g]));
+        }
+#pragma unroll
+        for (int e = 0; e < HP; ++e) {
+          const float cn = cr[e] * cd[e] - sr[e] * sd[e];
+          const float sn = sr[e] * cd[e] + cr[e] * sd[e];
+          cr[e] = cn;
+          sr[e] = sn;
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
+        }
+        if (valid) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float sc = part[g];
+            if (sc > mrun[g] + 8.0f) {
+              const float alpha = ex2(mrun[g] - sc);
+              lrun[g] *= alpha;
+#pragma unroll
+              for (int e = 0; e < 2 * HP; ++e) acc[g][e] *= alpha;
+              mrun[g] = sc;
+            }
+            const float pg = ex2(sc - mrun[g]);
+            lrun[g] += pg;
+#pragma unroll
+            for (int e = 0; e < HP; ++e) {
+              acc[g][e] = fmaf(pg, v1[e], acc[g][e]);
+              acc[g][HP + e] = fmaf(pg, v2[e], acc[g][HP + e]);
+            }
+          }
+        }
+      }
+      // the last warp done with this stage refills it (its reads all precede the atomic)
+      __syncwarp();
+      if ((tid & 31) == 0) {
+        if (atomicAdd(&sm.done[st], 1) == kConsumerWarps - 1) {
+          sm.done[st] = 0;
+          if (ch + kStages < nchunks) {
+            fence_proxy_async_smem();
+            issue_chunk(ch + kStages);
+          }
+        }
+      }
+    }
+    if (!ok) {
+      // a wait ran out: let every copy still in flight land before the CTA leaves
+      if (tid == 0)
+        for (int ch = 0; ch < nchunks; ++ch)
+          mbar_wait(&sm.full[ch % kStages], (ch / kStages) & 1, nullptr, nullptr);
     }
   }
 
@@ -310,12 +400,10 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
     lrun[g] = lrun[g] * fs + lo * fo;
     mrun[g] = M;
   }
-  // ---- combine the warps of this CTA through shared memory
-  constexpr int kWarps = kDecThreads / 32;
-  __shared__ float s_m[kWarps][G], s_l[kWarps][G];
-  __shared__ float s_acc[kWarps][G][D];
+  // ---- combine the consumer warps of this CTA through shared memory
+  __shared__ float s_m[kConsumerWarps][G], s_l[kConsumerWarps][G];
+  __shared__ float s_acc[kConsumerWarps][G][D];
   __shared__ float s_res[G][D + 2];  // this CTA's combined (acc..., m, l) per head
-  const int warp = tid >> 5;
   if ((tid & 31) < 16) {
     if (lane16 == 0) {
 #pragma unroll
@@ -334,13 +422,13 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
     }
   }
   __syncthreads();
-  for (int e = tid; e < G * D; e += kDecThreads) {
+  for (int e = tid; e < G * D; e += blockDim.x) {
     const int g = e / D, col = e % D;
     float M = -INFINITY;
-    for (int x = 0; x < kWarps; ++x) M = fmaxf(M, s_m[x][g]);
+    for (int x = 0; x < kConsumerWarps; ++x) M = fmaxf(M, s_m[x][g]);
     const float Mu = (M == -INFINITY) ? 0.f : M;
     float sum = 0.f, lsum = 0.f;
-    for (int x = 0; x < kWarps; ++x) {
+    for (int x = 0; x < kConsumerWarps; ++x) {
       const float f = ex2(s_m[x][g] - Mu);
       sum += s_acc[x][g][col] * f;
       lsum += s_l[x][g] * f;
@@ -354,7 +442,7 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads)
   cluster.sync();
   // ---- CTA 0 of the cluster combines the kSplit partial results through DSMEM
   if (cluster.block_rank() == 0) {
-    for (int e = tid; e < G * D; e += kDecThreads) {
+    for (int e = tid; e < G * D; e += blockDim.x) {
       const int g = e / D, col = e % D;
       float mm[kSplit], ll[kSplit], aa[kSplit];
       float M = -INFINITY;
@@ -422,12 +510,23 @@ cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new, c
 template <int D, int G>
 static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void* o, float* lse,
                                    float scale, cudaStream_t stream) {
+  constexpr size_t smem = sizeof(DecSmem<D>);
+  static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(sepcache_decode_kernel<D, G>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   dim3 grid(kSplit, st.Hkv, st.S);
-  sepcache_decode_kernel<D, G><<<grid, kDecThreads, 0, stream>>>(
+  sepcache_decode_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(
       st.Hq, st.Hkv, st.a, st.s, st.w, reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
       reinterpret_cast<const __nv_bfloat16*>(st.v_slots), st.meta,
       reinterpret_cast<const float2*>(st.rope_cs), static_cast<const __nv_bfloat16*>(q),
-      static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f);
+      static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f, device_error_word());
   return cudaGetLastError();
 }
 

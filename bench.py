@@ -501,7 +501,8 @@ def single_row(args, dev):
         del step
         return out
     cfg = {"llama-prefill": workloads.LLAMA3_8B_PREFILL, "long-context": workloads.LONG_CONTEXT,
-           "long-context-dense": workloads.LONG_CONTEXT}[args.workload]
+           "long-context-dense": workloads.LONG_CONTEXT,
+           "pythia-train": workloads.PYTHIA160M}[args.workload]
     n = cfg.L if args.workload == "long-context-dense" else cfg.n
     inp = workloads.attn_inputs(cfg, with_do=args.workload != "llama-prefill")
     d = {k: v.to(dev) for k, v in inp.items() if v is not None}
@@ -535,8 +536,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="train-decode",
-                    choices=["train-decode", "llama-prefill", "long-context", "long-context-dense",
-                             "decode"])
+                    choices=["train-decode", "pythia-train", "llama-prefill", "long-context",
+                             "long-context-dense", "decode"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",

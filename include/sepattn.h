@@ -66,6 +66,7 @@ enum {
  * (n neighbours counted including the query itself). Outputs:
  *   anchor_idx [B, L] int32  positions j with f[j], ascending; entries past anchor_cnt[b] = -1.
  *   anchor_cnt [B]    int32  number of anchors.
+ *   anchor_bits [B, W] uint32 W = ceil(L / 32): bit k of word w is f[32w + k] (0 past L).
  *   gather_end [B, T] int32  T = ceil(L / bm). With lo(t) = max(0, t*bm - n + 1) / bn (integer
  *                            division), gather_end[b][t] = number of anchors at positions
  *                            < lo(t)*bn: the anchors that every row of query tile t keeps and
@@ -78,8 +79,9 @@ enum {
  * bm >= 1, bn >= 1. The attention calls need bm = SEP_TILE_M and bn = SEP_TILE_N.
  */
 int sep_mask_build(const uint8_t* sep, int B, int L, int a, int n, int bm, int bn,
-                   int32_t* anchor_idx, int32_t* anchor_cnt, int32_t* gather_end,
-                   int8_t* tile_map, int64_t* kept_pairs, sep_stream_t stream);
+                   int32_t* anchor_idx, int32_t* anchor_cnt, uint32_t* anchor_bits,
+                   int32_t* gather_end, int8_t* tile_map, int64_t* kept_pairs,
+                   sep_stream_t stream);
 
 /* The outputs of sep_mask_build (built with bm = SEP_TILE_M, bn = SEP_TILE_N) plus the flags. */
 typedef struct SepMask {
@@ -87,6 +89,7 @@ typedef struct SepMask {
   const uint8_t* sep;         /* [B, L] the flags the mask was built from */
   const int32_t* anchor_idx;  /* [B, L] */
   const int32_t* anchor_cnt;  /* [B] */
+  const uint32_t* anchor_bits; /* [B, ceil(L/32)] */
   const int32_t* gather_end;  /* [B, ceil(L/128)] */
   const int8_t* tile_map;     /* [B, ceil(L/128), ceil(L/128)] */
 } SepMask;

@@ -54,8 +54,8 @@ int check_attn_args(const void* q, const void* k, const void* v, int B, int L, i
   if (Hq % Hkv != 0) return SEP_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SEP_ERR_UNSUPPORTED;
   if (mask->B != B || mask->L != L || mask->a != a || mask->n != n) return SEP_ERR_INVALID_ARG;
-  if (!mask->sep || !mask->anchor_idx || !mask->anchor_cnt || !mask->gather_end ||
-      !mask->tile_map)
+  if (!mask->sep || !mask->anchor_idx || !mask->anchor_cnt || !mask->anchor_bits ||
+      !mask->gather_end || !mask->tile_map)
     return SEP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SEP_ERR_MISALIGNED;
   return SEP_OK;
@@ -97,13 +97,15 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? SEP_OK : SEP_ERR_CUDA
 extern "C" {
 
 int sep_mask_build(const uint8_t* sep, int B, int L, int a, int n, int bm, int bn,
-                   int32_t* anchor_idx, int32_t* anchor_cnt, int32_t* gather_end,
-                   int8_t* tile_map, int64_t* kept_pairs, sep_stream_t stream) {
-  if (!sep || !anchor_idx || !anchor_cnt || !gather_end || !tile_map) return SEP_ERR_INVALID_ARG;
+                   int32_t* anchor_idx, int32_t* anchor_cnt, uint32_t* anchor_bits,
+                   int32_t* gather_end, int8_t* tile_map, int64_t* kept_pairs,
+                   sep_stream_t stream) {
+  if (!sep || !anchor_idx || !anchor_cnt || !anchor_bits || !gather_end || !tile_map)
+    return SEP_ERR_INVALID_ARG;
   if (B < 1 || L < 1 || a < 0 || n < 1 || bm < 1 || bn < 1) return SEP_ERR_INVALID_ARG;
   if (L > (1 << 30)) return SEP_ERR_UNSUPPORTED;
   return cuda_status(sep::launch_mask_build(sep, B, L, a, n, bm, bn, anchor_idx, anchor_cnt,
-                                            gather_end, tile_map, kept_pairs,
+                                            anchor_bits, gather_end, tile_map, kept_pairs,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -141,7 +143,7 @@ static int attn_fwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const
       return SEP_ERR_CUDA;
     AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
     return cuda_status(
-        sep::launch_attn_fwd(maps, sh, mask->sep, mask->gather_end, mask->tile_map, o, lse, s));
+        sep::launch_attn_fwd(maps, sh, mask->anchor_bits, mask->gather_end, mask->tile_map, o, lse, s));
   }
   return SEP_OK;
 }
@@ -194,7 +196,7 @@ static int attn_bwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const
     return SEP_ERR_CUDA;
   AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
   return cuda_status(sep::launch_attn_bwd(
-      maps, sh, mask->sep, mask->anchor_idx, mask->anchor_cnt, mask->gather_end, mask->tile_map,
+      maps, sh, mask->anchor_bits, mask->anchor_idx, mask->anchor_cnt, mask->gather_end, mask->tile_map,
       o, lse, dout, q, k, v, dq, dk, dv, kc, vc, reinterpret_cast<float*>(ws + w.delta),
       reinterpret_cast<float*>(ws + w.dka), reinterpret_cast<float*>(ws + w.dva), stages, s));
 }

@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
 // ------------------------------------------------------------------ shared parameter block
 struct BwdParams {
   CUtensorMap tmQ, tmK, tmV, tmKc, tmVc, tmdO;
-  const uint8_t* sep;
+  const uint32_t* anchor_bits;  // [B, W] packed anchor flags
   const int32_t* anchor_idx;
   const int32_t* anchor_cnt;
   const int32_t* gather_end;
@@ -95,7 +95,7 @@ struct BwdParams {
   float* dka;  // [B, L, Hkv, D] fp32 anchor partials (rows < anchor_cnt)
   float* dva;
   unsigned* err;
-  int B, L, Hq, Hkv, T, a, n;
+  int B, L, Hq, Hkv, T, W, a, n;
   float scale, scale_log2;
 };
 
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(192, 1) sep_attn_bwd_dq_kernel(const __grid_co
     const long long i = (long long)t * 128 + row;
     const bool valid = i < p.L;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint8_t* sep_row = p.sep + (size_t)b * p.L;
+    const uint32_t* bits_row = p.anchor_bits + (size_t)b * p.W;
     const int8_t* tmap = p.tile_map + ((size_t)b * p.T + t) * p.T;
     const float sl2 = p.scale_log2;
     const size_t rowstat = ((size_t)b * p.Hq + h) * p.L + (valid ? i : 0);
@@ -291,7 +291,8 @@ __global__ void __launch_bounds__(192, 1) sep_attn_bwd_dq_kernel(const __grid_co
         if (tmap[u] != SEP_TILE_FULL) {
 #pragma unroll
           for (int w = 0; w < 4; ++w)
-            keep[w] = window_keep_word(w, i, k0, p.n, p.L, anchor_bits32(sep_row, k0 + 32 * w, p.L, p.a));
+            keep[w] = window_keep_word(w, i, k0, p.n, p.L,
+                                       (u * 4 + w < p.W) ? __ldg(bits_row + u * 4 + w) : 0u);
         } else if (k0 + 128 > p.L) {
 #pragma unroll
           for (int w = 0; w < 4; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, w);
@@ -587,7 +588,7 @@ __global__ void __launch_bounds__(192, 1) sep_attn_bwd_dkv_kernel(const __grid_c
     const long long j = window ? (long long)u * 128 + krow : -1;
     const int r = window ? -1 : c * 128 + krow;
     bool fj = false;
-    if (window && j < p.L) fj = (j < p.a) || p.sep[(size_t)b * p.L + j] != 0;
+    if (window && j < p.L) fj = (__ldg(p.anchor_bits + (size_t)b * p.W + (j >> 5)) >> (j & 31)) & 1u;
     bool ok = true;
     for (int q = 0; q < npairs; ++q) {
       const int st = q % NST;
@@ -752,7 +753,7 @@ __global__ void __launch_bounds__(256) anchor_combine_kernel(
   }
 }
 
-cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint8_t* sep,
+cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint32_t* anchor_bits,
                             const int32_t* anchor_idx, const int32_t* anchor_cnt,
                             const int32_t* gather_end, const int8_t* tile_map, const void* o,
                             const float* lse, const void* dout, const void* q, const void* k,
@@ -794,7 +795,7 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.tmKc = maps.kc;
   prm.tmVc = maps.vc;
   prm.tmdO = maps.dout;
-  prm.sep = sep;
+  prm.anchor_bits = anchor_bits;
   prm.anchor_idx = anchor_idx;
   prm.anchor_cnt = anchor_cnt;
   prm.gather_end = gather_end;
@@ -812,6 +813,7 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.Hq = s.Hq;
   prm.Hkv = s.Hkv;
   prm.T = (s.L + 127) / 128;
+  prm.W = (s.L + 31) / 32;
   prm.a = s.a;
   prm.n = s.n;
   prm.scale = s.scale;

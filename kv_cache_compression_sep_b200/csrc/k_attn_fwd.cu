@@ -24,6 +24,8 @@
 // S_{j+1} is issued before PV_j so the tensor core works while softmax runs.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "sep_common.cuh"
 #include "sep_launch.h"
 #include "sep_tiles.cuh"
@@ -32,13 +34,13 @@ namespace sep {
 
 struct FwdParams {
   CUtensorMap tmQ, tmK, tmV, tmKc, tmVc;
-  const uint8_t* sep;
+  const uint32_t* anchor_bits;  // [B, W] packed anchor flags
   const int32_t* gather_end;
   const int8_t* tile_map;
   __nv_bfloat16* o;
   float* lse;
   unsigned* err;
-  int B, L, Hq, Hkv, T, a, n;
+  int B, L, Hq, Hkv, T, W, a, n;
   float scale_log2;
 };
 
@@ -48,19 +50,20 @@ struct FwdCfg {
   static constexpr int KB = D / 64;                 // 128-byte column boxes per row
   static constexpr int BOX_BYTES = 128 * 64 * 2;    // one [128 rows][64 cols] bf16 box
   static constexpr int TILE_BYTES = KB * BOX_BYTES; // one [128][D] tile
-  static constexpr int NST = (D == 128) ? 2 : 4;    // K/V pipeline stages (1 CTA per SM)
-  static constexpr int SMEM_TILES = TILE_BYTES * (1 + 2 * NST);
-  static constexpr int TMEM_COLS = 512;
-  static constexpr int COL_S = 0;      // S[0], S[1]: 128 fp32 columns each
-  static constexpr int COL_O = 256;    // O: D fp32 columns
-  static constexpr int COL_P = 384;    // P[0], P[1]: 64 columns each (bf16 pairs)
+  static constexpr int NST = (D == 128) ? 2 : 2;    // K/V pipeline stages
+  static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * NST);  // Q x2, NST x (K, V)
+  static constexpr int COL_S = 0;        // S: 128 fp32 columns
+  static constexpr int COL_O = 128;      // O: D fp32 columns
+  static constexpr int COL_P = 128 + D;  // P: 64 columns (bf16 pairs)
+  static constexpr int TMEM_COLS = (COL_P + 64 <= 256) ? 256 : 512;
+  static constexpr int CTAS_PER_SM = (TMEM_COLS == 256) ? 2 : 1;
 };
 
 template <int NST>
 struct FwdBar {
-  uint64_t q_full;
+  uint64_t q_full[2], q_empty[2];
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
-  uint64_t s_full[2], p_ready[2], pv_done[2];
+  uint64_t s_full, s_free, p_ready, pv_done;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -71,42 +74,81 @@ constexpr size_t fwd_smem_bytes() {
   return 1024 /*alignment slack*/ + FwdCfg<D>::SMEM_TILES + sizeof(FwdBar<FwdCfg<D>::NST>);
 }
 
+// Work item x (heaviest query tiles first): query tile t, head h, batch b, and its key tiles.
+struct FwdItem {
+  int t, h, b, nwin, ge, N;
+};
+__device__ __forceinline__ FwdItem fwd_item_base(const FwdParams& p, int x) {
+  FwdItem it;
+  const int per_t = p.Hq * p.B;
+  it.t = p.T - 1 - x / per_t;
+  const int rem = x % per_t;
+  it.h = rem % p.Hq;
+  it.b = rem / p.Hq;
+  it.nwin = it.t - window_lo_tile(it.t, p.n) + 1;
+  it.ge = 0;
+  it.N = it.nwin;
+  return it;
+}
+__device__ __forceinline__ int fwd_item_ge(const FwdParams& p, int x) {
+  const FwdItem it = fwd_item_base(p, x);
+  return p.gather_end[(size_t)it.b * p.T + it.t];
+}
+__device__ __forceinline__ FwdItem fwd_item_with(const FwdParams& p, int x, int ge) {
+  FwdItem it = fwd_item_base(p, x);
+  it.ge = ge;
+  it.N = it.nwin + (ge + 127) / 128;
+  return it;
+}
+
+// Raw mask inputs of one window key tile: its tile-map class and 128 anchor-flag bits.
+struct TileRaw {
+  uint32_t fb[4];
+  int cls;
+};
+__device__ __forceinline__ TileRaw load_tile_raw(const FwdParams& p, int b, int t, int u) {
+  TileRaw r;
+  r.cls = p.tile_map[((size_t)b * p.T + t) * p.T + u];
+  const uint32_t* w = p.anchor_bits + (size_t)b * p.W + (size_t)u * 4;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) r.fb[q] = (u * 4 + q < p.W) ? __ldg(w + q) : 0u;
+  return r;
+}
+
+// Persistent: CTA c handles items c, c + gridDim.x, ... Every role walks the same flattened
+// sequence of key tiles (g = 0, 1, ... over all its items), so pipeline phases carry across
+// item boundaries and the next item's loads and first MMA overlap the current item's tail.
 template <int D>
-__global__ void __launch_bounds__(192, 1) sep_attn_fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
+    sep_attn_fwd_kernel(const __grid_constant__ FwdParams p, int nitems) {
   using C = FwdCfg<D>;
   constexpr int NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::TILE_BYTES;
+  uint8_t* sQ = smem;                       // 2 buffers (item parity)
+  uint8_t* sK = sQ + 2 * C::TILE_BYTES;
   uint8_t* sV = sK + NST * C::TILE_BYTES;
   FwdBar<NST>* bar = reinterpret_cast<FwdBar<NST>*>(sV + NST * C::TILE_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = p.T - 1 - (int)blockIdx.x;  // heaviest query tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int kvh = h / (p.Hq / p.Hkv);
-  const int lo_tile = window_lo_tile(t, p.n);
-  const int nwin = t - lo_tile + 1;
-  const int ge = p.gather_end[(size_t)b * p.T + t];
-  const int ngat = (ge + C::BN - 1) / C::BN;
-  const int N = nwin + ngat;
   volatile int* abort_flag = &bar->abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->q_full[s], 1);
+      mbar_init(&bar->q_empty[s], 1);
+    }
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->p_ready[s], 128);
-      mbar_init(&bar->pv_done[s], 1);
-    }
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->s_free, 128);
+    mbar_init(&bar->p_ready, 128);
+    mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
@@ -126,36 +168,54 @@ __global__ void __launch_bounds__(192, 1) sep_attn_fwd_kernel(const __grid_const
       tma_prefetch_desc(&p.tmQ);
       tma_prefetch_desc(&p.tmK);
       tma_prefetch_desc(&p.tmV);
-      mbar_arrive_expect_tx(&bar->q_full, C::TILE_BYTES);
-      for (int kb = 0; kb < C::KB; ++kb)
-        tma_load_4d(sQ + kb * C::BOX_BYTES, &p.tmQ, &bar->q_full, kb * 64, h, t * C::BM, b);
-      for (int j = 0; j < N; ++j) {
-        const int st = j % NST, r = j / NST;
-        const bool win = j < nwin;
-        const CUtensorMap* mk = win ? &p.tmK : &p.tmKc;
-        const CUtensorMap* mv = win ? &p.tmV : &p.tmVc;
-        const int row0 = win ? (t - j) * C::BN : (j - nwin) * C::BN;
-        if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag)) break;
-        mbar_arrive_expect_tx(&bar->k_full[st], C::TILE_BYTES);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_4d(sK + st * C::TILE_BYTES + kb * C::BOX_BYTES, mk, &bar->k_full[st], kb * 64,
-                      kvh, row0, b);
-        if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag)) {
-          // K of this tile is in flight: let it land before leaving
-          mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
+      tma_prefetch_desc(&p.tmKc);
+      tma_prefetch_desc(&p.tmVc);
+      int g = 0;
+      bool ok = true;
+      int ge_cur = fwd_item_ge(p, blockIdx.x);
+      for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
+        const FwdItem it = fwd_item_with(p, x, ge_cur);
+        if (x + (int)gridDim.x < nitems) ge_cur = fwd_item_ge(p, x + gridDim.x);  // prefetch
+        const int kvh = it.h / (p.Hq / p.Hkv);
+        const int qb = k & 1;
+        if (k >= 2 && !mbar_wait(&bar->q_empty[qb], ((k - 2) >> 1) & 1, p.err, abort_flag)) {
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bar->v_full[st], C::TILE_BYTES);
+        mbar_arrive_expect_tx(&bar->q_full[qb], C::TILE_BYTES);
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_4d(sV + st * C::TILE_BYTES + kb * C::BOX_BYTES, mv, &bar->v_full[st], kb * 64,
-                      kvh, row0, b);
+          tma_load_4d(sQ + qb * C::TILE_BYTES + kb * C::BOX_BYTES, &p.tmQ, &bar->q_full[qb],
+                      kb * 64, it.h, it.t * C::BM, it.b);
+        for (int j = 0; j < it.N; ++j, ++g) {
+          const int st = g % NST, r = g / NST;
+          const bool win = j < it.nwin;
+          const CUtensorMap* mk = win ? &p.tmK : &p.tmKc;
+          const CUtensorMap* mv = win ? &p.tmV : &p.tmVc;
+          const int row0 = win ? (it.t - j) * C::BN : (j - it.nwin) * C::BN;
+          if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar->k_full[st], C::TILE_BYTES);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_4d(sK + st * C::TILE_BYTES + kb * C::BOX_BYTES, mk, &bar->k_full[st],
+                        kb * 64, kvh, row0, it.b);
+          if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag)) {
+            mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar->v_full[st], C::TILE_BYTES);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_4d(sV + st * C::TILE_BYTES + kb * C::BOX_BYTES, mv, &bar->v_full[st],
+                        kb * 64, kvh, row0, it.b);
+        }
       }
-      if (*abort_flag) {
-        // drain: wait (bounded) until every issued load has landed
-        mbar_wait(&bar->q_full, 0, nullptr, nullptr);
-        for (int j = max(0, N - NST); j < N; ++j) {
-          mbar_wait(&bar->k_full[j % NST], (j / NST) & 1, nullptr, nullptr);
-          mbar_wait(&bar->v_full[j % NST], (j / NST) & 1, nullptr, nullptr);
+      if (!ok) {
+        // drain: let every load issued for the last NST tiles and both Q buffers land
+        for (int gg = max(0, g - NST); gg < g; ++gg) {
+          mbar_wait(&bar->k_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
+          mbar_wait(&bar->v_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
         }
       }
     }
@@ -165,137 +225,182 @@ __global__ void __launch_bounds__(192, 1) sep_attn_fwd_kernel(const __grid_const
       constexpr uint32_t idS = make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = make_idesc_bf16(128, D, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      bool ok = mbar_wait(&bar->q_full, 0, p.err, abort_flag);
-      auto issue_S = [&](int j) -> bool {
-        const int st = j % NST;
-        if (!mbar_wait(&bar->k_full[st], (j / NST) & 1, p.err, abort_flag)) return false;
+      bool ok = true;
+      int g = 0;           // global index of the next S tile
+      int pv_pending = -1; // global index of the tile whose PV is still to issue
+      int pv_first = 0;    // that tile is the first of its item (overwrite O)
+      auto issue_PV = [&](int gg, int first) -> bool {
+        const int st = gg % NST;
+        if (!mbar_wait(&bar->p_ready, gg & 1, p.err, abort_flag)) return false;
+        if (!mbar_wait(&bar->v_full[st], (gg / NST) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t dS = tmem + C::COL_S + (j & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          const uint64_t ad = make_sdesc_sw128(sQa + off, 16, 1024);
-          const uint64_t bd = make_sdesc_sw128(sKa + st * C::TILE_BYTES + off, 16, 1024);
-          mma_ss(dS, ad, bd, idS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bar->s_full[j & 1]);
-        tc_commit(&bar->k_empty[st]);
-        return true;
-      };
-      auto issue_PV = [&](int j) -> bool {
-        const int st = j % NST;
-        if (!mbar_wait(&bar->p_ready[j & 1], (j >> 1) & 1, p.err, abort_flag)) return false;
-        if (!mbar_wait(&bar->v_full[st], (j / NST) & 1, p.err, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t aP = tmem + C::COL_P + (j & 1) * 64;
+        const uint32_t aP = tmem + C::COL_P;
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk) {
           const uint64_t bd =
               make_sdesc_sw128(sVa + st * C::TILE_BYTES + kk * 2048, C::BOX_BYTES, 1024);
-          mma_ts(tmem + C::COL_O, aP + kk * 8, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::COL_O, aP + kk * 8, bd, idO, (!first || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&bar->pv_done[j & 1]);
+        tc_commit(&bar->pv_done);
         tc_commit(&bar->v_empty[st]);
         return true;
       };
-      if (ok) ok = issue_S(0);
-      for (int j = 0; ok && j < N; ++j) {
-        if (j + 1 < N && !issue_S(j + 1)) break;
-        if (!issue_PV(j)) break;
+      int ge_cur = fwd_item_ge(p, blockIdx.x);
+      for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
+        const FwdItem it = fwd_item_with(p, x, ge_cur);
+        if (x + (int)gridDim.x < nitems) ge_cur = fwd_item_ge(p, x + gridDim.x);  // prefetch
+        const int qb = k & 1;
+        if (!mbar_wait(&bar->q_full[qb], (k >> 1) & 1, p.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sQb = sQa + qb * C::TILE_BYTES;
+        for (int j = 0; j < it.N; ++j, ++g) {
+          const int st = g % NST;
+          if (!mbar_wait(&bar->k_full[st], (g / NST) & 1, p.err, abort_flag)) { ok = false; break; }
+          // S has one buffer: the softmax warps must have loaded S_{g-1}
+          if (g > 0 && !mbar_wait(&bar->s_free, (g - 1) & 1, p.err, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+            const uint64_t ad = make_sdesc_sw128(sQb + off, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(sKa + st * C::TILE_BYTES + off, 16, 1024);
+            mma_ss(tmem + C::COL_S, ad, bd, idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bar->s_full);
+          tc_commit(&bar->k_empty[st]);
+          if (j == it.N - 1) tc_commit(&bar->q_empty[qb]);
+          // P V of the previous tile, while the softmax warps work on this one
+          if (pv_pending >= 0 && !issue_PV(pv_pending, pv_first)) { ok = false; break; }
+          pv_pending = g;
+          pv_first = (j == 0);
+        }
       }
-      // make sure every MMA issued has completed before TMEM is released
+      if (ok && pv_pending >= 0) issue_PV(pv_pending, pv_first);
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }
   } else {
     // ------------------------------------------------------------ softmax warpgroup
     const int row = threadIdx.x;  // 0..127 = TMEM lane
-    const long long i = (long long)t * C::BM + row;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint8_t* sep_row = p.sep + (size_t)b * p.L;
-    const int8_t* tmap = p.tile_map + ((size_t)b * p.T + t) * p.T;
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < N; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[sb], (j >> 1) & 1, p.err, abort_flag))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t s[128];
-      {
-        uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-        uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-        uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-        uint32_t (&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-        const uint32_t a0 = tmem + lane_off + C::COL_S + sb * 128;
-        tmem_ld32(a0, c0);
-        tmem_ld32(a0 + 32, c1);
-        tmem_ld32(a0 + 64, c2);
-        tmem_ld32(a0 + 96, c3);
-        tmem_ld_wait();
-      }
-      // ---- mask
-      uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      bool masked = false;
-      if (j < nwin) {
-        const int u = t - j;
-        const long long k0 = (long long)u * C::BN;
-        const int cls = tmap[u];
-        if (cls != SEP_TILE_FULL) {
-          masked = true;
+    int g = 0;
+    int ge_cur = fwd_item_ge(p, blockIdx.x);
+    TileRaw cur;  // mask inputs of the next tile to process, loaded one tile ahead
+    {
+      const FwdItem f0 = fwd_item_base(p, blockIdx.x);
+      cur = load_tile_raw(p, f0.b, f0.t, f0.t);
+    }
+    for (int x = blockIdx.x; ok && x < nitems; x += gridDim.x) {
+      const FwdItem it = fwd_item_with(p, x, ge_cur);
+      const int xn = x + gridDim.x;
+      if (xn < nitems) ge_cur = fwd_item_ge(p, xn);  // prefetch the next item's gather count
+      const long long i = (long long)it.t * C::BM + row;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < it.N; ++j, ++g) {
+        const TileRaw raw = cur;
+        // prefetch the next tile's mask inputs (next window tile of this item, or the
+        // diagonal tile of the next item)
+        if (j + 1 < it.nwin) {
+          cur = load_tile_raw(p, it.b, it.t, it.t - (j + 1));
+        } else if (j + 1 == it.N && xn < nitems) {
+          const FwdItem fn = fwd_item_base(p, xn);
+          cur = load_tile_raw(p, fn.b, fn.t, fn.t);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, g & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[128];
+        {
+          uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+          uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
+          uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
+          uint32_t (&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
+          const uint32_t a0 = tmem + lane_off + C::COL_S;
+          tmem_ld32(a0, c0);
+          tmem_ld32(a0 + 32, c1);
+          tmem_ld32(a0 + 64, c2);
+          tmem_ld32(a0 + 96, c3);
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&bar->s_free);  // S may be overwritten by the next tile's MMA
+        // ---- mask
+        uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        bool masked = false;
+        if (j < it.nwin) {
+          const int u = it.t - j;
+          const long long k0 = (long long)u * C::BN;
+          if (raw.cls != SEP_TILE_FULL) {
+            masked = true;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t fb = anchor_bits32(sep_row, k0 + 32 * w, p.L, p.a);
-            keep[w] = window_keep_word(w, i, k0, p.n, p.L, fb);
+            for (int w = 0; w < 4; ++w) keep[w] = window_keep_word(w, i, k0, p.n, p.L, raw.fb[w]);
+          } else if (k0 + C::BN > p.L) {
+            masked = true;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, w);
           }
-        } else if (k0 + C::BN > p.L) {
-          masked = true;
+        } else {
+          const int rem = it.ge - (j - it.nwin) * C::BN;  // valid anchors in this chunk
+          if (rem < C::BN) {
+            masked = true;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const long long hi = (long long)p.L - 1 - (k0 + 32 * w);
-            keep[w] = (hi < 0) ? 0u : (hi >= 31 ? 0xffffffffu : ((2u << hi) - 1u));
+            for (int w = 0; w < 4; ++w) keep[w] = range_word(0, rem - 1, w);
           }
         }
-      } else {
-        const int rem = ge - (j - nwin) * C::BN;  // valid anchors in this chunk
-        if (rem < C::BN) {
-          masked = true;
+        float mx = -INFINITY;
+        if (masked) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int hi = rem - 1 - 32 * w;
-            keep[w] = (hi < 0) ? 0u : (hi >= 31 ? 0xffffffffu : ((2u << hi) - 1u));
+          for (int c = 0; c < 128; ++c) {
+            const float v = ((keep[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(s[c]) : -INFINITY;
+            s[c] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+        }
+        // ---- online max with lazy rescale (only when the max grows by more than 2^8)
+        const float m_tile = mx * sl2;
+        float alpha = 1.0f;
+        bool any_rescale = false;
+        if (j == 0) {
+          m_run = m_tile;
+        } else {
+          const bool need = m_tile > m_run + 8.0f;
+          any_rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2(m_run - m_tile);
+            l_run *= alpha;
+            m_run = m_tile;
           }
         }
-      }
-      float mx = -INFINITY;
-      if (masked) {
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        // ---- P = exp2(S * scale*log2e - m), row sum, packed to bf16 pairs in place over the
+        // already consumed S registers (pair c/2 <= c)
+        float sum = 0.f;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const float v = ((keep[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(s[c]) : -INFINITY;
-          s[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+        for (int c = 0; c < 128; c += 2) {
+          const float e0 = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
+          const float e1 = ex2(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
+          sum += e0 + e1;
+          s[c >> 1] = pack_bf16x2(e0, e1);
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
-      }
-      // ---- online max with lazy rescale (only when the max grows by more than 2^8)
-      const float m_tile = mx * sl2;
-      if (j == 0) {
-        m_run = m_tile;
-      } else {
-        const bool need = m_tile > m_run + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1,
-                                                 p.err, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float alpha = need ? ex2(m_run - m_tile) : 1.0f;
+        uint32_t* pk = s;
+        l_run += sum;
+        // P and O: the previous tile's P V must be complete (it read P and accumulated O)
+        if (g > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (any_rescale) {
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t ov[32];
@@ -306,47 +411,27 @@ __global__ void __launch_bounds__(192, 1) sep_attn_fwd_kernel(const __grid_const
             for (int q = 0; q < 32; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * alpha);
             tmem_st32(ao, ov);
           }
-          tmem_st_wait();
-          if (need) {
-            l_run *= alpha;
-            m_run = m_tile;
-          }
         }
+        {
+          const uint32_t ap = tmem + lane_off + C::COL_P;
+          tmem_st32(ap, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+          tmem_st32(ap + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&bar->p_ready);
       }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // ---- P = exp2(S * scale*log2e - m), row sum, pack to bf16 pairs
-      uint32_t pk[64];
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float e0 = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
-        const float e1 = ex2(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
-        sum += e0 + e1;
-        pk[c >> 1] = pack_bf16x2(e0, e1);
-      }
-      l_run += sum;
-      // P[j%2] was read by PV_{j-2}: wait for it before overwriting
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar->pv_done[sb], ((j - 2) >> 1) & 1,
-                                                     p.err, abort_flag))) {
+      if (!ok) break;
+      // ---- epilogue of this item: O / l, LSE (O is reused by the next item's first P V,
+      // which the MMA warp issues only after this thread's next p_ready arrive)
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {
         ok = false;
         break;
       }
-      {
-        const uint32_t ap = tmem + lane_off + C::COL_P + sb * 64;
-        tmem_st32(ap, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(ap + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      mbar_arrive(&bar->p_ready[sb]);
-    }
-    // ---- epilogue: O / l, LSE
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar->pv_done[(N - 1) & 1], ((N - 1) >> 1) & 1,
-                                                p.err, abort_flag))) {
       tc_fence_after();
       const float inv_l = 1.0f / l_run;
       const bool valid = i < p.L;
-      __nv_bfloat16* orow = p.o + (((size_t)b * p.L + (valid ? i : 0)) * p.Hq + h) * D;
+      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.L + (valid ? i : 0)) * p.Hq + it.h) * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t ov[32];
@@ -365,7 +450,8 @@ __global__ void __launch_bounds__(192, 1) sep_attn_fwd_kernel(const __grid_const
         }
       }
       if (valid)
-        p.lse[((size_t)b * p.Hq + h) * p.L + i] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        p.lse[((size_t)it.b * p.Hq + it.h) * p.L + i] =
+            (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
     tc_fence_before();
   }
@@ -418,10 +504,23 @@ cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* 
   return cudaGetLastError();
 }
 
+static int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 template <int D>
 static cudaError_t launch_fwd_t(const FwdParams& prm, int T, int Hq, int B, cudaStream_t stream) {
   constexpr size_t smem = fwd_smem_bytes<D>();
-  static_assert(smem <= 227 * 1024, "shared memory budget");
+  static_assert(smem * FwdCfg<D>::CTAS_PER_SM <= 228 * 1024, "shared memory budget");
   static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -432,11 +531,13 @@ static cudaError_t launch_fwd_t(const FwdParams& prm, int T, int Hq, int B, cuda
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  sep_attn_fwd_kernel<D><<<dim3(T, Hq, B), 192, smem, stream>>>(prm);
+  const int nitems = T * Hq * B;
+  const int grid = std::min(nitems, sm_count() * FwdCfg<D>::CTAS_PER_SM);
+  sep_attn_fwd_kernel<D><<<grid, 192, smem, stream>>>(prm, nitems);
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint8_t* sep,
+cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint32_t* anchor_bits,
                             const int32_t* gather_end, const int8_t* tile_map, void* o,
                             float* lse, cudaStream_t stream) {
   FwdParams prm;
@@ -445,7 +546,7 @@ cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.tmV = maps.v;
   prm.tmKc = maps.kc;
   prm.tmVc = maps.vc;
-  prm.sep = sep;
+  prm.anchor_bits = anchor_bits;
   prm.gather_end = gather_end;
   prm.tile_map = tile_map;
   prm.o = static_cast<__nv_bfloat16*>(o);
@@ -456,6 +557,7 @@ cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.Hq = s.Hq;
   prm.Hkv = s.Hkv;
   prm.T = (s.L + 127) / 128;
+  prm.W = (s.L + 31) / 32;
   prm.a = s.a;
   prm.n = s.n;
   prm.scale_log2 = s.scale * 1.4426950408889634f;

@@ -25,12 +25,14 @@ __global__ void __launch_bounds__(kScanThreads) mask_scan_kernel(const uint8_t* 
                                                                  int L, int a, int n,
                                                                  int32_t* __restrict__ anchor_idx,
                                                                  int32_t* __restrict__ anchor_cnt,
+                                                                 uint32_t* __restrict__ anchor_bits,
                                                                  int64_t* __restrict__ kept) {
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   sep += (size_t)b * L;
   anchor_idx += (size_t)b * L;
+  anchor_bits += (size_t)b * ((L + 31) / 32);
 
   __shared__ int s_warp[32];
   __shared__ long long s_red[32];
@@ -47,6 +49,11 @@ __global__ void __launch_bounds__(kScanThreads) mask_scan_kernel(const uint8_t* 
     for (int k = 0; k < kScanItems; ++k) {
       const int j = j0 + k;
       if (j < L && (j < a || sep[j] != 0)) bits |= 1u << k;
+    }
+    // packed flags: lanes 2k and 2k+1 hold the two 16-position halves of word j0 / 32
+    {
+      const uint32_t hi = __shfl_down_sync(0xffffffffu, bits, 1);
+      if ((lane & 1) == 0 && j0 < L) anchor_bits[j0 / 32] = bits | (hi << 16);
     }
     const int cnt = __popc(bits);
     // block exclusive scan of cnt
@@ -166,9 +173,11 @@ unsigned* device_error_word() {
 }
 
 cudaError_t launch_mask_build(const uint8_t* sep, int B, int L, int a, int n, int bm, int bn,
-                              int32_t* anchor_idx, int32_t* anchor_cnt, int32_t* gather_end,
-                              int8_t* tile_map, int64_t* kept, cudaStream_t stream) {
-  mask_scan_kernel<<<B, kScanThreads, 0, stream>>>(sep, L, a, n, anchor_idx, anchor_cnt, kept);
+                              int32_t* anchor_idx, int32_t* anchor_cnt, uint32_t* anchor_bits,
+                              int32_t* gather_end, int8_t* tile_map, int64_t* kept,
+                              cudaStream_t stream) {
+  mask_scan_kernel<<<B, kScanThreads, 0, stream>>>(sep, L, a, n, anchor_idx, anchor_cnt,
+                                                   anchor_bits, kept);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int T = (L + bm - 1) / bm, U = (L + bn - 1) / bn;

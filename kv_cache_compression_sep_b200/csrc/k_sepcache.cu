@@ -229,13 +229,24 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 2)
     const int c0 = r0 + ch * kChunk;
     const int rows = min(kChunk, r1 - c0);
     mbar_arrive_expect_tx(&sm.full[st], (uint32_t)(rows * D * 2 * 2));
+    // ranks map to slots piecewise contiguously: initial block, then the separator ring, then
+    // the window ring; a run ends at a block boundary or where a ring wraps
     int r = c0;
-    while (r < c0 + rows) {
-      const int slot = rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w);
-      int len = 1;  // extend while the next rank sits in the next slot
-      while (r + len < c0 + rows &&
-             rank_to_slot(r + len, ninit, sep_head, sep_cnt, win_head, a, s, w) == slot + len)
-        ++len;
+    const int end = c0 + rows;
+    while (r < end) {
+      int slot, len;
+      if (r < ninit) {
+        slot = r;
+        len = min(end, ninit) - r;
+      } else if (r < ninit + sep_cnt) {
+        const int x = (sep_head + (r - ninit)) % s;
+        slot = a + x;
+        len = min(min(end, ninit + sep_cnt) - r, s - x);
+      } else {
+        const int x = (win_head + (r - ninit - sep_cnt)) % w;
+        slot = a + s + x;
+        len = min(end - r, w - x);
+      }
       const size_t src = (row_base + slot) * D;
       bulk_load(&sm.k[st][r - c0][0], k_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
       bulk_load(&sm.v[st][r - c0][0], v_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);

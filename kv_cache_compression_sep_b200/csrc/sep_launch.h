@@ -15,8 +15,9 @@ namespace sep {
 unsigned* device_error_word();
 
 cudaError_t launch_mask_build(const uint8_t* sep, int B, int L, int a, int n, int bm, int bn,
-                              int32_t* anchor_idx, int32_t* anchor_cnt, int32_t* gather_end,
-                              int8_t* tile_map, int64_t* kept, cudaStream_t stream);
+                              int32_t* anchor_idx, int32_t* anchor_cnt, uint32_t* anchor_bits,
+                              int32_t* gather_end, int8_t* tile_map, int64_t* kept,
+                              cudaStream_t stream);
 
 // Stage bits of launch_attn_bwd.
 constexpr int kBwdPrep = 1, kBwdDq = 2, kBwdDkv = 4, kBwdAll = 7;
@@ -36,11 +37,11 @@ struct AttnShape {
   float scale;
 };
 
-cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint8_t* sep,
+cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint32_t* anchor_bits,
                             const int32_t* gather_end, const int8_t* tile_map, void* o,
                             float* lse, cudaStream_t stream);
 
-cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint8_t* sep,
+cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint32_t* anchor_bits,
                             const int32_t* anchor_idx, const int32_t* anchor_cnt,
                             const int32_t* gather_end, const int8_t* tile_map, const void* o,
                             const float* lse, const void* dout, const void* q, const void* k,

@@ -32,7 +32,7 @@ def _load():
     lib = ctypes.CDLL(_LIB_PATH)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
-        "sep_mask_build": (I, [P, I, I, I, I, I, I, P, P, P, P, P, P]),
+        "sep_mask_build": (I, [P, I, I, I, I, I, I, P, P, P, P, P, P, P]),
         "sep_attn_fwd_workspace_size": (Z, [I, I, I, I]),
         "sep_attn_fwd": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
         "sep_attn_fwd_stage": (I, [I, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
@@ -59,7 +59,8 @@ _lib = _load()
 class _SepMask(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("L", ctypes.c_int), ("a", ctypes.c_int), ("n", ctypes.c_int),
                 ("sep", ctypes.c_void_p), ("anchor_idx", ctypes.c_void_p),
-                ("anchor_cnt", ctypes.c_void_p), ("gather_end", ctypes.c_void_p),
+                ("anchor_cnt", ctypes.c_void_p), ("anchor_bits", ctypes.c_void_p),
+                ("gather_end", ctypes.c_void_p),
                 ("tile_map", ctypes.c_void_p)]
 
 
@@ -100,6 +101,7 @@ class SepMask:
     sep: torch.Tensor
     anchor_idx: torch.Tensor
     anchor_cnt: torch.Tensor
+    anchor_bits: torch.Tensor
     gather_end: torch.Tensor
     tile_map: torch.Tensor
     kept: torch.Tensor
@@ -109,8 +111,8 @@ class SepMask:
     def _c(self):
         B, L = self.sep.shape
         return _SepMask(B, L, self.a, self.n, self.sep.data_ptr(), self.anchor_idx.data_ptr(),
-                        self.anchor_cnt.data_ptr(), self.gather_end.data_ptr(),
-                        self.tile_map.data_ptr())
+                        self.anchor_cnt.data_ptr(), self.anchor_bits.data_ptr(),
+                        self.gather_end.data_ptr(), self.tile_map.data_ptr())
 
 
 def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = TILE,
@@ -126,12 +128,13 @@ def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = 
         out = SepMask(sep=sep,
                       anchor_idx=torch.empty(B, L, dtype=torch.int32, device=dev),
                       anchor_cnt=torch.empty(B, dtype=torch.int32, device=dev),
+                      anchor_bits=torch.empty(B, -(-L // 32), dtype=torch.int32, device=dev),
                       gather_end=torch.empty(B, T, dtype=torch.int32, device=dev),
                       tile_map=torch.empty(B, T, U, dtype=torch.int8, device=dev),
                       kept=torch.empty(B, dtype=torch.int64, device=dev), a=a, n=n)
     _check(_lib.sep_mask_build(_ptr(sep), B, L, a, n, bm, bn, _ptr(out.anchor_idx),
-                               _ptr(out.anchor_cnt), _ptr(out.gather_end), _ptr(out.tile_map),
-                               _ptr(out.kept), _stream()), "sep_mask_build")
+                               _ptr(out.anchor_cnt), _ptr(out.anchor_bits), _ptr(out.gather_end),
+                               _ptr(out.tile_map), _ptr(out.kept), _stream()), "sep_mask_build")
     return out
 
 

@@ -102,7 +102,8 @@ def mask_build(sep, a, n, bm, bn):
           of query row t*bm; those anchors are kept by every row of query tile t,
       tile_map [B, T, U] int8: SKIP if no pair of the (t, u) block is kept, FULL if every
           in-bounds pair is kept, PARTIAL otherwise,
-      kept [B] int64: kept pairs.
+      kept [B] int64: kept pairs,
+      anchor_bits [B, ceil(L/32)] uint32: bit k of word w is f[32w + k] (0 past L).
     """
     sep = np.atleast_2d(np.asarray(sep))
     B, L = sep.shape
@@ -113,8 +114,13 @@ def mask_build(sep, a, n, bm, bn):
     gather_end = np.zeros((B, T), dtype=np.int32)
     tile_map = np.zeros((B, T, U), dtype=np.int8)
     kept = np.zeros(B, dtype=np.int64)
+    W = -(-L // 32)
+    anchor_bits = np.zeros((B, W), dtype=np.uint32)
     for b in range(B):
         f = anchor_flags(sep[b], a)
+        for j in range(L):
+            if f[j]:
+                anchor_bits[b, j // 32] |= np.uint32(1 << (j % 32))
         M = keep_mask(sep[b], a, n)
         pos = [j for j in range(L) if f[j]]
         anchor_idx[b, : len(pos)] = pos
@@ -133,7 +139,7 @@ def mask_build(sep, a, n, bm, bn):
                 else:
                     tile_map[b, t, u] = PARTIAL
     return dict(anchor_idx=anchor_idx, anchor_cnt=anchor_cnt, gather_end=gather_end,
-                tile_map=tile_map, kept=kept)
+                tile_map=tile_map, kept=kept, anchor_bits=anchor_bits)
 
 
 def _f64(x):

@@ -23,12 +23,14 @@ def _run(S, sep_np, a, n, bm, bn):
     m = S.sep_mask_build(sep, a, n, bm, bn)
     torch.cuda.synchronize()
     assert S.sep_last_device_error() == 0
-    return {k: getattr(m, k).cpu().numpy() for k in
-            ("anchor_idx", "anchor_cnt", "gather_end", "tile_map", "kept")}
+    out = {k: getattr(m, k).cpu().numpy() for k in
+           ("anchor_idx", "anchor_cnt", "gather_end", "tile_map", "kept")}
+    out["anchor_bits"] = m.anchor_bits.cpu().numpy().view(np.uint32)
+    return out
 
 
 def _compare(got, ref):
-    for k in ("anchor_idx", "anchor_cnt", "gather_end", "tile_map", "kept"):
+    for k in ("anchor_idx", "anchor_cnt", "gather_end", "tile_map", "kept", "anchor_bits"):
         np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
 
 
@@ -42,6 +44,7 @@ def test_golden_example(S):
         assert got["tile_map"][0, t].tolist() == row
     assert got["gather_end"][0].tolist() == g["gather_end"]
     assert int(got["kept"][0]) == g["kept_total"][0]
+    assert got["anchor_bits"][0].tolist() == g["anchor_bits"]
 
 
 @pytest.mark.parametrize("B,L,a,n,bm,bn,p", [
@@ -90,6 +93,10 @@ def test_long_context_sampled(S, n):
     lo = np.maximum(0, np.arange(T) * 128 - n + 1) // 128 * 128
     np.testing.assert_array_equal(got["gather_end"][0], np.searchsorted(pos, lo, side="left"))
     assert int(got["kept"][0]) == int(R.kept_pairs_closed_form(sep, cfg.a, n)[0])
+    fb = np.zeros(cfg.L // 32, dtype=np.uint64)
+    for k in range(32):
+        fb |= f.reshape(-1, 32)[:, k].astype(np.uint64) << np.uint64(k)
+    np.testing.assert_array_equal(got["anchor_bits"][0], fb.astype(np.uint32))
     rng = np.random.default_rng(0)
     tiles = [(0, 0), (T - 1, T - 1), (T - 1, 0), (T - 1, T - 3), (500, 498)]
     tiles += [(int(t), int(u)) for t, u in zip(rng.integers(0, T, 60), rng.integers(0, T, 60))]

@@ -43,6 +43,7 @@ def test_golden_artefacts():
         assert tm[t].tolist() == row, t
     assert art["gather_end"][0].tolist() == g["gather_end"]
     assert int(art["kept"][0]) == g["kept_total"][0]
+    assert art["anchor_bits"][0].tolist() == g["anchor_bits"]
 
 
 def _brute_kept(sep, a, n, i):

@@ -74,7 +74,7 @@ FwdWs fwd_ws(int B, int L, int Hkv, int d) {
   return w;
 }
 struct BwdWs {
-  size_t kc, vc, delta, dka, dva, total;
+  size_t kc, vc, delta, dka, dva, sched, total;
 };
 BwdWs bwd_ws(int B, int L, int Hq, int Hkv, int d) {
   BwdWs w;
@@ -86,7 +86,8 @@ BwdWs bwd_ws(int B, int L, int Hq, int Hkv, int d) {
   w.delta = 2 * kv;
   w.dka = w.delta + dl;
   w.dva = w.dka + kvf;
-  w.total = w.dva + kvf;
+  w.sched = w.dva + kvf;
+  w.total = w.sched + round_up(sep::bwd_sched_bytes(B, L), 256);
   return w;
 }
 
@@ -139,7 +140,7 @@ static int attn_fwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const
     std::memset(&maps, 0, sizeof(maps));
     if (!encode_map(&maps.q, q, B, L, Hq, d) || !encode_map(&maps.k, k, B, L, Hkv, d) ||
         !encode_map(&maps.v, v, B, L, Hkv, d) || !encode_map(&maps.kc, kc, B, L, Hkv, d) ||
-        !encode_map(&maps.vc, vc, B, L, Hkv, d))
+        !encode_map(&maps.vc, vc, B, L, Hkv, d) || !encode_map(&maps.o, o, B, L, Hq, d))
       return SEP_ERR_CUDA;
     AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
     return cuda_status(
@@ -192,13 +193,15 @@ static int attn_bwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const
   if (!encode_map(&maps.q, q, B, L, Hq, d) || !encode_map(&maps.k, k, B, L, Hkv, d) ||
       !encode_map(&maps.v, v, B, L, Hkv, d) || !encode_map(&maps.kc, kc, B, L, Hkv, d) ||
       !encode_map(&maps.vc, vc, B, L, Hkv, d) || !encode_map(&maps.o, o, B, L, Hq, d) ||
-      !encode_map(&maps.dout, dout, B, L, Hq, d))
+      !encode_map(&maps.dout, dout, B, L, Hq, d) || !encode_map(&maps.dq, dq, B, L, Hq, d) ||
+      !encode_map(&maps.dk, dk, B, L, Hkv, d) || !encode_map(&maps.dv, dv, B, L, Hkv, d))
     return SEP_ERR_CUDA;
   AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
   return cuda_status(sep::launch_attn_bwd(
       maps, sh, mask->anchor_bits, mask->anchor_idx, mask->anchor_cnt, mask->gather_end, mask->tile_map,
       o, lse, dout, q, k, v, dq, dk, dv, kc, vc, reinterpret_cast<float*>(ws + w.delta),
-      reinterpret_cast<float*>(ws + w.dka), reinterpret_cast<float*>(ws + w.dva), stages, s));
+      reinterpret_cast<float*>(ws + w.dka), reinterpret_cast<float*>(ws + w.dva), ws + w.sched,
+      stages, s));
 }
 
 int sep_attn_bwd(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, const sep_bf16* o,

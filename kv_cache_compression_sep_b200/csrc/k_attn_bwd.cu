@@ -30,7 +30,6 @@
 namespace sep {
 
 constexpr int kBoxBytes = 128 * 64 * 2;
-constexpr int kAnchorSeg = 16;  // query tiles per anchor-chunk CTA of the dK/dV kernel
 
 // ------------------------------------------------------------------ prep kernels
 __global__ void __launch_bounds__(256) zero_anchor_partials_kernel(
@@ -81,7 +80,7 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restr
 
 // ------------------------------------------------------------------ shared parameter block
 struct BwdParams {
-  CUtensorMap tmQ, tmK, tmV, tmKc, tmVc, tmdO;
+  CUtensorMap tmQ, tmK, tmV, tmKc, tmVc, tmdO, tmdQ, tmdK, tmdV;
   const uint32_t* anchor_bits;  // [B, W] packed anchor flags
   const int32_t* anchor_idx;
   const int32_t* anchor_cnt;
@@ -100,21 +99,27 @@ struct BwdParams {
 };
 
 // ------------------------------------------------------------------ dQ kernel
+// Query-major, persistent over a flattened key-tile stream (same item order and key tiles as
+// the forward). Per key tile: S = Q K^T and dP = dO V^T into TMEM; the softmax warpgroups
+// (two per row: key columns 64wg..64wg+63) form dS = P (dP - Delta) with P = exp2(S c - lse2)
+// and store it to TMEM as bf16; dQ += dS K (A from TMEM, B = K MN-major). The scaled dQ tile
+// leaves through shared memory and one TMA store.
 template <int D>
 struct DqCfg {
   static constexpr int KB = D / 64;
   static constexpr int TILE = KB * kBoxBytes;
-  static constexpr int NST = (D == 128) ? 2 : 4;
-  static constexpr int SMEM_TILES = TILE * (2 + 2 * NST);  // Q, dO, NST x (K, V)
-  static constexpr int COL_S = 0, COL_DP = 256, COL_DQ = 384;
+  static constexpr int NST = 2;
+  static constexpr int DOB = (D == 128) ? 1 : 2;               // dO buffers
+  static constexpr int SMEM_TILES = TILE * (2 + DOB + 2 * NST);  // Q x2, dO, NST x (K, V)
+  static constexpr int COL_S = 0, COL_DP = 128, COL_DQ = 256, COL_DS = 256 + D;
+  static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, dQ storer
 };
 
-template <int NST>
+template <int NST, int DOB>
 struct DqBar {
-  uint64_t q_full;
+  uint64_t q_full[2], q_empty[2], q_staged[2], do_full[DOB], do_empty[DOB];
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
-  uint64_t s_full[2], ds_ready[2], dq_done[2];
-  uint64_t dp_free;
+  uint64_t s_full, s_free, ds_ready, dq_done;
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -122,51 +127,89 @@ struct DqBar {
 
 template <int D>
 constexpr size_t dq_smem_bytes() {
-  return 1024 + DqCfg<D>::SMEM_TILES + sizeof(DqBar<DqCfg<D>::NST>);
+  return 1024 + DqCfg<D>::SMEM_TILES + sizeof(DqBar<DqCfg<D>::NST, DqCfg<D>::DOB>);
+}
+
+struct BwdItem {
+  int t, h, b, nwin, ge, N;
+};
+__device__ __forceinline__ BwdItem bwd_item_base(const BwdParams& p, int x) {
+  BwdItem it;
+  const int per_t = p.Hq * p.B;
+  it.t = p.T - 1 - x / per_t;
+  const int rem = x % per_t;
+  it.h = rem % p.Hq;
+  it.b = rem / p.Hq;
+  it.nwin = it.t - window_lo_tile(it.t, p.n) + 1;
+  it.ge = 0;
+  it.N = it.nwin;
+  return it;
+}
+__device__ __forceinline__ int bwd_item_ge(const BwdParams& p, int x) {
+  const BwdItem it = bwd_item_base(p, x);
+  return p.gather_end[(size_t)it.b * p.T + it.t];
+}
+__device__ __forceinline__ BwdItem bwd_item_with(const BwdParams& p, int x, int ge) {
+  BwdItem it = bwd_item_base(p, x);
+  it.ge = ge;
+  it.N = it.nwin + (ge + 127) / 128;
+  return it;
+}
+struct BwdTileRaw {
+  uint32_t fb[4];
+  int cls;
+};
+__device__ __forceinline__ BwdTileRaw bwd_tile_raw(const BwdParams& p, int b, int t, int u) {
+  BwdTileRaw r;
+  r.cls = p.tile_map[((size_t)b * p.T + t) * p.T + u];
+  const uint32_t* w = p.anchor_bits + (size_t)b * p.W + (size_t)u * 4;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) r.fb[q] = (u * 4 + q < p.W) ? __ldg(w + q) : 0u;
+  return r;
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) sep_attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
+    sep_attn_bwd_dq_kernel(const __grid_constant__ BwdParams p, int nitems) {
   using C = DqCfg<D>;
-  constexpr int NST = C::NST;
+  constexpr int NST = C::NST, DOB = C::DOB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + C::TILE;
-  uint8_t* sK = sdO + C::TILE;
+  uint8_t* sQ = smem;                 // 2 buffers (item parity), reused to stage dQ
+  uint8_t* sdO = sQ + 2 * C::TILE;    // DOB buffers (item % DOB)
+  uint8_t* sK = sdO + DOB * C::TILE;
   uint8_t* sV = sK + NST * C::TILE;
-  DqBar<NST>* bar = reinterpret_cast<DqBar<NST>*>(sV + NST * C::TILE);
+  DqBar<NST, DOB>* bar = reinterpret_cast<DqBar<NST, DOB>*>(sV + NST * C::TILE);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = p.T - 1 - (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int kvh = h / (p.Hq / p.Hkv);
-  const int lo_tile = window_lo_tile(t, p.n);
-  const int nwin = t - lo_tile + 1;
-  const int ge = p.gather_end[(size_t)b * p.T + t];
-  const int N = nwin + (ge + 127) / 128;
   volatile int* abort_flag = &bar->abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar->q_full[s], 1);
+      mbar_init(&bar->q_empty[s], 1);
+      mbar_init(&bar->q_staged[s], 256);
+    }
+    for (int s = 0; s < DOB; ++s) {
+      mbar_init(&bar->do_full[s], 1);
+      mbar_init(&bar->do_empty[s], 1);
+    }
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->ds_ready[s], 128);
-      mbar_init(&bar->dq_done[s], 1);
-    }
-    mbar_init(&bar->dp_free, 128);
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->s_free, 256);
+    mbar_init(&bar->ds_ready, 256);
+    mbar_init(&bar->dq_done, 1);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&bar->tmem_base, 512);
     tmem_relinquish();
   }
@@ -175,314 +218,479 @@ __global__ void __launch_bounds__(192, 1) sep_attn_bwd_dq_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bar->q_full, 2 * C::TILE);
-      for (int kb = 0; kb < C::KB; ++kb) {
-        tma_load_4d(sQ + kb * kBoxBytes, &p.tmQ, &bar->q_full, kb * 64, h, t * 128, b);
-        tma_load_4d(sdO + kb * kBoxBytes, &p.tmdO, &bar->q_full, kb * 64, h, t * 128, b);
-      }
-      for (int j = 0; j < N; ++j) {
-        const int st = j % NST, r = j / NST;
-        const bool win = j < nwin;
-        const int row0 = win ? (t - j) * 128 : (j - nwin) * 128;
-        if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag)) break;
-        mbar_arrive_expect_tx(&bar->k_full[st], C::TILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_4d(sK + st * C::TILE + kb * kBoxBytes, win ? &p.tmK : &p.tmKc,
-                      &bar->k_full[st], kb * 64, kvh, row0, b);
-        if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag)) {
-          mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
+      int g = 0;
+      bool ok = true;
+      int ge_cur = bwd_item_ge(p, blockIdx.x);
+      for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
+        const BwdItem it = bwd_item_with(p, x, ge_cur);
+        if (x + (int)gridDim.x < nitems) ge_cur = bwd_item_ge(p, x + gridDim.x);
+        const int kvh = it.h / (p.Hq / p.Hkv);
+        const int qb = k & 1;
+        if (k >= 2 && !mbar_wait(&bar->q_empty[qb], ((k - 2) >> 1) & 1, p.err, abort_flag)) {
+          ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&bar->v_full[st], C::TILE);
+        mbar_arrive_expect_tx(&bar->q_full[qb], C::TILE);
         for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_4d(sV + st * C::TILE + kb * kBoxBytes, win ? &p.tmV : &p.tmVc,
-                      &bar->v_full[st], kb * 64, kvh, row0, b);
+          tma_load_4d(sQ + qb * C::TILE + kb * kBoxBytes, &p.tmQ, &bar->q_full[qb], kb * 64, it.h,
+                      it.t * 128, it.b);
+        const int db = k % DOB;
+        for (int j = 0; j < it.N; ++j, ++g) {
+          if (j == 1 || (j == 0 && it.N == 1)) {
+            // dO of this item: after the first K/V tile is on its way (its buffer frees when the
+            // dP products of item k - DOB are done)
+            if (k >= DOB &&
+                !mbar_wait(&bar->do_empty[db], ((k - DOB) / DOB) & 1, p.err, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bar->do_full[db], C::TILE);
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_4d(sdO + db * C::TILE + kb * kBoxBytes, &p.tmdO, &bar->do_full[db],
+                          kb * 64, it.h, it.t * 128, it.b);
+          }
+          const int st = g % NST, r = g / NST;
+          const bool win = j < it.nwin;
+          const int row0 = win ? (it.t - j) * 128 : (j - it.nwin) * 128;
+          if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar->k_full[st], C::TILE);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_4d(sK + st * C::TILE + kb * kBoxBytes, win ? &p.tmK : &p.tmKc,
+                        &bar->k_full[st], kb * 64, kvh, row0, it.b);
+          if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag)) {
+            mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bar->v_full[st], C::TILE);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_4d(sV + st * C::TILE + kb * kBoxBytes, win ? &p.tmV : &p.tmVc,
+                        &bar->v_full[st], kb * 64, kvh, row0, it.b);
+        }
       }
-      if (*abort_flag) {
-        mbar_wait(&bar->q_full, 0, nullptr, nullptr);
-        for (int j = max(0, N - NST); j < N; ++j) {
-          mbar_wait(&bar->k_full[j % NST], (j / NST) & 1, nullptr, nullptr);
-          mbar_wait(&bar->v_full[j % NST], (j / NST) & 1, nullptr, nullptr);
+      if (!ok) {
+        for (int gg = max(0, g - NST); gg < g; ++gg) {
+          mbar_wait(&bar->k_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
+          mbar_wait(&bar->v_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t idQ = make_idesc_bf16(128, D, false, true);
       const uint32_t sQa = smem_u32(sQ), sdOa = smem_u32(sdO);
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
-      bool ok = mbar_wait(&bar->q_full, 0, p.err, abort_flag);
-      auto issue_SdP = [&](int j) -> bool {
-        const int st = j % NST;
-        if (!mbar_wait(&bar->k_full[st], (j / NST) & 1, p.err, abort_flag)) return false;
-        if (!mbar_wait(&bar->v_full[st], (j / NST) & 1, p.err, abort_flag)) return false;
-        // S[j%2] held dS_{j-2}, read by dQ_{j-2}
-        if (j >= 2 && !mbar_wait(&bar->dq_done[j & 1], ((j - 2) >> 1) & 1, p.err, abort_flag))
-          return false;
-        // dP was read by the softmax warps for tile j-1
-        if (j >= 1 && !mbar_wait(&bar->dp_free, (j - 1) & 1, p.err, abort_flag)) return false;
+      bool ok = true;
+      int g = 0, pend = -1, pend_first = 0;
+      auto issue_dQ = [&](int gg, int first) -> bool {
+        const int st = gg % NST;
+        if (!mbar_wait(&bar->ds_ready, gg & 1, p.err, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t dS = tmem + C::COL_S + (j & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(dS, make_sdesc_sw128(sQa + off, 16, 1024),
-                 make_sdesc_sw128(sKa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(sdOa + off, 16, 1024),
-                 make_sdesc_sw128(sVa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bar->s_full[j & 1]);
-        tc_commit(&bar->v_empty[st]);
-        return true;
-      };
-      auto issue_dQ = [&](int j) -> bool {
-        const int st = j % NST;
-        if (!mbar_wait(&bar->ds_ready[j & 1], (j >> 1) & 1, p.err, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t aS = tmem + C::COL_S + (j & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          mma_ts(tmem + C::COL_DQ, aS + kk * 8,
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + C::COL_DQ, tmem + C::COL_DS + kk * 8,
                  make_sdesc_sw128(sKa + st * C::TILE + kk * 2048, kBoxBytes, 1024), idQ,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bar->dq_done[j & 1]);
+                 (!first || kk > 0) ? 1u : 0u);
+        tc_commit(&bar->dq_done);
         tc_commit(&bar->k_empty[st]);
         return true;
       };
-      if (ok) ok = issue_SdP(0);
-      for (int j = 0; ok && j < N; ++j) {
-        if (j + 1 < N && !issue_SdP(j + 1)) break;
-        if (!issue_dQ(j)) break;
+      int ge_cur = bwd_item_ge(p, blockIdx.x);
+      for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
+        const BwdItem it = bwd_item_with(p, x, ge_cur);
+        if (x + (int)gridDim.x < nitems) ge_cur = bwd_item_ge(p, x + gridDim.x);
+        const int qb = k & 1, db = k % DOB;
+        if (!mbar_wait(&bar->q_full[qb], (k >> 1) & 1, p.err, abort_flag)) { ok = false; break; }
+        const uint32_t sQb = sQa + qb * C::TILE, sdOb = sdOa + db * C::TILE;
+        for (int j = 0; j < it.N; ++j, ++g) {
+          const int st = g % NST;
+          if (!mbar_wait(&bar->k_full[st], (g / NST) & 1, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bar->v_full[st], (g / NST) & 1, p.err, abort_flag)) { ok = false; break; }
+          if (g > 0 && !mbar_wait(&bar->s_free, (g - 1) & 1, p.err, abort_flag)) { ok = false; break; }
+          if (j == 0 && !mbar_wait(&bar->do_full[db], (k / DOB) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+            mma_ss(tmem + C::COL_S, make_sdesc_sw128(sQb + off, 16, 1024),
+                   make_sdesc_sw128(sKa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+            mma_ss(tmem + C::COL_DP, make_sdesc_sw128(sdOb + off, 16, 1024),
+                   make_sdesc_sw128(sVa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bar->s_full);
+          tc_commit(&bar->v_empty[st]);
+          if (j == it.N - 1) tc_commit(&bar->do_empty[db]);
+          if (pend >= 0 && !issue_dQ(pend, pend_first)) { ok = false; break; }
+          pend = g;
+          pend_first = (j == 0);
+        }
       }
+      if (ok && pend >= 0) issue_dQ(pend, pend_first);
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ dQ tile storer
+    if (lane == 0) {
+      bool ok = true;
+      for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
+        const BwdItem it = bwd_item_base(p, x);
+        if (!mbar_wait(&bar->q_staged[k & 1], (k >> 1) & 1, p.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* stage = sQ + (k & 1) * C::TILE;
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_store_4d(&p.tmdQ, stage + kb * kBoxBytes, kb * 64, it.h, it.t * 128, it.b);
+        bulk_commit_group();
+        bulk_wait_read_all();
+        mbar_arrive(&bar->q_empty[k & 1]);
+      }
+      bulk_wait_all();
+    }
   } else {
-    const int row = threadIdx.x;
-    const long long i = (long long)t * 128 + row;
-    const bool valid = i < p.L;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t* bits_row = p.anchor_bits + (size_t)b * p.W;
-    const int8_t* tmap = p.tile_map + ((size_t)b * p.T + t) * p.T;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int row = threadIdx.x & 127;
+    const int wg = threadIdx.x >> 7;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
-    const size_t rowstat = ((size_t)b * p.Hq + h) * p.L + (valid ? i : 0);
-    const float lse2 = valid ? p.lse[rowstat] * 1.4426950408889634f : INFINITY;
-    const float dlt = valid ? p.delta[rowstat] : 0.f;
     bool ok = true;
-    for (int j = 0; j < N; ++j) {
-      const int sb = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[sb], (j >> 1) & 1, p.err, abort_flag))) {
+    int g = 0, k_item = 0;
+    int ge_cur = bwd_item_ge(p, blockIdx.x);
+    BwdTileRaw cur;
+    {
+      const BwdItem f0 = bwd_item_base(p, blockIdx.x);
+      cur = bwd_tile_raw(p, f0.b, f0.t, f0.t);
+    }
+    for (int x = blockIdx.x; ok && x < nitems; x += gridDim.x) {
+      const BwdItem it = bwd_item_with(p, x, ge_cur);
+      const int xn = x + gridDim.x;
+      if (xn < nitems) ge_cur = bwd_item_ge(p, xn);
+      const long long i = (long long)it.t * 128 + row;
+      const bool valid = i < p.L;
+      const size_t rowstat = ((size_t)it.b * p.Hq + it.h) * p.L + (valid ? i : 0);
+      const float lse2 = valid ? p.lse[rowstat] * 1.4426950408889634f : INFINITY;
+      const float dlt = valid ? p.delta[rowstat] : 0.f;
+      for (int j = 0; j < it.N; ++j, ++g) {
+        const BwdTileRaw raw = cur;
+        if (j + 1 < it.nwin) {
+          cur = bwd_tile_raw(p, it.b, it.t, it.t - (j + 1));
+        } else if (j + 1 == it.N && xn < nitems) {
+          const BwdItem fn = bwd_item_base(p, xn);
+          cur = bwd_tile_raw(p, fn.b, fn.t, fn.t);
+        }
+        uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
+        if (j < it.nwin) {
+          const int u = it.t - j;
+          const long long k0 = (long long)u * 128;
+          if (raw.cls != SEP_TILE_FULL) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w)
+              keep[w] = window_keep_word(2 * wg + w, i, k0, p.n, p.L, raw.fb[2 * wg + w]);
+          } else if (k0 + 128 > p.L) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, 2 * wg + w);
+          }
+        } else {
+          const int rem = it.ge - (j - it.nwin) * 128;
+          if (rem < 128) {
+#pragma unroll
+            for (int w = 0; w < 2; ++w) keep[w] = range_word(0, rem - 1, 2 * wg + w);
+          }
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, g & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv[64], dp[64];
+        {
+          const uint32_t aS = tmem + lane_off + C::COL_S + wg * 64;
+          const uint32_t aP = tmem + lane_off + C::COL_DP + wg * 64;
+          tmem_ld32(aS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(aS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_ld32(aP, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+          tmem_ld32(aP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&bar->s_free);  // S and dP may be overwritten by the next tile's MMAs
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float v[2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const bool kp = (keep[(c + q) >> 5] >> ((c + q) & 31)) & 1u;
+            const float pr = kp ? ex2(fmaf(__uint_as_float(sv[c + q]), sl2, -lse2)) : 0.f;
+            v[q] = pr * (__uint_as_float(dp[c + q]) - dlt);
+          }
+          sv[c >> 1] = pack_bf16x2(v[0], v[1]);
+        }
+        // dS has one buffer: the previous tile's dQ MMA must have read it
+        if (g > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&bar->dq_done, (g - 1) & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem + lane_off + C::COL_DS + wg * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar->ds_ready);
+      }
+      if (!ok) break;
+      // ---- epilogue: scale * dQ as bf16 through the item's (free) Q buffer, one TMA store
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->dq_done, (g - 1) & 1, p.err, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (j < nwin) {
-        const int u = t - j;
-        const long long k0 = (long long)u * 128;
-        if (tmap[u] != SEP_TILE_FULL) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            keep[w] = window_keep_word(w, i, k0, p.n, p.L,
-                                       (u * 4 + w < p.W) ? __ldg(bits_row + u * 4 + w) : 0u);
-        } else if (k0 + 128 > p.L) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, w);
-        }
-      } else {
-        const int rem = ge - (j - nwin) * 128;
-        if (rem < 128) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) keep[w] = range_word(0, rem - 1, w);
-        }
-      }
-      const uint32_t aS = tmem + lane_off + C::COL_S + sb * 128;
-      const uint32_t aP = tmem + lane_off + C::COL_DP;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(aS + ch * 32, s);
-        tmem_ld32(aP + ch * 32, dp);
-        tmem_ld_wait();
-        if (ch == 3) {
-          tc_fence_before();
-          mbar_arrive(&bar->dp_free);
-        }
-        uint32_t ds[16];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float v[2];
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const bool kp = (keep[ch] >> (c + q)) & 1u;
-            const float pr = kp ? ex2(fmaf(__uint_as_float(s[c + q]), sl2, -lse2)) : 0.f;
-            v[q] = pr * (__uint_as_float(dp[c + q]) - dlt);
-          }
-          ds[c >> 1] = pack_bf16x2(v[0], v[1]);
-        }
-        // dS chunk ch lands in columns 16ch..16ch+15 of the S buffer (already read)
-        uint32_t (&d16)[16] = ds;
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-            "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aS + ch * 16),
-            "r"(d16[0]), "r"(d16[1]), "r"(d16[2]), "r"(d16[3]), "r"(d16[4]), "r"(d16[5]),
-            "r"(d16[6]), "r"(d16[7]), "r"(d16[8]), "r"(d16[9]), "r"(d16[10]), "r"(d16[11]),
-            "r"(d16[12]), "r"(d16[13]), "r"(d16[14]), "r"(d16[15])
-            : "memory");
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bar->ds_ready[sb]);
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&bar->dq_done[(N - 1) & 1], ((N - 1) >> 1) & 1,
-                                                p.err, abort_flag))) {
-      tc_fence_after();
-      __nv_bfloat16* drow = p.dq + (((size_t)b * p.L + (valid ? i : 0)) * p.Hq + h) * D;
+      uint8_t* stage = sQ + (k_item & 1) * C::TILE;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::COL_DQ + cc * 32, v);
+        tmem_ld32(tmem + lane_off + C::COL_DQ + wg * (D / 2) + cc * 32, v);
         tmem_ld_wait();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(drow + cc * 32);
+        uint32_t pkd[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w4[4];
+        for (int q = 0; q < 16; ++q)
+          pkd[q] = pack_bf16x2(__uint_as_float(v[2 * q]) * p.scale,
+                               __uint_as_float(v[2 * q + 1]) * p.scale);
+        const int col0 = wg * (D / 2) + cc * 32;
+        uint8_t* box = stage + (col0 >> 6) * kBoxBytes;
 #pragma unroll
-            for (int z = 0; z < 4; ++z)
-              w4[z] = pack_bf16x2(__uint_as_float(v[8 * q + 2 * z]) * p.scale,
-                                  __uint_as_float(v[8 * q + 2 * z + 1]) * p.scale);
-            dst[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(box + sw128_offset(row, ((col0 & 63) >> 3) + q)) =
+              make_uint4(pkd[4 * q], pkd[4 * q + 1], pkd[4 * q + 2], pkd[4 * q + 3]);
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar->q_staged[k_item & 1]);  // the storer warp writes the tile out
+      ++k_item;
     }
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
+// ------------------------------------------------------------------ dK/dV work list
+// Items of the key-major pass, one per (key unit, segment of query tiles):
+//   window item: key tile u of batch b with query tiles t_begin..t_end-1 (those whose window key
+//                tiles lo(t)..t contain u), split into segments of at most kSegT tiles;
+//   anchor item: compacted anchor chunk c (anchors 128c..128c+127) with the query tiles that
+//                gather it (gather_end[t] > 128c), in segments of kSegT tiles.
+// Every kv head processes every item. Built on the device by bwd_schedule_kernel.
+constexpr int kSegT = 16;
+
+struct WorkItem {
+  int b, unit, t_begin, t_end;  // unit: key tile u (window) or anchor chunk c
+};
+
+// One CTA per batch element: per-key-tile anchor prefix counts, then the anchor and window items.
+__global__ void __launch_bounds__(1024) bwd_schedule_kernel(
+    const int32_t* __restrict__ anchor_cnt, const int32_t* __restrict__ gather_end,
+    const uint32_t* __restrict__ anchor_bits, int L, int n, int T, int W, int32_t* __restrict__ tile_prefix,
+    WorkItem* __restrict__ anchor_items, WorkItem* __restrict__ window_items,
+    int32_t* __restrict__ counters /* [0] anchor items, [1] window items */) {
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  __shared__ int s_warp[32];
+  __shared__ int s_carry;
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  // ---- exclusive prefix over key tiles of the anchor counts
+  for (int base = 0; base < T; base += blockDim.x) {
+    const int u = base + tid;
+    int c = 0;
+    if (u < T) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (u * 4 + q < W) c += __popc(anchor_bits[(size_t)b * W + u * 4 + q]);
+    }
+    int incl = c;
+    const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int wv = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+      int wi = wv;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += y;
+      }
+      if (lane < (int)(blockDim.x >> 5)) s_warp[lane] = wi - wv;
+    }
+    __syncthreads();
+    const int carry = s_carry;
+    if (u < T) tile_prefix[(size_t)b * T + u] = carry + s_warp[warp] + incl - c;
+    __syncthreads();
+    if (tid == blockDim.x - 1) s_carry = carry + s_warp[warp] + incl;
+    __syncthreads();
+  }
+  // ---- anchor items
+  const int cnt = anchor_cnt[b];
+  const int nch = (cnt + 127) / 128;
+  const int32_t* ge = gather_end + (size_t)b * T;
+  for (int c = tid; c < nch; c += blockDim.x) {
+    int lo = 0, hi = T;  // first query tile that gathers anchor 128c
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (ge[mid] > c * 128) hi = mid; else lo = mid + 1;
+    }
+    const int nseg = (T - lo + kSegT - 1) / kSegT;
+    if (nseg > 0) {
+      const int at = atomicAdd(&counters[0], nseg);
+      for (int sg = 0; sg < nseg; ++sg) {
+        const int t0 = lo + sg * kSegT;
+        anchor_items[at + sg] = WorkItem{b, c, t0, min(T, t0 + kSegT)};
+      }
+    }
+  }
+  // ---- window items: query tiles t with lo(t) <= u <= t, in segments
+  for (int u = tid; u < T; u += blockDim.x) {
+    int te = u + 1;
+    while (te < T && window_lo_tile(te, n) <= u) ++te;
+    const int nseg = (te - u + kSegT - 1) / kSegT;
+    const int at = atomicAdd(&counters[1], nseg);
+    for (int sg = 0; sg < nseg; ++sg) {
+      const int t0 = u + sg * kSegT;
+      window_items[at + sg] = WorkItem{b, u, t0, min(te, t0 + kSegT)};
+    }
+  }
+}
+
 // ------------------------------------------------------------------ dK/dV kernel
+// Key-major, persistent over the work list (anchor items first, then window items; every kv
+// head of an item in turn). Per (query tile, query head) pair the query tile is split in two
+// 64-row halves h = 0, 1, each owned by one softmax warpgroup (thread = key row = TMEM lane):
+//   S^T_h = K Q_h^T, dP^T_h = V dO_h^T            (M = 128 keys, N = 64 queries)
+//   P^T = exp2(S^T c - lse2), dS^T = P^T (dP^T - Delta), written over S^T_h / dP^T_h as bf16
+//   dV += P^T_h dO_h, dK += dS^T_h Q_h             (A from TMEM, B MN-major in smem)
+// The MMA warp issues one half's S^T/dP^T while the other half's softmax runs. dV and dK stay
+// in TMEM for the whole item. Epilogue, with `direct` set (every window item covers all query
+// tiles of its key tile): non-anchor rows are final and leave as bf16 through shared memory and
+// a TMA store; anchor rows add their fp32 window part into the compact anchor partials. Anchor
+// items add into the compact partials. Without `direct` (long windows split into segments) every
+// row adds into position-indexed fp32 accumulators.
 template <int D>
 struct DkvCfg {
   static constexpr int KB = D / 64;
   static constexpr int TILE = KB * kBoxBytes;
-  static constexpr int NST = 2;
-  static constexpr int SMEM_TILES = TILE * (2 + 2 * NST);  // K, V, NST x (Q, dO)
-  static constexpr int COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr int KVB = (D == 128) ? 1 : 2;  // K/V buffers (items in flight)
+  static constexpr int NST = (D == 128) ? 2 : 3;  // Q/dO stages (pairs in flight)
+  static constexpr int SMEM_TILES = TILE * (2 * KVB + 2 * NST);
+  static constexpr int COL_S0 = 0;     // half h: S^T at 128h, dP^T at 128h + 64
+  static constexpr int COL_DV = 256, COL_DK = 256 + D;
+  static constexpr int THREADS = 320;
 };
 
-template <int NST>
+template <int NST, int KVB>
 struct DkvBar {
-  uint64_t kv_full;
+  uint64_t kv_full[KVB], kv_empty[KVB];
   uint64_t q_full[NST], q_empty[NST];
-  uint64_t s_full, pds_ready, mm_done;
+  uint64_t s_full[2], pds_ready[2], mm_done[2];
+  uint64_t acc_full, acc_free;
   uint64_t drain;
   float lse2[NST][128];
   float delta[NST][128];
-  int anchor_before;  // anchors at positions < 128u (window items)
-  int warp_anchor[4];
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int D>
 constexpr size_t dkv_smem_bytes() {
-  return 1024 + DkvCfg<D>::SMEM_TILES + sizeof(DkvBar<DkvCfg<D>::NST>);
+  return 1024 + DkvCfg<D>::SMEM_TILES + sizeof(DkvBar<DkvCfg<D>::NST, DkvCfg<D>::KVB>);
 }
 
-__device__ __forceinline__ int count_lt_dev(const int32_t* __restrict__ idx, int cnt, long long x) {
-  int lo = 0, hi = cnt;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if ((long long)idx[mid] < x)
-      lo = mid + 1;
-    else
-      hi = mid;
-  }
-  return lo;
+struct DkvItem {
+  int b, unit, t_begin, t_end;
+  bool window;
+  int kvh, npairs;
+};
+
+__device__ __forceinline__ DkvItem dkv_item(const BwdParams& p, const WorkItem* aitems,
+                                           const WorkItem* witems, int n_anchor, int x, int G) {
+  DkvItem it;
+  it.kvh = x % p.Hkv;
+  const int e = x / p.Hkv;
+  const WorkItem w = (e < n_anchor) ? aitems[e] : witems[e - n_anchor];
+  it.window = e >= n_anchor;
+  it.b = w.b;
+  it.unit = w.unit;
+  it.t_begin = w.t_begin;
+  it.t_end = w.t_end;
+  it.npairs = (w.t_end - w.t_begin) * G;
+  return it;
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) sep_attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p,
-                                                                 int nseg) {
+__global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
+    sep_attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p, const WorkItem* __restrict__ aitems,
+                            const WorkItem* __restrict__ witems,
+                            const int32_t* __restrict__ counters,
+                            const int32_t* __restrict__ tile_prefix, int direct) {
   using C = DkvCfg<D>;
-  constexpr int NST = C::NST;
+  constexpr int NST = C::NST, KVB = C::KVB;
   const int G = p.Hq / p.Hkv;
-  const int kvh = blockIdx.y, b = blockIdx.z;
-  const int item = blockIdx.x;
-  const int cnt = p.anchor_cnt[b];
-  const int32_t* ge_row = p.gather_end + (size_t)b * p.T;
-
-  // ---- which key rows and which query tiles this CTA handles
-  bool window;
-  int u = 0, c = 0, t_begin, t_end;
-  if (item < p.T) {
-    window = true;
-    u = p.T - 1 - item;
-    t_begin = u;
-    t_end = u;
-    while (t_end + 1 < p.T && window_lo_tile(t_end + 1, p.n) <= u) ++t_end;
-    ++t_end;
-  } else {
-    window = false;
-    const int x = item - p.T;
-    c = x / nseg;
-    const int sg = x % nseg;
-    if (c * 128 >= cnt) return;
-    // first query tile that gathers anchor 128c: gather_end is non-decreasing in t
-    int lo = 0, hi = p.T;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (ge_row[mid] > c * 128)
-        hi = mid;
-      else
-        lo = mid + 1;
-    }
-    t_begin = lo + sg * kAnchorSeg;
-    t_end = min(p.T, t_begin + kAnchorSeg);
-    if (t_begin >= p.T) return;
-  }
-  const int npairs = (t_end - t_begin) * G;
+  const int n_anchor = counters[0];
+  const int nitems = (n_anchor + counters[1]) * p.Hkv;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sK = smem;
-  uint8_t* sV = sK + C::TILE;
-  uint8_t* sQ = sV + C::TILE;
-  uint8_t* sdO = sQ + NST * C::TILE;
-  DkvBar<NST>* bar = reinterpret_cast<DkvBar<NST>*>(sdO + NST * C::TILE);
+  uint8_t* sK = smem;                       // KVB buffers
+  uint8_t* sV = sK + KVB * C::TILE;         // KVB buffers
+  uint8_t* sQ = sV + KVB * C::TILE;         // NST stages
+  uint8_t* sdO = sQ + NST * C::TILE;        // NST stages
+  DkvBar<NST, KVB>* bar = reinterpret_cast<DkvBar<NST, KVB>*>(sdO + NST * C::TILE);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bar->abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bar->kv_full, 1);
+    for (int s = 0; s < KVB; ++s) {
+      mbar_init(&bar->kv_full[s], 1);
+      mbar_init(&bar->kv_empty[s], 1);
+    }
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar->q_full[s], 1 + 32);
       mbar_init(&bar->q_empty[s], 1);
     }
-    mbar_init(&bar->s_full, 1);
-    mbar_init(&bar->pds_ready, 128);
-    mbar_init(&bar->mm_done, 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bar->s_full[h], 1);
+      mbar_init(&bar->pds_ready[h], 128);
+      mbar_init(&bar->mm_done[h], 1);
+    }
+    mbar_init(&bar->acc_full, 1);
+    mbar_init(&bar->acc_free, 256);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
-    bar->anchor_before = window ? count_lt_dev(p.anchor_idx + (size_t)b * p.L, cnt, (long long)u * 128) : 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&bar->tmem_base, 512);
     tmem_relinquish();
   }
@@ -491,242 +699,338 @@ __global__ void __launch_bounds__(192, 1) sep_attn_bwd_dkv_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 4) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bar->kv_full, 2 * C::TILE);
-      const int krow = window ? u * 128 : c * 128;
-      for (int kb = 0; kb < C::KB; ++kb) {
-        tma_load_4d(sK + kb * kBoxBytes, window ? &p.tmK : &p.tmKc, &bar->kv_full, kb * 64, kvh,
-                    krow, b);
-        tma_load_4d(sV + kb * kBoxBytes, window ? &p.tmV : &p.tmVc, &bar->kv_full, kb * 64, kvh,
-                    krow, b);
-      }
-    }
-    for (int q = 0; q < npairs; ++q) {
-      const int st = q % NST, r = q / NST;
-      const int t = t_begin + q / G, h = kvh * G + q % G;
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer (whole warp)
+    int P = 0;
+    bool ok = true;
+    for (int I = 0, x = blockIdx.x; ok && x < nitems; ++I, x += gridDim.x) {
+      const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+      const int kb = I % KVB;
       bool okw = true;
-      if (r > 0) okw = mbar_wait(&bar->q_empty[st], (r - 1) & 1, p.err, abort_flag);
-      if (!__all_sync(0xffffffffu, okw)) break;
+      if (I >= KVB) okw = mbar_wait(&bar->kv_empty[kb], ((I - KVB) / KVB) & 1, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bar->q_full[st], 2 * C::TILE);
-        for (int kb = 0; kb < C::KB; ++kb) {
-          tma_load_4d(sQ + st * C::TILE + kb * kBoxBytes, &p.tmQ, &bar->q_full[st], kb * 64, h,
-                      t * 128, b);
-          tma_load_4d(sdO + st * C::TILE + kb * kBoxBytes, &p.tmdO, &bar->q_full[st], kb * 64, h,
-                      t * 128, b);
+        mbar_arrive_expect_tx(&bar->kv_full[kb], 2 * C::TILE);
+        const int krow = it.unit * 128;
+        for (int q = 0; q < C::KB; ++q) {
+          tma_load_4d(sK + kb * C::TILE + q * kBoxBytes, it.window ? &p.tmK : &p.tmKc,
+                      &bar->kv_full[kb], q * 64, it.kvh, krow, it.b);
+          tma_load_4d(sV + kb * C::TILE + q * kBoxBytes, it.window ? &p.tmV : &p.tmVc,
+                      &bar->kv_full[kb], q * 64, it.kvh, krow, it.b);
         }
       }
-      // per-query statistics of this tile: log2-domain lse (+inf past L) and Delta
-      const size_t base = ((size_t)b * p.Hq + h) * p.L;
+      for (int q = 0; q < it.npairs; ++q, ++P) {
+        const int st = P % NST, r = P / NST;
+        const int t = it.t_begin + q / G, h = it.kvh * G + q % G;
+        okw = true;
+        if (r > 0) okw = mbar_wait(&bar->q_empty[st], (r - 1) & 1, p.err, abort_flag);
+        if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar->q_full[st], 2 * C::TILE);
+          for (int z = 0; z < C::KB; ++z) {
+            tma_load_4d(sQ + st * C::TILE + z * kBoxBytes, &p.tmQ, &bar->q_full[st], z * 64, h,
+                        t * 128, it.b);
+            tma_load_4d(sdO + st * C::TILE + z * kBoxBytes, &p.tmdO, &bar->q_full[st], z * 64, h,
+                        t * 128, it.b);
+          }
+        }
+        // per-query statistics: log2-domain lse (+inf past L: P = 0 there) and Delta
+        const size_t base = ((size_t)it.b * p.Hq + h) * p.L;
 #pragma unroll
-      for (int z = 0; z < 4; ++z) {
-        const int col = lane * 4 + z;
-        const long long i = (long long)t * 128 + col;
-        const bool v = i < p.L;
-        bar->lse2[st][col] = v ? p.lse[base + i] * 1.4426950408889634f : INFINITY;
-        bar->delta[st][col] = v ? p.delta[base + i] : 0.f;
+        for (int z = 0; z < 4; ++z) {
+          const int col = lane * 4 + z;
+          const long long i = (long long)t * 128 + col;
+          const bool v = i < p.L;
+          bar->lse2[st][col] = v ? __ldg(p.lse + base + i) * 1.4426950408889634f : INFINITY;
+          bar->delta[st][col] = v ? __ldg(p.delta + base + i) : 0.f;
+        }
+        mbar_arrive(&bar->q_full[st]);
       }
-      mbar_arrive(&bar->q_full[st]);
     }
-    if (lane == 0 && *abort_flag) {
-      mbar_wait(&bar->kv_full, 0, nullptr, nullptr);
-      for (int q = max(0, npairs - NST); q < npairs; ++q)
-        mbar_wait(&bar->q_full[q % NST], (q / NST) & 1, nullptr, nullptr);
+    if (lane == 0 && !ok) {
+      for (int pp = max(0, P - NST); pp < P; ++pp)
+        mbar_wait(&bar->q_full[pp % NST], (pp / NST) & 1, nullptr, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = make_idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idS = make_idesc_bf16(128, 64, false, false);
       constexpr uint32_t idG = make_idesc_bf16(128, D, false, true);
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t sQa = smem_u32(sQ), sdOa = smem_u32(sdO);
-      bool ok = mbar_wait(&bar->kv_full, 0, p.err, abort_flag);
-      for (int q = 0; ok && q < npairs; ++q) {
-        const int st = q % NST;
-        if (!mbar_wait(&bar->q_full[st], (q / NST) & 1, p.err, abort_flag)) break;
-        // S^T / dP^T columns are read (as P^T / dS^T) by the previous pair's gradient MMAs
-        if (q > 0 && !mbar_wait(&bar->mm_done, (q - 1) & 1, p.err, abort_flag)) break;
-        tc_fence_after();
+      bool ok = true;
+      int P = 0;
+      for (int I = 0, x = blockIdx.x; ok && x < nitems; ++I, x += gridDim.x) {
+        const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+        const int kb = I % KVB;
+        if (!mbar_wait(&bar->kv_full[kb], (I / KVB) & 1, p.err, abort_flag)) { ok = false; break; }
+        const uint32_t kA = sKa + kb * C::TILE, vA = sVa + kb * C::TILE;
+        for (int q = 0; q < it.npairs && ok; ++q, ++P) {
+          const int st = P % NST;
+          if (!mbar_wait(&bar->q_full[st], (P / NST) & 1, p.err, abort_flag)) { ok = false; break; }
+          const uint32_t qA = sQa + st * C::TILE, dA = sdOa + st * C::TILE;
+          // S^T and dP^T of both halves; a half's buffers hold the previous pair's P^T/dS^T
+          // until that pair's dV/dK products are done
+          for (int h = 0; h < 2; ++h) {
+            if (P > 0 && !mbar_wait(&bar->mm_done[h], (P - 1) & 1, p.err, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t cS = tmem + 128 * h, cP = cS + 64;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::COL_S, make_sdesc_sw128(sKa + off, 16, 1024),
-                 make_sdesc_sw128(sQa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-        }
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+              const uint32_t qoff = (kk >> 2) * kBoxBytes + h * 64 * 128 + (kk & 3) * 32;
+              mma_ss(cS, make_sdesc_sw128(kA + off, 16, 1024),
+                     make_sdesc_sw128(qA + qoff, 16, 1024), idS, kk > 0 ? 1u : 0u);
+              mma_ss(cP, make_sdesc_sw128(vA + off, 16, 1024),
+                     make_sdesc_sw128(dA + qoff, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bar->s_full[h]);
+          }
+          if (!ok) break;
+          // the first dV/dK product of an item overwrites the accumulators: the previous
+          // item's epilogue must have read them
+          if (q == 0 && I > 0 && !mbar_wait(&bar->acc_free, (I - 1) & 1, p.err, abort_flag)) {
+            ok = false;
+            break;
+          }
+          for (int h = 0; h < 2; ++h) {
+            if (!mbar_wait(&bar->pds_ready[h], P & 1, p.err, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t cS = tmem + 128 * h, cP = cS + 64;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::COL_DP, make_sdesc_sw128(sVa + off, 16, 1024),
-                 make_sdesc_sw128(sdOa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 64 / 16; ++kk) {
+              const uint32_t roff = (h * 64 + kk * 16) * 128;
+              const uint32_t acc = (q > 0 || h > 0 || kk > 0) ? 1u : 0u;
+              mma_ts(tmem + C::COL_DV, cS + kk * 8, make_sdesc_sw128(dA + roff, kBoxBytes, 1024),
+                     idG, acc);
+              mma_ts(tmem + C::COL_DK, cP + kk * 8, make_sdesc_sw128(qA + roff, kBoxBytes, 1024),
+                     idG, acc);
+            }
+            tc_commit(&bar->mm_done[h]);
+          }
+          if (!ok) break;
+          tc_commit(&bar->q_empty[st]);
         }
-        tc_commit(&bar->s_full);
-        if (!mbar_wait(&bar->pds_ready, q & 1, p.err, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
-                 make_sdesc_sw128(sdOa + st * C::TILE + kk * 2048, kBoxBytes, 1024), idG,
-                 (q > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
-                 make_sdesc_sw128(sQa + st * C::TILE + kk * 2048, kBoxBytes, 1024), idG,
-                 (q > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bar->mm_done);
-        tc_commit(&bar->q_empty[st]);
+        if (!ok) break;
+        tc_commit(&bar->acc_full);
       }
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }
   } else {
-    // ---------------------------------------------------------------- softmax warps (thread = key)
-    const int krow = threadIdx.x;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int h = threadIdx.x >> 7;      // query half owned by this warpgroup
+    const int krow = threadIdx.x & 127;  // key row = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float sl2 = p.scale_log2;
-    // this thread's key: position j (window) or compact anchor row r (gathered)
-    const long long j = window ? (long long)u * 128 + krow : -1;
-    const int r = window ? -1 : c * 128 + krow;
-    bool fj = false;
-    if (window && j < p.L) fj = (__ldg(p.anchor_bits + (size_t)b * p.W + (j >> 5)) >> (j & 31)) & 1u;
     bool ok = true;
-    for (int q = 0; q < npairs; ++q) {
-      const int st = q % NST;
-      const int t = t_begin + q / G;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, q & 1, p.err, abort_flag))) {
-        ok = false;
-        break;
+    int P = 0;
+    for (int I = 0, x = blockIdx.x; ok && x < nitems; ++I, x += gridDim.x) {
+      const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+      const int kb = I % KVB;
+      long long j = -1;  // key position (window items)
+      bool fj = false;
+      int r = -1;        // compact anchor row (anchor items)
+      uint32_t tile_words[4] = {0u, 0u, 0u, 0u};
+      if (it.window) {
+        j = (long long)it.unit * 128 + krow;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          tile_words[q] = (it.unit * 4 + q < p.W) ? __ldg(p.anchor_bits + (size_t)it.b * p.W + it.unit * 4 + q) : 0u;
+        fj = j < p.L && ((tile_words[krow >> 5] >> (krow & 31)) & 1u);
+      } else {
+        r = it.unit * 128 + krow;
       }
-      // q_full also covers the per-query statistics written by the producer warp
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->q_full[st], (q / NST) & 1, p.err, abort_flag))) {
+      const int* ge_row = p.gather_end + (size_t)it.b * p.T;
+      // loaded now, used at the epilogue
+      const int pre_tile = it.window ? __ldg(tile_prefix + (size_t)it.b * p.T + it.unit) : 0;
+      const int cnt_b = __ldg(p.anchor_cnt + it.b);
+      const int8_t* tm_col = p.tile_map + (size_t)it.b * p.T * p.T + it.unit;  // [t][u] at t * T
+      // per-pair mask input (tile class or gather count), loaded one pair ahead
+      int nxt = it.window ? (int)__ldg(tm_col + (size_t)it.t_begin * p.T) : __ldg(ge_row + it.t_begin);
+      for (int q = 0; q < it.npairs; ++q, ++P) {
+        const int st = P % NST;
+        const int t = it.t_begin + q / G;
+        const int cur = nxt;
+        if (q + 1 < it.npairs) {
+          const int tn = it.t_begin + (q + 1) / G;
+          nxt = it.window ? (int)__ldg(tm_col + (size_t)tn * p.T) : __ldg(ge_row + tn);
+        }
+        // keep bits over the 64 query columns of this half
+        uint32_t keep[2];
+        const long long q0 = (long long)t * 128 + 64 * h;
+        if (it.window) {
+          const int cls = cur;
+          if (j >= p.L) {
+            keep[0] = keep[1] = 0u;
+          } else if (cls == SEP_TILE_FULL) {
+            keep[0] = keep[1] = 0xffffffffu;
+          } else {  // query i keeps j iff i >= j and (i - j < n or f[j])
+            const long long lo = j - q0;
+            const long long hi = fj ? 63 : j + p.n - 1 - q0;
+            keep[0] = range_word(lo, hi, 0);
+            keep[1] = range_word(lo, hi, 1);
+          }
+        } else {
+          const uint32_t all = (r < cur) ? 0xffffffffu : 0u;
+          keep[0] = keep[1] = all;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[h], P & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        // q_full also covers the per-query statistics written by the producer warp
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->q_full[st], (P / NST) & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t aS = tmem + lane_off + 128 * h, aP = aS + 64;
+        const float* lse2 = &bar->lse2[st][64 * h];
+        const float* dl = &bar->delta[st][64 * h];
+        // two 32-column chunks; packed chunk c lands in columns 16c..16c+15, already read
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t sv[32], dp[32];
+          tmem_ld32(aS + 32 * ch, sv);
+          tmem_ld32(aP + 32 * ch, dp);
+          tmem_ld_wait();
+          uint32_t pk[16], dk16[16];
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int col = 32 * ch + c + z;
+              const bool kp = (keep[ch] >> (c + z)) & 1u;
+              const float pr = kp ? ex2(fmaf(__uint_as_float(sv[c + z]), sl2, -lse2[col])) : 0.f;
+              pv[z] = pr;
+              dv2[z] = pr * (__uint_as_float(dp[c + z]) - dl[col]);
+            }
+            pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
+            dk16[c >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+          }
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+              "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aS + 16 * ch),
+              "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+              "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
+              "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
+              : "memory");
+          asm volatile(
+              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+              "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aP + 16 * ch),
+              "r"(dk16[0]), "r"(dk16[1]), "r"(dk16[2]), "r"(dk16[3]), "r"(dk16[4]), "r"(dk16[5]),
+              "r"(dk16[6]), "r"(dk16[7]), "r"(dk16[8]), "r"(dk16[9]), "r"(dk16[10]),
+              "r"(dk16[11]), "r"(dk16[12]), "r"(dk16[13]), "r"(dk16[14]), "r"(dk16[15])
+              : "memory");
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bar->pds_ready[h]);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------------- item epilogue
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->acc_full, I & 1, p.err, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // keep bits over the 128 query columns of tile t for this key
-      uint32_t keep[4];
-      const long long q0 = (long long)t * 128;
-      if (window) {
-        const int cls = p.tile_map[((size_t)b * p.T + t) * p.T + u];
-        if (j >= p.L) {
+      // warpgroup 0 finishes dV, warpgroup 1 finishes dK (row krow of the key unit)
+      const float mul = h ? p.scale : 1.f;
+      const uint32_t col0 = h ? C::COL_DK : C::COL_DV;
+      float* part = h ? p.dka : p.dva;
+      long long dst_row = -1;  // fp32 accumulator row, or -1
+      bool stage_row = false;
+      if (direct) {
+        if (it.window) {
+          stage_row = true;
+          if (fj) {
+            int before = pre_tile;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) keep[w] = 0u;
-        } else if (cls == SEP_TILE_FULL) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) keep[w] = 0xffffffffu;
-        } else {
-          // query i keeps j iff i >= j and (i - j < n or f[j])
-          const long long lo = j - q0;
-          const long long hi = fj ? 127 : j + p.n - 1 - q0;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) keep[w] = range_word(lo, hi, w);
+            for (int q = 0; q < 4; ++q)
+              if (q < (krow >> 5)) before += __popc(tile_words[q]);
+            before += __popc(tile_words[krow >> 5] & ((1u << (krow & 31)) - 1u));
+            dst_row = before;
+          }
+        } else if (r < cnt_b) {
+          dst_row = r;
         }
       } else {
-        const uint32_t all = (r < ge_row[t]) ? 0xffffffffu : 0u;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) keep[w] = all;
+        if (it.window) {
+          if (j < p.L) dst_row = j;
+        } else if (r < cnt_b) {
+          dst_row = p.anchor_idx[(size_t)it.b * p.L + r];
+        }
       }
-      const float* lse2 = bar->lse2[st];
-      const float* dl = bar->delta[st];
-      const uint32_t aS = tmem + lane_off + C::COL_S;
-      const uint32_t aP = tmem + lane_off + C::COL_DP;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(aS + ch * 32, s);
-        tmem_ld32(aP + ch * 32, dp);
+      float* dst = dst_row >= 0 ? part + (((size_t)it.b * p.L + dst_row) * p.Hkv + it.kvh) * D : nullptr;
+      uint8_t* stage = (h ? sK : sV) + kb * C::TILE;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t acc[32];
+        tmem_ld32(tmem + lane_off + col0 + cc * 32, acc);
         tmem_ld_wait();
-        uint32_t pk[16], dk16[16];
+        if (dst) {
 #pragma unroll
-        for (int cc = 0; cc < 32; cc += 2) {
-          float pv[2], dv2[2];
-#pragma unroll
-          for (int z = 0; z < 2; ++z) {
-            const int col = ch * 32 + cc + z;
-            const bool kp = (keep[ch] >> (cc + z)) & 1u;
-            const float pr = kp ? ex2(fmaf(__uint_as_float(s[cc + z]), sl2, -lse2[col])) : 0.f;
-            pv[z] = pr;
-            dv2[z] = pr * (__uint_as_float(dp[cc + z]) - dl[col]);
-          }
-          pk[cc >> 1] = pack_bf16x2(pv[0], pv[1]);
-          dk16[cc >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+          for (int z = 0; z < 8; ++z)
+            atomicAdd(reinterpret_cast<float4*>(dst + cc * 32) + z,
+                      make_float4(__uint_as_float(acc[4 * z]) * mul, __uint_as_float(acc[4 * z + 1]) * mul,
+                                  __uint_as_float(acc[4 * z + 2]) * mul, __uint_as_float(acc[4 * z + 3]) * mul));
         }
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-            "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aS + ch * 16),
-            "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
-            "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
-            "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-            : "memory");
-        asm volatile(
-            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-            "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aP + ch * 16),
-            "r"(dk16[0]), "r"(dk16[1]), "r"(dk16[2]), "r"(dk16[3]), "r"(dk16[4]), "r"(dk16[5]),
-            "r"(dk16[6]), "r"(dk16[7]), "r"(dk16[8]), "r"(dk16[9]), "r"(dk16[10]),
-            "r"(dk16[11]), "r"(dk16[12]), "r"(dk16[13]), "r"(dk16[14]), "r"(dk16[15])
-            : "memory");
+        if (stage_row) {
+          // bf16 row into this item's K (dK) or V (dV) buffer, swizzled box layout
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 v4 = make_uint4(
+                pack_bf16x2(__uint_as_float(acc[8 * q]) * mul, __uint_as_float(acc[8 * q + 1]) * mul),
+                pack_bf16x2(__uint_as_float(acc[8 * q + 2]) * mul, __uint_as_float(acc[8 * q + 3]) * mul),
+                pack_bf16x2(__uint_as_float(acc[8 * q + 4]) * mul, __uint_as_float(acc[8 * q + 5]) * mul),
+                pack_bf16x2(__uint_as_float(acc[8 * q + 6]) * mul, __uint_as_float(acc[8 * q + 7]) * mul));
+            const int chunk16 = cc * 4 + q;  // 16-byte chunk of the row
+            *reinterpret_cast<uint4*>(stage + (chunk16 >> 3) * kBoxBytes +
+                                      sw128_offset(krow, chunk16 & 7)) = v4;
+          }
+        }
       }
-      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bar->pds_ready);
-    }
-    // ---- epilogue: dV and dK rows of this key
-    // compact index of this key if it is an anchor (window items): anchors before the tile plus
-    // anchors before it inside the tile
-    const unsigned ball = __ballot_sync(0xffffffffu, fj);
-    if (lane == 0) bar->warp_anchor[warp] = __popc(ball);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    int cidx = -1;
-    if (window && fj) {
-      int before = bar->anchor_before + __popc(ball & ((1u << lane) - 1u));
-      for (int w = 0; w < warp; ++w) before += bar->warp_anchor[w];
-      cidx = before;
-    } else if (!window && r < cnt) {
-      cidx = r;
-    }
-    if (ok && npairs > 0 &&
-        __all_sync(0xffffffffu, mbar_wait(&bar->mm_done, (npairs - 1) & 1, p.err, abort_flag))) {
-      tc_fence_after();
-      const bool write_direct = window && j < p.L && !fj;
-#pragma unroll 1
-      for (int part = 0; part < 2; ++part) {  // 0: dV, 1: dK
-        const float mul = part ? p.scale : 1.f;
-        const uint32_t col0 = part ? C::COL_DK : C::COL_DV;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + col0 + cc * 32, v);
-          tmem_ld_wait();
-          if (write_direct) {
-            __nv_bfloat16* dst = (part ? p.dk : p.dv) + (((size_t)b * p.L + j) * p.Hkv + kvh) * D + cc * 32;
-            uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-            for (int z = 0; z < 4; ++z) {
-              uint32_t w4[4];
-#pragma unroll
-              for (int y = 0; y < 4; ++y)
-                w4[y] = pack_bf16x2(__uint_as_float(v[8 * z + 2 * y]) * mul,
-                                    __uint_as_float(v[8 * z + 2 * y + 1]) * mul);
-              d4[z] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-          } else if (cidx >= 0) {
-            float* dst = (part ? p.dka : p.dva) + (((size_t)b * p.L + cidx) * p.Hkv + kvh) * D + cc * 32;
-#pragma unroll
-            for (int z = 0; z < 8; ++z) {
-              atomicAdd(reinterpret_cast<float4*>(dst) + z,
-                        make_float4(__uint_as_float(v[4 * z]) * mul, __uint_as_float(v[4 * z + 1]) * mul,
-                                    __uint_as_float(v[4 * z + 2]) * mul, __uint_as_float(v[4 * z + 3]) * mul));
-            }
+      mbar_arrive(&bar->acc_free);  // the next item may overwrite dV / dK
+      if (stage_row) fence_proxy_async_smem();
+      asm volatile("bar.sync 5, 256;" ::: "memory");
+      if (threadIdx.x == 0) {
+        if (direct && it.window) {
+          for (int z = 0; z < C::KB; ++z) {
+            tma_store_4d(&p.tmdV, sV + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
+            tma_store_4d(&p.tmdK, sK + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
           }
+          bulk_commit_group();
+          bulk_wait_read_all();
         }
+        mbar_arrive(&bar->kv_empty[kb]);
       }
     }
+    if (threadIdx.x == 0) bulk_wait_all();
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Position-indexed fp32 accumulators to bf16 dK / dV (used when window items are segmented).
+__global__ void __launch_bounds__(256) acc_to_bf16_kernel(const float4* __restrict__ dka,
+                                                          const float4* __restrict__ dva,
+                                                          long long n4, uint2* __restrict__ dk,
+                                                          uint2* __restrict__ dv) {
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n4;
+       e += (long long)gridDim.x * blockDim.x) {
+    const float4 x = dka[e], y = dva[e];
+    dk[e] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+    dv[e] = make_uint2(pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
   }
 }
 
@@ -753,27 +1057,84 @@ __global__ void __launch_bounds__(256) anchor_combine_kernel(
   }
 }
 
+size_t bwd_sched_bytes(int B, int L) {
+  const size_t T = (L + 127) / 128;
+  const size_t cap = (size_t)B * T * ((T + kSegT - 1) / kSegT);
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  return up(2 * sizeof(int32_t)) + up((size_t)B * T * sizeof(int32_t)) + 2 * up(cap * sizeof(WorkItem));
+}
+
+static int sm_count_dev() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+template <int D>
+static cudaError_t set_bwd_attrs() {
+  static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && attr_set[dev]) return cudaSuccess;
+  constexpr size_t smq = dq_smem_bytes<D>(), smkv = dkv_smem_bytes<D>();
+  static_assert(smq <= 227 * 1024 && smkv <= 227 * 1024, "shared memory budget");
+  if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<D>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<D>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
+    return e;
+  if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  return cudaSuccess;
+}
+
 cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint32_t* anchor_bits,
                             const int32_t* anchor_idx, const int32_t* anchor_cnt,
                             const int32_t* gather_end, const int8_t* tile_map, const void* o,
                             const float* lse, const void* dout, const void* q, const void* k,
                             const void* v, void* dq, void* dk, void* dv, void* kc, void* vc,
-                            float* delta, float* dka, float* dva, int stages,
+                            float* delta, float* dka, float* dva, void* sched, int stages,
                             cudaStream_t stream) {
   (void)q;
+  (void)tile_map;
   cudaError_t e = cudaSuccess;
+  const int T = (s.L + 127) / 128, W = (s.L + 31) / 32;
+  // window items are single segments (direct dK/dV stores) unless windows span > kSegT tiles
+  const int win_tiles = (s.n - 1 + 127) / 128 + 1;
+  const int direct = (win_tiles <= kSegT || T <= kSegT) ? 1 : 0;
+  // schedule region: counters, tile prefix counts, anchor items, window items
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t cap = (size_t)s.B * T * ((T + kSegT - 1) / kSegT);
+  uint8_t* sw = static_cast<uint8_t*>(sched);
+  int32_t* counters = reinterpret_cast<int32_t*>(sw);
+  int32_t* tile_prefix = reinterpret_cast<int32_t*>(sw + up(2 * sizeof(int32_t)));
+  WorkItem* aitems = reinterpret_cast<WorkItem*>(sw + up(2 * sizeof(int32_t)) + up((size_t)s.B * T * sizeof(int32_t)));
+  WorkItem* witems = aitems + up(cap * sizeof(WorkItem)) / sizeof(WorkItem);
+  const size_t acc_bytes = (size_t)s.B * s.L * s.Hkv * s.d * sizeof(float);
+
   if (stages & kBwdPrep) {
-  e = launch_compact_anchors(k, v, anchor_idx, anchor_cnt, s.B, s.L, s.Hkv, s.d, kc, vc, stream);
-  if (e != cudaSuccess) return e;
-  {
-    const int rowvec = s.Hkv * s.d / 4;
-    dim3 grid((s.L + 31) / 32, s.B);
-    zero_anchor_partials_kernel<<<grid, 256, 0, stream>>>(anchor_cnt, s.L, rowvec, 32,
-                                                          reinterpret_cast<float4*>(dka),
-                                                          reinterpret_cast<float4*>(dva));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  {
+    if ((e = launch_compact_anchors(k, v, anchor_idx, anchor_cnt, s.B, s.L, s.Hkv, s.d, kc, vc,
+                                    stream)) != cudaSuccess)
+      return e;
+    if (direct) {
+      const int rowvec = s.Hkv * s.d / 4;
+      dim3 grid((s.L + 31) / 32, s.B);
+      zero_anchor_partials_kernel<<<grid, 256, 0, stream>>>(anchor_cnt, s.L, rowvec, 32,
+                                                            reinterpret_cast<float4*>(dka),
+                                                            reinterpret_cast<float4*>(dva));
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
+      if ((e = cudaMemsetAsync(dka, 0, acc_bytes, stream)) != cudaSuccess) return e;
+      if ((e = cudaMemsetAsync(dva, 0, acc_bytes, stream)) != cudaSuccess) return e;
+    }
     const long long rows = (long long)s.B * s.L * s.Hq;
     const unsigned blocks = (unsigned)((rows + 255) / 256);
     if (s.d == 128)
@@ -785,7 +1146,10 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
                                                    static_cast<const __nv_bfloat16*>(dout), s.B,
                                                    s.L, s.Hq, delta);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+    if ((e = cudaMemsetAsync(counters, 0, 2 * sizeof(int32_t), stream)) != cudaSuccess) return e;
+    bwd_schedule_kernel<<<s.B, 1024, 0, stream>>>(anchor_cnt, gather_end, anchor_bits, s.L, s.n,
+                                                  T, W, tile_prefix, aitems, witems, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (!(stages & (kBwdDq | kBwdDkv))) return cudaSuccess;
   BwdParams prm;
@@ -795,6 +1159,9 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.tmKc = maps.kc;
   prm.tmVc = maps.vc;
   prm.tmdO = maps.dout;
+  prm.tmdQ = maps.dq;
+  prm.tmdK = maps.dk;
+  prm.tmdV = maps.dv;
   prm.anchor_bits = anchor_bits;
   prm.anchor_idx = anchor_idx;
   prm.anchor_cnt = anchor_cnt;
@@ -812,59 +1179,45 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.L = s.L;
   prm.Hq = s.Hq;
   prm.Hkv = s.Hkv;
-  prm.T = (s.L + 127) / 128;
-  prm.W = (s.L + 31) / 32;
+  prm.T = T;
+  prm.W = W;
   prm.a = s.a;
   prm.n = s.n;
   prm.scale = s.scale;
   prm.scale_log2 = s.scale * 1.4426950408889634f;
-  const int nseg = (prm.T + kAnchorSeg - 1) / kAnchorSeg;
-  const int nchunks = prm.T;  // anchor chunks of 128 rows: at most ceil(L / 128)
-  dim3 grid_q(prm.T, s.Hq, s.B);
-  dim3 grid_kv(prm.T + nchunks * nseg, s.Hkv, s.B);
+  const int nsm = sm_count_dev();
+  const int dq_items = T * s.Hq * s.B;
+  const int grid_q = dq_items < nsm ? dq_items : nsm;
   if (s.d == 128) {
-    constexpr size_t smq = dq_smem_bytes<128>(), smkv = dkv_smem_bytes<128>();
-    static_assert(smq <= 227 * 1024 && smkv <= 227 * 1024, "shared memory budget");
-    static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<128>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
-        return e;
-      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<128>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
-        return e;
-      if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
-    if (stages & kBwdDq) sep_attn_bwd_dq_kernel<128><<<grid_q, 192, smq, stream>>>(prm);
+    if ((e = set_bwd_attrs<128>()) != cudaSuccess) return e;
+    if (stages & kBwdDq)
+      sep_attn_bwd_dq_kernel<128><<<grid_q, DqCfg<128>::THREADS, dq_smem_bytes<128>(), stream>>>(prm, dq_items);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (stages & kBwdDkv) sep_attn_bwd_dkv_kernel<128><<<grid_kv, 192, smkv, stream>>>(prm, nseg);
+    if (stages & kBwdDkv)
+      sep_attn_bwd_dkv_kernel<128><<<nsm, DkvCfg<128>::THREADS, dkv_smem_bytes<128>(), stream>>>(
+          prm, aitems, witems, counters, tile_prefix, direct);
   } else {
-    constexpr size_t smq = dq_smem_bytes<64>(), smkv = dkv_smem_bytes<64>();
-    static_assert(smq <= 227 * 1024 && smkv <= 227 * 1024, "shared memory budget");
-    static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dq_kernel<64>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smq)) != cudaSuccess)
-        return e;
-      if ((e = cudaFuncSetAttribute(sep_attn_bwd_dkv_kernel<64>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smkv)) != cudaSuccess)
-        return e;
-      if (dev >= 0 && dev < 64) attr_set[dev] = true;
-    }
-    if (stages & kBwdDq) sep_attn_bwd_dq_kernel<64><<<grid_q, 192, smq, stream>>>(prm);
+    if ((e = set_bwd_attrs<64>()) != cudaSuccess) return e;
+    if (stages & kBwdDq)
+      sep_attn_bwd_dq_kernel<64><<<grid_q, DqCfg<64>::THREADS, dq_smem_bytes<64>(), stream>>>(prm, dq_items);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (stages & kBwdDkv) sep_attn_bwd_dkv_kernel<64><<<grid_kv, 192, smkv, stream>>>(prm, nseg);
+    if (stages & kBwdDkv)
+      sep_attn_bwd_dkv_kernel<64><<<nsm, DkvCfg<64>::THREADS, dkv_smem_bytes<64>(), stream>>>(
+          prm, aitems, witems, counters, tile_prefix, direct);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (stages & kBwdDkv) {
-    dim3 grid((s.L + 31) / 32, s.B);
-    anchor_combine_kernel<<<grid, 256, 0, stream>>>(anchor_idx, anchor_cnt, s.L, s.Hkv * s.d, 32,
-                                                    dka, dva, static_cast<__nv_bfloat16*>(dk),
-                                                    static_cast<__nv_bfloat16*>(dv));
+    if (direct) {
+      dim3 grid((s.L + 31) / 32, s.B);
+      anchor_combine_kernel<<<grid, 256, 0, stream>>>(anchor_idx, anchor_cnt, s.L, s.Hkv * s.d, 32,
+                                                      dka, dva, static_cast<__nv_bfloat16*>(dk),
+                                                      static_cast<__nv_bfloat16*>(dv));
+    } else {
+      const long long n4 = (long long)s.B * s.L * s.Hkv * s.d / 4;
+      acc_to_bf16_kernel<<<nsm * 8, 256, 0, stream>>>(
+          reinterpret_cast<const float4*>(dka), reinterpret_cast<const float4*>(dva), n4,
+          static_cast<uint2*>(dk), static_cast<uint2*>(dv));
+    }
   }
   return cudaGetLastError();
 }

@@ -33,7 +33,7 @@
 namespace sep {
 
 struct FwdParams {
-  CUtensorMap tmQ, tmK, tmV, tmKc, tmVc;
+  CUtensorMap tmQ, tmK, tmV, tmKc, tmVc, tmO;
   const uint32_t* anchor_bits;  // [B, W] packed anchor flags
   const int32_t* gather_end;
   const int8_t* tile_map;
@@ -50,21 +50,23 @@ struct FwdCfg {
   static constexpr int KB = D / 64;                 // 128-byte column boxes per row
   static constexpr int BOX_BYTES = 128 * 64 * 2;    // one [128 rows][64 cols] bf16 box
   static constexpr int TILE_BYTES = KB * BOX_BYTES; // one [128][D] tile
-  static constexpr int NST = (D == 128) ? 2 : 2;    // K/V pipeline stages
+  static constexpr int NST = (D == 128) ? 2 : 4;    // K/V pipeline stages
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * NST);  // Q x2, NST x (K, V)
   static constexpr int COL_S = 0;        // S: 128 fp32 columns
   static constexpr int COL_O = 128;      // O: D fp32 columns
   static constexpr int COL_P = 128 + D;  // P: 64 columns (bf16 pairs)
   static constexpr int TMEM_COLS = (COL_P + 64 <= 256) ? 256 : 512;
-  static constexpr int CTAS_PER_SM = (TMEM_COLS == 256) ? 2 : 1;
+  static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, O storer
 };
 
 template <int NST>
 struct FwdBar {
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2], o_staged[2];
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
   uint64_t s_full, s_free, p_ready, pv_done;
   uint64_t drain;
+  float xch[2][2][128];  // row-max halves exchanged by the two softmax warpgroups (by tile parity)
+  float xl[2][128];      // row-sum halves, exchanged once per item
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -118,8 +120,11 @@ __device__ __forceinline__ TileRaw load_tile_raw(const FwdParams& p, int b, int 
 // Persistent: CTA c handles items c, c + gridDim.x, ... Every role walks the same flattened
 // sequence of key tiles (g = 0, 1, ... over all its items), so pipeline phases carry across
 // item boundaries and the next item's loads and first MMA overlap the current item's tail.
+// Warps 0-7 run the softmax: warpgroup wg = 0, 1 handles key columns 64wg..64wg+63 of every
+// query row (thread = row = TMEM lane), so two warps per SM sub-partition share the
+// exponentials; warp 8 is the TMA producer, warp 9 the MMA issuer.
 template <int D>
-__global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     sep_attn_fwd_kernel(const __grid_constant__ FwdParams p, int nitems) {
   using C = FwdCfg<D>;
   constexpr int NST = C::NST;
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar->q_full[s], 1);
       mbar_init(&bar->q_empty[s], 1);
+      mbar_init(&bar->o_staged[s], 256);
     }
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bar->k_full[s], 1);
@@ -146,14 +152,14 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
       mbar_init(&bar->v_empty[s], 1);
     }
     mbar_init(&bar->s_full, 1);
-    mbar_init(&bar->s_free, 128);
-    mbar_init(&bar->p_ready, 128);
+    mbar_init(&bar->s_free, 256);
+    mbar_init(&bar->p_ready, 256);
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->drain, 1);
     bar->abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -162,7 +168,7 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&p.tmQ);
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = make_idesc_bf16(128, 128, false, false);
@@ -270,7 +276,6 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
           }
           tc_commit(&bar->s_full);
           tc_commit(&bar->k_empty[st]);
-          if (j == it.N - 1) tc_commit(&bar->q_empty[qb]);
           // P V of the previous tile, while the softmax warps work on this one
           if (pv_pending >= 0 && !issue_PV(pv_pending, pv_first)) { ok = false; break; }
           pv_pending = g;
@@ -281,13 +286,35 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ O tile storer
+    if (lane == 0) {
+      bool ok = true;
+      for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
+        const FwdItem it = fwd_item_base(p, x);
+        if (!mbar_wait(&bar->o_staged[k & 1], (k >> 1) & 1, p.err, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* stage = sQ + (k & 1) * C::TILE_BYTES;
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_store_4d(&p.tmO, stage + kb * C::BOX_BYTES, kb * 64, it.h, it.t * C::BM, it.b);
+        bulk_commit_group();
+        bulk_wait_read_all();  // the staging buffer may now take a later item's Q
+        mbar_arrive(&bar->q_empty[k & 1]);
+      }
+      bulk_wait_all();  // O stores complete before the CTA exits
+    }
   } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int row = threadIdx.x;  // 0..127 = TMEM lane
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int row = threadIdx.x & 127;  // query row = TMEM lane
+    const int wg = threadIdx.x >> 7;    // column half
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t pair_bar = 1 + (warp & 3);  // named barrier of warps w and w + 4 (64 threads)
     const float sl2 = p.scale_log2;
     bool ok = true;
     int g = 0;
+    int k_item = 0;  // this CTA's item counter (Q buffer parity)
     int ge_cur = fwd_item_ge(p, blockIdx.x);
     TileRaw cur;  // mask inputs of the next tile to process, loaded one tile ahead
     {
@@ -315,23 +342,17 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
           break;
         }
         tc_fence_after();
-        uint32_t s[128];
+        uint32_t s[64];
         {
-          uint32_t (&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-          uint32_t (&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-          uint32_t (&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-          uint32_t (&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
-          const uint32_t a0 = tmem + lane_off + C::COL_S;
-          tmem_ld32(a0, c0);
-          tmem_ld32(a0 + 32, c1);
-          tmem_ld32(a0 + 64, c2);
-          tmem_ld32(a0 + 96, c3);
+          const uint32_t a0 = tmem + lane_off + C::COL_S + wg * 64;
+          tmem_ld32(a0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+          tmem_ld32(a0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
           tmem_ld_wait();
         }
         tc_fence_before();
         mbar_arrive(&bar->s_free);  // S may be overwritten by the next tile's MMA
-        // ---- mask
-        uint32_t keep[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        // ---- mask of this thread's 64 columns (words 2wg, 2wg+1 of the tile)
+        uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
         bool masked = false;
         if (j < it.nwin) {
           const int u = it.t - j;
@@ -339,33 +360,43 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
           if (raw.cls != SEP_TILE_FULL) {
             masked = true;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) keep[w] = window_keep_word(w, i, k0, p.n, p.L, raw.fb[w]);
+            for (int w = 0; w < 2; ++w)
+              keep[w] = window_keep_word(2 * wg + w, i, k0, p.n, p.L, raw.fb[2 * wg + w]);
           } else if (k0 + C::BN > p.L) {
             masked = true;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, w);
+            for (int w = 0; w < 2; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, 2 * wg + w);
           }
         } else {
           const int rem = it.ge - (j - it.nwin) * C::BN;  // valid anchors in this chunk
           if (rem < C::BN) {
             masked = true;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) keep[w] = range_word(0, rem - 1, w);
+            for (int w = 0; w < 2; ++w) keep[w] = range_word(0, rem - 1, 2 * wg + w);
           }
         }
-        float mx = -INFINITY;
+        // ---- row max of the half (8 independent chains), exchanged with the other half
+        float mx8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
         if (masked) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
+          for (int c = 0; c < 64; ++c) {
             const float v = ((keep[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(s[c]) : -INFINITY;
             s[c] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
+            mx8[c & 7] = fmaxf(mx8[c & 7], v);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(s[c]));
+          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
         }
-        // ---- online max with lazy rescale (only when the max grows by more than 2^8)
+        const float mh = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        bar->xch[g & 1][wg][row] = mh;
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        const float mx = fmaxf(mh, bar->xch[g & 1][wg ^ 1][row]);
+        // ---- online max with lazy rescale (only when the max grows by more than 2^8); both
+        // halves of a row take the same decision from the same values
         const float m_tile = mx * sl2;
         float alpha = 1.0f;
         bool any_rescale = false;
@@ -381,18 +412,19 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
           }
         }
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        // ---- P = exp2(S * scale*log2e - m), row sum, packed to bf16 pairs in place over the
-        // already consumed S registers (pair c/2 <= c)
-        float sum = 0.f;
+        // ---- P = exp2(S * scale*log2e - m), partial row sum (8 chains), packed to bf16 pairs
+        // in place over the already consumed S registers (pair c/2 <= c)
+        float sum8[8];
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
+        for (int q = 0; q < 8; ++q) sum8[q] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
           const float e0 = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
           const float e1 = ex2(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
-          sum += e0 + e1;
+          sum8[(c >> 1) & 7] += e0 + e1;
           s[c >> 1] = pack_bf16x2(e0, e1);
         }
-        uint32_t* pk = s;
-        l_run += sum;
+        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         // P and O: the previous tile's P V must be complete (it read P and accumulated O)
         if (g > 0 &&
             !__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {
@@ -402,9 +434,9 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
         tc_fence_after();
         if (any_rescale) {
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
+          for (int cc = 0; cc < D / 64; ++cc) {
             uint32_t ov[32];
-            const uint32_t ao = tmem + lane_off + C::COL_O + cc * 32;
+            const uint32_t ao = tmem + lane_off + C::COL_O + wg * (D / 2) + cc * 32;
             tmem_ld32(ao, ov);
             tmem_ld_wait();
 #pragma unroll
@@ -412,52 +444,60 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::CTAS_PER_SM)
             tmem_st32(ao, ov);
           }
         }
-        {
-          const uint32_t ap = tmem + lane_off + C::COL_P;
-          tmem_st32(ap, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-          tmem_st32(ap + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-          tmem_st_wait();
-        }
+        tmem_st32(tmem + lane_off + C::COL_P + wg * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bar->p_ready);
       }
       if (!ok) break;
-      // ---- epilogue of this item: O / l, LSE (O is reused by the next item's first P V,
-      // which the MMA warp issues only after this thread's next p_ready arrive)
+      // ---- epilogue of this item: row sum of both halves, O / l, LSE (O is reused by the next
+      // item's first P V, which the MMA warp issues only after this thread's next p_ready)
+      // (its own slot: the next item's first row-max exchange may start before the other half
+      // has read this value; the next write here is an item later, after further pair barriers)
+      bar->xl[wg][row] = l_run;
+      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      const float l_tot = l_run + bar->xl[wg ^ 1][row];
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv_l = 1.0f / l_run;
+      const float inv_l = 1.0f / l_tot;
       const bool valid = i < p.L;
-      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.L + (valid ? i : 0)) * p.Hq + it.h) * D;
+      // O / l as bf16 into the item's Q buffer (every S MMA of the item has completed, so Q is
+      // no longer read), in the swizzled box layout, then one TMA store of the whole tile
+      uint8_t* stage = sQ + (k_item & 1) * C::TILE_BYTES;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t ov[32];
-        tmem_ld32(tmem + lane_off + C::COL_O + cc * 32, ov);
+        tmem_ld32(tmem + lane_off + C::COL_O + wg * (D / 2) + cc * 32, ov);
         tmem_ld_wait();
         uint32_t pkd[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q)
           pkd[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv_l,
                                __uint_as_float(ov[2 * q + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+        const int col0 = wg * (D / 2) + cc * 32;  // first column of these 32
+        uint8_t* box = stage + (col0 >> 6) * C::BOX_BYTES;
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(pkd[4 * q], pkd[4 * q + 1], pkd[4 * q + 2], pkd[4 * q + 3]);
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = ((col0 & 63) >> 3) + q;
+          *reinterpret_cast<uint4*>(box + sw128_offset(row, chunk)) =
+              make_uint4(pkd[4 * q], pkd[4 * q + 1], pkd[4 * q + 2], pkd[4 * q + 3]);
         }
       }
-      if (valid)
+      fence_proxy_async_smem();
+      mbar_arrive(&bar->o_staged[k_item & 1]);  // the storer warp writes the tile out
+      if (valid && wg == 0)
         p.lse[((size_t)it.b * p.Hq + it.h) * p.L + i] =
-            (m_run + __log2f(l_run)) * 0.69314718055994531f;
+            (m_run + __log2f(l_tot)) * 0.69314718055994531f;
+      ++k_item;
     }
     tc_fence_before();
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -520,7 +560,7 @@ static int sm_count() {
 template <int D>
 static cudaError_t launch_fwd_t(const FwdParams& prm, int T, int Hq, int B, cudaStream_t stream) {
   constexpr size_t smem = fwd_smem_bytes<D>();
-  static_assert(smem * FwdCfg<D>::CTAS_PER_SM <= 228 * 1024, "shared memory budget");
+  static_assert(smem <= 227 * 1024, "shared memory budget");
   static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -532,8 +572,8 @@ static cudaError_t launch_fwd_t(const FwdParams& prm, int T, int Hq, int B, cuda
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   const int nitems = T * Hq * B;
-  const int grid = std::min(nitems, sm_count() * FwdCfg<D>::CTAS_PER_SM);
-  sep_attn_fwd_kernel<D><<<grid, 192, smem, stream>>>(prm, nitems);
+  const int grid = std::min(nitems, sm_count());
+  sep_attn_fwd_kernel<D><<<grid, FwdCfg<D>::THREADS, smem, stream>>>(prm, nitems);
   return cudaGetLastError();
 }
 
@@ -546,6 +586,7 @@ cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.tmV = maps.v;
   prm.tmKc = maps.kc;
   prm.tmVc = maps.vc;
+  prm.tmO = maps.o;
   prm.anchor_bits = anchor_bits;
   prm.gather_end = gather_end;
   prm.tile_map = tile_map;

@@ -12,24 +12,20 @@
 // Slot storage per (sequence, KV head) is [c][d] with c = a + s + w: slots 0..a-1 initial,
 // a..a+s-1 separator ring, a+s..c-1 window ring. Keys are stored without rotation.
 //
-// Decode: one thread-block cluster of kSplit CTAs per (sequence, KV head). Each CTA streams a
-// contiguous range of ranks with 16 half-warps (one key per half-warp per step, 8 elements of
-// the row per lane, coalesced loads), rotates keys in registers (cos/sin advanced by a complex
-// recurrence from the table row of the first rank), keeps an online softmax per query head,
-// and combines: half-warps through shared memory, CTAs of the cluster through distributed
-// shared memory. No global scratch is used.
-#include <cooperative_groups.h>
+// Decode: one CTA per (sequence, KV head), all of them resident at once (4 per SM), so the
+// whole cache streams in a single wave. Each CTA streams its ranks through a shared-memory ring
+// filled by bulk copies, with 8 half-warps (one key per half-warp per step, the row spread over
+// 16 lanes), rotates keys in registers (cos/sin advanced by a complex recurrence from the table
+// row of the first rank), keeps an online softmax per query head, and combines its half-warps
+// through shared memory. No global scratch is used.
 #include <cuda_runtime.h>
 
 #include "sep_common.cuh"
 #include "sep_launch.h"
 
-namespace cg = cooperative_groups;
-
 namespace sep {
 
-constexpr int kSplit = 4;          // CTAs per cluster (per sequence and KV head)
-constexpr int kDecThreads = 256;   // 16 half-warps
+constexpr int kDecThreads = 128;   // 8 half-warps per CTA; one CTA per (sequence, KV head)
 constexpr int kHalfWarps = kDecThreads / 16;
 
 // ------------------------------------------------------------------ init
@@ -182,7 +178,7 @@ __device__ __forceinline__ void load_bf16_vec_smem(const __nv_bfloat16* p, float
 // first stages; afterwards the last warp to finish reading a stage refills it with the chunk
 // kStages further on, so no thread waits to issue. Half-warp hw handles ranks r0 + hw + 16k;
 // lane16 owns HP rotation pairs (k, k + d/2), k = lane16 * HP + e, of every row it reads.
-constexpr int kChunk = 32;
+constexpr int kChunk = 16;
 constexpr int kStages = 4;
 constexpr int kConsumerWarps = kDecThreads / 32;
 
@@ -196,7 +192,7 @@ struct DecSmem {
 };
 
 template <int D, int G>
-__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 2)
+__global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
     sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int w,
                            const __nv_bfloat16* __restrict__ k_slots,
                            const __nv_bfloat16* __restrict__ v_slots,
@@ -205,10 +201,9 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 2)
                            float* __restrict__ lse, float scale_log2, unsigned* err) {
   constexpr int HP = D / 32;       // rotation pairs per lane
   constexpr int HALF = D / 2;
-  const int split = blockIdx.x, kvh = blockIdx.y, seq = blockIdx.z;
+  const int kvh = blockIdx.x, seq = blockIdx.y;
   const int c = a + s + w;
   const int tid = threadIdx.x, lane16 = tid & 15, hw = tid >> 4, warp = tid >> 5;
-  cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(128) uint8_t dsm_raw[];
   DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
 
@@ -218,8 +213,7 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 2)
   const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
   const int occ = ninit + sep_cnt + win_cnt;
   const int mq = occ - 1;  // the query's own rank
-  const int per = (occ + kSplit - 1) / kSplit;
-  const int r0 = split * per, r1 = min(occ, r0 + per);
+  const int r0 = 0, r1 = occ;
   const int nchunks = r1 > r0 ? (r1 - r0 + kChunk - 1) / kChunk : 0;
   const size_t row_base = ((size_t)seq * Hkv + kvh) * c;
   volatile int* abort_flag = &sm.abort_flag;
@@ -450,36 +444,14 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kDecThreads, 2)
       s_res[g][D + 1] = lsum;
     }
   }
-  cluster.sync();
-  // ---- CTA 0 of the cluster combines the kSplit partial results through DSMEM
-  if (cluster.block_rank() == 0) {
-    for (int e = tid; e < G * D; e += blockDim.x) {
-      const int g = e / D, col = e % D;
-      float mm[kSplit], ll[kSplit], aa[kSplit];
-      float M = -INFINITY;
-#pragma unroll
-      for (int x = 0; x < kSplit; ++x) {
-        const float* rr = cluster.map_shared_rank(&s_res[0][0], x);
-        mm[x] = rr[g * (D + 2) + D];
-        ll[x] = rr[g * (D + 2) + D + 1];
-        aa[x] = rr[g * (D + 2) + col];
-        M = fmaxf(M, mm[x]);
-      }
-      const float Mu = (M == -INFINITY) ? 0.f : M;
-      float sum = 0.f, lsum = 0.f;
-#pragma unroll
-      for (int x = 0; x < kSplit; ++x) {
-        const float f = ex2(mm[x] - Mu);
-        sum += aa[x] * f;
-        lsum += ll[x] * f;
-      }
-      const int hq = kvh * G + g;
-      o[((size_t)seq * Hq + hq) * D + col] = __float2bfloat16(sum / lsum);
-      if (col == 0 && lse)
-        lse[(size_t)seq * Hq + hq] = (M + __log2f(lsum)) * 0.69314718055994531f;
-    }
+  __syncthreads();
+  for (int e = tid; e < G * D; e += blockDim.x) {
+    const int g = e / D, col = e % D;
+    const int hq = kvh * G + g;
+    o[((size_t)seq * Hq + hq) * D + col] = __float2bfloat16(s_res[g][col] / s_res[g][D + 1]);
+    if (col == 0 && lse)
+      lse[(size_t)seq * Hq + hq] = (s_res[g][D] + __log2f(s_res[g][D + 1])) * 0.69314718055994531f;
   }
-  cluster.sync();  // keep every CTA's shared memory alive until CTA 0 has read it
 }
 
 // ------------------------------------------------------------------ export order
@@ -532,7 +504,7 @@ static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void*
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  dim3 grid(kSplit, st.Hkv, st.S);
+  dim3 grid(st.Hkv, st.S);
   sepcache_decode_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(
       st.Hq, st.Hkv, st.a, st.s, st.w, reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
       reinterpret_cast<const __nv_bfloat16*>(st.v_slots), st.meta,

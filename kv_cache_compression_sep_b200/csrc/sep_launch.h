@@ -29,7 +29,7 @@ cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* 
 
 struct AttnMaps {
   CUtensorMap q, k, v, kc, vc;  // 4-D {d, H, L, B}, box {64, 1, 128, 1}, 128-byte swizzle
-  CUtensorMap o, dout;          // used by the backward kernels
+  CUtensorMap o, dout, dq, dk, dv;  // O store (forward); dO load, dQ/dK/dV stores (backward)
 };
 
 struct AttnShape {
@@ -46,8 +46,11 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
                             const int32_t* gather_end, const int8_t* tile_map, const void* o,
                             const float* lse, const void* dout, const void* q, const void* k,
                             const void* v, void* dq, void* dk, void* dv, void* kc, void* vc,
-                            float* delta, float* dka, float* dva, int stages,
+                            float* delta, float* dka, float* dva, void* sched, int stages,
                             cudaStream_t stream);
+
+// Bytes of the backward work-list region inside the workspace.
+size_t bwd_sched_bytes(int B, int L);
 
 cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream);
 cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new,

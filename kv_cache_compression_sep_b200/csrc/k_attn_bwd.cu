@@ -753,69 +753,100 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
+    // Order over the flattened pair stream: G(P, A), S(P+1, A), G(P, B), S(P+1, B), where S
+    // issues S^T/dP^T of a half and G its dV/dK products; half A's next softmax can then run
+    // while half B's is still working. At an item boundary with a single K/V buffer, both G
+    // of the last pair come first (the next item's K/V needs this item's epilogue).
     if (lane == 0) {
       constexpr uint32_t idS = make_idesc_bf16(128, 64, false, false);
       constexpr uint32_t idG = make_idesc_bf16(128, D, false, true);
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t sQa = smem_u32(sQ), sdOa = smem_u32(sdO);
       bool ok = true;
-      int P = 0;
-      for (int I = 0, x = blockIdx.x; ok && x < nitems; ++I, x += gridDim.x) {
-        const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
-        const int kb = I % KVB;
-        if (!mbar_wait(&bar->kv_full[kb], (I / KVB) & 1, p.err, abort_flag)) { ok = false; break; }
-        const uint32_t kA = sKa + kb * C::TILE, vA = sVa + kb * C::TILE;
-        for (int q = 0; q < it.npairs && ok; ++q, ++P) {
-          const int st = P % NST;
-          if (!mbar_wait(&bar->q_full[st], (P / NST) & 1, p.err, abort_flag)) { ok = false; break; }
-          const uint32_t qA = sQa + st * C::TILE, dA = sdOa + st * C::TILE;
-          // S^T and dP^T of both halves; a half's buffers hold the previous pair's P^T/dS^T
-          // until that pair's dV/dK products are done
-          for (int h = 0; h < 2; ++h) {
-            if (P > 0 && !mbar_wait(&bar->mm_done[h], (P - 1) & 1, p.err, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t cS = tmem + 128 * h, cP = cS + 64;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-              const uint32_t qoff = (kk >> 2) * kBoxBytes + h * 64 * 128 + (kk & 3) * 32;
-              mma_ss(cS, make_sdesc_sw128(kA + off, 16, 1024),
-                     make_sdesc_sw128(qA + qoff, 16, 1024), idS, kk > 0 ? 1u : 0u);
-              mma_ss(cP, make_sdesc_sw128(vA + off, 16, 1024),
-                     make_sdesc_sw128(dA + qoff, 16, 1024), idS, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&bar->s_full[h]);
-          }
-          if (!ok) break;
-          // the first dV/dK product of an item overwrites the accumulators: the previous
-          // item's epilogue must have read them
-          if (q == 0 && I > 0 && !mbar_wait(&bar->acc_free, (I - 1) & 1, p.err, abort_flag)) {
-            ok = false;
-            break;
-          }
-          for (int h = 0; h < 2; ++h) {
-            if (!mbar_wait(&bar->pds_ready[h], P & 1, p.err, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t cS = tmem + 128 * h, cP = cS + 64;
-#pragma unroll
-            for (int kk = 0; kk < 64 / 16; ++kk) {
-              const uint32_t roff = (h * 64 + kk * 16) * 128;
-              const uint32_t acc = (q > 0 || h > 0 || kk > 0) ? 1u : 0u;
-              mma_ts(tmem + C::COL_DV, cS + kk * 8, make_sdesc_sw128(dA + roff, kBoxBytes, 1024),
-                     idG, acc);
-              mma_ts(tmem + C::COL_DK, cP + kk * 8, make_sdesc_sw128(qA + roff, kBoxBytes, 1024),
-                     idG, acc);
-            }
-            tc_commit(&bar->mm_done[h]);
-          }
-          if (!ok) break;
-          tc_commit(&bar->q_empty[st]);
+      // cursor over (item, pair): the pair P's item index and local pair index
+      struct Cur {
+        int I, x, q, P;
+        DkvItem it;
+      };
+      auto first = [&]() {
+        Cur c;
+        c.I = 0; c.x = blockIdx.x; c.q = 0; c.P = 0;
+        if (c.x < nitems) c.it = dkv_item(p, aitems, witems, n_anchor, c.x, G);
+        return c;
+      };
+      auto next = [&](Cur c) {
+        ++c.P;
+        if (++c.q >= c.it.npairs) {
+          c.q = 0;
+          ++c.I;
+          c.x += gridDim.x;
+          if (c.x < nitems) c.it = dkv_item(p, aitems, witems, n_anchor, c.x, G);
         }
-        if (!ok) break;
-        tc_commit(&bar->acc_full);
+        return c;
+      };
+      auto issue_S = [&](const Cur& c, int h) -> bool {
+        const int kb = c.I % KVB, st = c.P % NST;
+        if (h == 0) {
+          if (c.q == 0 && !mbar_wait(&bar->kv_full[kb], (c.I / KVB) & 1, p.err, abort_flag)) return false;
+          if (!mbar_wait(&bar->q_full[st], (c.P / NST) & 1, p.err, abort_flag)) return false;
+        }
+        // the half's buffers hold the previous pair's P^T / dS^T until its products are done
+        if (c.P > 0 && !mbar_wait(&bar->mm_done[h], (c.P - 1) & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kA = sKa + kb * C::TILE, vA = sVa + kb * C::TILE;
+        const uint32_t qA = sQa + st * C::TILE, dA = sdOa + st * C::TILE;
+        const uint32_t cS = tmem + 128 * h, cP = cS + 64;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+          const uint32_t qoff = (kk >> 2) * kBoxBytes + h * 64 * 128 + (kk & 3) * 32;
+          mma_ss(cS, make_sdesc_sw128(kA + off, 16, 1024), make_sdesc_sw128(qA + qoff, 16, 1024),
+                 idS, kk > 0 ? 1u : 0u);
+          mma_ss(cP, make_sdesc_sw128(vA + off, 16, 1024), make_sdesc_sw128(dA + qoff, 16, 1024),
+                 idS, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar->s_full[h]);
+        return true;
+      };
+      auto issue_G = [&](const Cur& c, int h) -> bool {
+        const int st = c.P % NST;
+        // the first dV/dK product of an item overwrites the accumulators: the previous item's
+        // epilogue must have read them
+        if (h == 0 && c.q == 0 && c.I > 0 &&
+            !mbar_wait(&bar->acc_free, (c.I - 1) & 1, p.err, abort_flag))
+          return false;
+        if (!mbar_wait(&bar->pds_ready[h], c.P & 1, p.err, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qA = sQa + st * C::TILE, dA = sdOa + st * C::TILE;
+        const uint32_t cS = tmem + 128 * h, cP = cS + 64;
+#pragma unroll
+        for (int kk = 0; kk < 64 / 16; ++kk) {
+          const uint32_t roff = (h * 64 + kk * 16) * 128;
+          const uint32_t acc = (c.q > 0 || h > 0 || kk > 0) ? 1u : 0u;
+          mma_ts(tmem + C::COL_DV, cS + kk * 8, make_sdesc_sw128(dA + roff, kBoxBytes, 1024), idG,
+                 acc);
+          mma_ts(tmem + C::COL_DK, cP + kk * 8, make_sdesc_sw128(qA + roff, kBoxBytes, 1024), idG,
+                 acc);
+        }
+        tc_commit(&bar->mm_done[h]);
+        if (h == 1) {
+          tc_commit(&bar->q_empty[st]);
+          if (c.q == c.it.npairs - 1) tc_commit(&bar->acc_full);
+        }
+        return true;
+      };
+      Cur c = first();
+      if (c.x < nitems) ok = issue_S(c, 0) && issue_S(c, 1);
+      while (ok && c.x < nitems) {
+        const Cur n = next(c);
+        const bool more = n.x < nitems;
+        const bool boundary_wait = (KVB == 1) && (n.q == 0);  // next pair starts a new item
+        if (!issue_G(c, 0)) { ok = false; break; }
+        if (more && !boundary_wait && !issue_S(n, 0)) { ok = false; break; }
+        if (!issue_G(c, 1)) { ok = false; break; }
+        if (more && boundary_wait && !issue_S(n, 0)) { ok = false; break; }
+        if (more && !issue_S(n, 1)) { ok = false; break; }
+        c = n;
       }
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);

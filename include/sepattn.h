@@ -45,7 +45,8 @@ enum {
   SEP_ERR_MISALIGNED = 3,    /* a tensor base address not 16-byte aligned */
   SEP_ERR_CUDA = 4,          /* a CUDA runtime/driver call or a launch failed */
   SEP_ERR_TIMEOUT = 5,       /* device: a bounded pipeline wait ran out (reported sticky) */
-  SEP_ERR_WORKSPACE = 6      /* workspace pointer null or smaller than the size query says */
+  SEP_ERR_WORKSPACE = 6,     /* workspace pointer null or smaller than the size query says */
+  SEP_ERR_SCRATCH_LIMIT = 7  /* sep_attn_fwd_noalloc: problem larger than its fixed scratch */
 };
 
 /* Tile sizes the attention kernels use: query tiles of 128 rows, key tiles of 128 columns. */
@@ -219,6 +220,33 @@ int sep_last_device_error(void);
 
 /* Human-readable name of a status code. */
 const char* sep_status_string(int status);
+
+/*
+ * sep_attn_fwd_noalloc - sep_attn_fwd without a caller workspace and without any allocation.
+ *
+ * The SepLLM method has no counterpart to this call: it is an engineering variant of
+ * sep_attn_fwd (same arguments minus workspace, same kernels, same results). Some callers
+ * cannot hand over a workspace: a host whose device memory is all carved out in advance by a
+ * pool it owns (a serving engine that reserves HBM for its KV cache at start-up) has no spare
+ * buffer to give, and a latency-critical loop cannot call cudaMalloc / cudaFree, which may block
+ * on the driver or synchronise the whole device. This call uses instead a fixed array of
+ * SEP_NOALLOC_SCRATCH_BYTES that lives in the library's device image, and allocates nothing.
+ *
+ * Limit: the compacted anchor K and V need 2 * roundup256(B * L * Hkv * d * 2) bytes; a problem
+ * above SEP_NOALLOC_SCRATCH_BYTES returns SEP_ERR_SCRATCH_LIMIT before any device work.
+ * Setup: the first call on each device (with that device current) looks up the array's device
+ * address with cudaGetSymbolAddress, which loads the library's module on that device; make that
+ * first call before any stream capture. A failed lookup returns SEP_ERR_CUDA.
+ * Zeroing: none is needed; the compaction writes every row the attention kernel reads (the
+ * anchors, then zero rows up to the end of their last 128-row tile).
+ * Concurrency: every call on a device shares the one array. Calls that may overlap in time
+ * (different streams, or host threads, without ordering between them) race on it and give wrong
+ * results; calls in order on one stream are safe.
+ */
+#define SEP_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int sep_attn_fwd_noalloc(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v,
+                         int B, int L, int Hq, int Hkv, int d, float scale, int a, int n,
+                         const SepMask* mask, sep_bf16* o, float* lse, sep_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsepattn.so")
-SOURCES = ["k_mask.cu", "k_attn_fwd.cu", "k_attn_bwd.cu", "k_sepcache.cu", "api.cpp"]
+SOURCES = ["k_mask.cu", "k_attn_fwd.cu", "k_attn_bwd.cu", "k_sepcache.cu", "k_scratch.cu", "api.cpp"]
 HEADERS = ["sep_common.cuh", "sep_tiles.cuh", "sep_launch.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I" + os.path.join(ROOT, "include")]

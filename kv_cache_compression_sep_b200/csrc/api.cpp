@@ -288,6 +288,21 @@ int sep_last_device_error(void) {
   return (int)v;
 }
 
+int sep_attn_fwd_noalloc(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v, int B, int L,
+                         int Hq, int Hkv, int d, float scale, int a, int n, const SepMask* mask,
+                         sep_bf16* o, float* lse, sep_stream_t stream) {
+  // host checks first, so that an oversized problem is refused before any device work
+  int st = check_attn_args(q, k, v, B, L, Hq, Hkv, d, a, n, mask);
+  if (st != SEP_OK) return st;
+  if (!o || !lse) return SEP_ERR_INVALID_ARG;
+  if (fwd_ws(B, L, Hkv, d).total > (size_t)SEP_NOALLOC_SCRATCH_BYTES) return SEP_ERR_SCRATCH_LIMIT;
+  cudaError_t e = cudaSuccess;
+  void* scratch = sep::noalloc_fwd_scratch(&e);
+  if (!scratch) return SEP_ERR_CUDA;
+  return attn_fwd_impl(3, q, k, v, B, L, Hq, Hkv, d, scale, a, n, mask, o, lse, scratch,
+                       (size_t)SEP_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 const char* sep_status_string(int status) {
   switch (status) {
     case SEP_OK: return "ok";
@@ -297,6 +312,8 @@ const char* sep_status_string(int status) {
     case SEP_ERR_CUDA: return "CUDA error";
     case SEP_ERR_TIMEOUT: return "device pipeline wait timed out";
     case SEP_ERR_WORKSPACE: return "workspace missing or too small";
+    case SEP_ERR_SCRATCH_LIMIT:
+      return "problem needs more than the fixed scratch of sep_attn_fwd_noalloc";
     default: return "unknown status";
   }
 }

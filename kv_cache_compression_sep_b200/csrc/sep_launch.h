@@ -13,6 +13,8 @@ namespace sep {
 
 // Device address of the sticky error word on the current device (nullptr on failure).
 unsigned* device_error_word();
+// Fixed scratch of sep_attn_fwd_noalloc on the current device (first call per device: setup).
+void* noalloc_fwd_scratch(cudaError_t* err);
 
 cudaError_t launch_mask_build(const uint8_t* sep, int B, int L, int a, int n, int bm, int bn,
                               int32_t* anchor_idx, int32_t* anchor_cnt, uint32_t* anchor_bits,

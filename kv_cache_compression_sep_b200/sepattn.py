@@ -36,6 +36,7 @@ def _load():
         "sep_attn_fwd_workspace_size": (Z, [I, I, I, I]),
         "sep_attn_fwd": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
         "sep_attn_fwd_stage": (I, [I, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, Z, P]),
+        "sep_attn_fwd_noalloc": (I, [P, P, P, I, I, I, I, I, F, I, I, P, P, P, P]),
         "sep_attn_bwd_workspace_size": (Z, [I, I, I, I, I]),
         "sep_attn_bwd_stage": (I, [I, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, P, Z, P]),
         "sep_attn_bwd": (I, [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P, P, P, P, Z, P]),
@@ -174,6 +175,27 @@ def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspa
         _check(_lib.sep_attn_fwd(*args), "sep_attn_fwd")
     else:
         _check(_lib.sep_attn_fwd_stage(int(stage), *args), "sep_attn_fwd_stage")
+    return o, lse
+
+
+def sep_attn_fwd_noalloc(q, k, v, mask: SepMask, scale=None, out=None, lse=None):
+    """sep_attn_fwd through the library's fixed device scratch instead of a workspace.
+
+    The library allocates nothing for this call; the outputs are allocated here unless given.
+    Problems whose compacted anchors exceed SEP_NOALLOC_SCRATCH_BYTES raise SepError
+    (SEP_ERR_SCRATCH_LIMIT). Calls that may overlap in time share the scratch and race.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, torch.bfloat16, name)
+    B, L, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = d ** -0.5 if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device) if lse is None else lse
+    mc = mask._c()
+    _check(_lib.sep_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale),
+                                     mask.a, mask.n, ctypes.byref(mc), _ptr(o), _ptr(lse),
+                                     _stream()), "sep_attn_fwd_noalloc")
     return o, lse
 
 

@@ -31,51 +31,60 @@ namespace sep {
 
 constexpr int kBoxBytes = 128 * 64 * 2;
 
-// ------------------------------------------------------------------ prep kernels
-__global__ void __launch_bounds__(256) zero_anchor_partials_kernel(
-    const int32_t* __restrict__ anchor_cnt, int L, int rowvec, int rows_per_cta,
-    float4* __restrict__ dka, float4* __restrict__ dva) {
-  const int b = blockIdx.y;
-  const int cnt = anchor_cnt[b];
-  const int r0 = blockIdx.x * rows_per_cta;
-  if (r0 >= cnt) return;
-  const int rows = min(rows_per_cta, cnt - r0);
-  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int e = threadIdx.x; e < rows * rowvec; e += blockDim.x) {
-    const size_t dst = ((size_t)b * L + r0 + e / rowvec) * rowvec + e % rowvec;
-    dka[dst] = z;
-    dva[dst] = z;
-  }
-}
-
-// Delta[b][h][i] = sum_c dO[b,i,h,c] * O[b,i,h,c]; one thread per (b, i, h) row, 16-byte loads.
+// ------------------------------------------------------------------ prep kernel
+// One warp per position i of one sequence b (8 per CTA), all in one pass:
+//   Delta[b][h][i] = sum_c dO[b,i,h,c] * O[b,i,h,c] for every query head h (the O and dO rows of
+//   position i are Hq * d contiguous bf16: 16-byte chunks, D / 8 consecutive chunks per head,
+//   summed over the D / 8 lanes that hold them);
+//   row i of the compacted anchor K / V (i < roundup128(cnt));
+//   zero row i of the compact fp32 anchor partials (i < cnt, direct mode);
+//   and the two work-list counters (block 0).
 template <int D>
-__global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16* __restrict__ o,
-                                                    const __nv_bfloat16* __restrict__ dout,
-                                                    int B, int L, int Hq, float* __restrict__ delta) {
-  // consecutive threads take consecutive positions i of one (b, h): coalesced Delta stores
-  const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= (long long)B * L * Hq) return;
-  const int i = (int)(id % L);
-  const long long bh = id / L;
-  const int h = (int)(bh % Hq), b = (int)(bh / Hq);
-  const long long row = ((long long)b * L + i) * Hq + h;
-  const uint4* po = reinterpret_cast<const uint4*>(o + row * D);
-  const uint4* pd = reinterpret_cast<const uint4*>(dout + row * D);
-  float acc = 0.f;
+__global__ void __launch_bounds__(256) bwd_prep_kernel(
+    const uint4* __restrict__ o, const uint4* __restrict__ dout, const uint4* __restrict__ k,
+    const uint4* __restrict__ v, const int32_t* __restrict__ anchor_idx,
+    const int32_t* __restrict__ anchor_cnt, int L, int Hq, int Hkv, int zero_partials,
+    uint4* __restrict__ kc, uint4* __restrict__ vc, float4* __restrict__ dka,
+    float4* __restrict__ dva, float* __restrict__ delta, int32_t* __restrict__ counters) {
+  constexpr int CPH = D / 8;  // 16-byte chunks per head; divides 32
+  const int b = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (blockIdx.x == 0 && b == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
+  if (i >= L) return;
+  const size_t row = (size_t)b * L + i;
+  const int nch = Hq * CPH;
+  const uint4* po = o + row * nch;
+  const uint4* pd = dout + row * nch;
+  for (int c0 = 0; c0 < nch; c0 += 32) {
+    const int c = c0 + lane;
+    float acc = 0.f;
+    if (c < nch) {
+      const uint4 x = __ldg(po + c), y = __ldg(pd + c);
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-  for (int q = 0; q < D / 8; ++q) {
-    const uint4 x = __ldg(po + q), y = __ldg(pd + q);
-    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+      for (int z = 0; z < 4; ++z) {
+        const __nv_bfloat162 a2 = *reinterpret_cast<const __nv_bfloat162*>(&xs[z]);
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&ys[z]);
+        acc = fmaf(__low2float(a2), __low2float(b2), acc);
+        acc = fmaf(__high2float(a2), __high2float(b2), acc);
+      }
+    }
 #pragma unroll
-    for (int z = 0; z < 4; ++z) {
-      const __nv_bfloat162 a2 = *reinterpret_cast<const __nv_bfloat162*>(&xs[z]);
-      const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&ys[z]);
-      acc = fmaf(__low2float(a2), __low2float(b2), acc);
-      acc = fmaf(__high2float(a2), __high2float(b2), acc);
+    for (int off = CPH / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (c < nch && (lane % CPH) == 0) delta[((size_t)b * Hq + c / CPH) * L + i] = acc;
+  }
+  const int cnt = __ldg(anchor_cnt + b);
+  if (i < min(L, (cnt + 127) / 128 * 128))
+    compact_anchor_row(k, v, anchor_idx, cnt, L, b, i, Hkv * D / 8, kc, vc, lane);
+  if (zero_partials && i < cnt) {
+    const int pc = Hkv * D / 4;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = lane; c < pc; c += 32) {
+      dka[row * pc + c] = z;
+      dva[row * pc + c] = z;
     }
   }
-  delta[((size_t)b * Hq + h) * L + i] = acc;
 }
 
 // ------------------------------------------------------------------ shared parameter block
@@ -1066,25 +1075,21 @@ __global__ void __launch_bounds__(256) acc_to_bf16_kernel(const float4* __restri
 }
 
 // ------------------------------------------------------------------ anchor combine
-// dK/dV rows of the anchors: the fp32 sums of every part, rounded once to bf16.
+// dK/dV rows of the anchors: the fp32 sums of every part, rounded once to bf16. One warp per
+// compact anchor row (8 per CTA); q4 = float4 chunks per row.
 __global__ void __launch_bounds__(256) anchor_combine_kernel(
-    const int32_t* __restrict__ anchor_idx, const int32_t* __restrict__ anchor_cnt, int L,
-    int rowlen, int rows_per_cta, const float* __restrict__ dka, const float* __restrict__ dva,
-    __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
+    const int32_t* __restrict__ anchor_idx, const int32_t* __restrict__ anchor_cnt, int L, int q4,
+    const float4* __restrict__ dka, const float4* __restrict__ dva, uint2* __restrict__ dk,
+    uint2* __restrict__ dv) {
   const int b = blockIdx.y;
-  const int cnt = anchor_cnt[b];
-  const int r0 = blockIdx.x * rows_per_cta;
-  if (r0 >= cnt) return;
-  const int rows = min(rows_per_cta, cnt - r0);
-  const int q4 = rowlen / 4;
-  for (int e = threadIdx.x; e < rows * q4; e += blockDim.x) {
-    const int r = r0 + e / q4, z = e % q4;
-    const size_t src = ((size_t)b * L + r) * rowlen + z * 4;
-    const size_t dst = ((size_t)b * L + anchor_idx[(size_t)b * L + r]) * rowlen + z * 4;
-    const float4 x = *reinterpret_cast<const float4*>(dka + src);
-    const float4 y = *reinterpret_cast<const float4*>(dva + src);
-    *reinterpret_cast<uint2*>(dk + dst) = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
-    *reinterpret_cast<uint2*>(dv + dst) = make_uint2(pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= __ldg(anchor_cnt + b)) return;
+  const size_t src = ((size_t)b * L + r) * q4;
+  const size_t dst = ((size_t)b * L + __ldg(anchor_idx + (size_t)b * L + r)) * q4;
+  for (int c = threadIdx.x & 31; c < q4; c += 32) {
+    const float4 x = dka[src + c], y = dva[src + c];
+    dk[dst + c] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+    dv[dst + c] = make_uint2(pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
   }
 }
 
@@ -1152,32 +1157,18 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   const size_t acc_bytes = (size_t)s.B * s.L * s.Hkv * s.d * sizeof(float);
 
   if (stages & kBwdPrep) {
-    if ((e = launch_compact_anchors(k, v, anchor_idx, anchor_cnt, s.B, s.L, s.Hkv, s.d, kc, vc,
-                                    stream)) != cudaSuccess)
-      return e;
-    if (direct) {
-      const int rowvec = s.Hkv * s.d / 4;
-      dim3 grid((s.L + 31) / 32, s.B);
-      zero_anchor_partials_kernel<<<grid, 256, 0, stream>>>(anchor_cnt, s.L, rowvec, 32,
-                                                            reinterpret_cast<float4*>(dka),
-                                                            reinterpret_cast<float4*>(dva));
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    } else {
+    if (!direct) {
       if ((e = cudaMemsetAsync(dka, 0, acc_bytes, stream)) != cudaSuccess) return e;
       if ((e = cudaMemsetAsync(dva, 0, acc_bytes, stream)) != cudaSuccess) return e;
     }
-    const long long rows = (long long)s.B * s.L * s.Hq;
-    const unsigned blocks = (unsigned)((rows + 255) / 256);
-    if (s.d == 128)
-      delta_kernel<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                    static_cast<const __nv_bfloat16*>(dout), s.B,
-                                                    s.L, s.Hq, delta);
-    else
-      delta_kernel<64><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                   static_cast<const __nv_bfloat16*>(dout), s.B,
-                                                   s.L, s.Hq, delta);
+    const dim3 pgrid((s.L + 7) / 8, s.B);
+    auto prep = (s.d == 128) ? bwd_prep_kernel<128> : bwd_prep_kernel<64>;
+    prep<<<pgrid, 256, 0, stream>>>(
+        static_cast<const uint4*>(o), static_cast<const uint4*>(dout), static_cast<const uint4*>(k),
+        static_cast<const uint4*>(v), anchor_idx, anchor_cnt, s.L, s.Hq, s.Hkv, direct,
+        static_cast<uint4*>(kc), static_cast<uint4*>(vc), reinterpret_cast<float4*>(dka),
+        reinterpret_cast<float4*>(dva), delta, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(counters, 0, 2 * sizeof(int32_t), stream)) != cudaSuccess) return e;
     bwd_schedule_kernel<<<s.B, 1024, 0, stream>>>(anchor_cnt, gather_end, anchor_bits, s.L, s.n,
                                                   T, W, tile_prefix, aitems, witems, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1239,10 +1230,10 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (stages & kBwdDkv) {
     if (direct) {
-      dim3 grid((s.L + 31) / 32, s.B);
-      anchor_combine_kernel<<<grid, 256, 0, stream>>>(anchor_idx, anchor_cnt, s.L, s.Hkv * s.d, 32,
-                                                      dka, dva, static_cast<__nv_bfloat16*>(dk),
-                                                      static_cast<__nv_bfloat16*>(dv));
+      dim3 grid((s.L + 7) / 8, s.B);
+      anchor_combine_kernel<<<grid, 256, 0, stream>>>(
+          anchor_idx, anchor_cnt, s.L, s.Hkv * s.d / 4, reinterpret_cast<const float4*>(dka),
+          reinterpret_cast<const float4*>(dva), static_cast<uint2*>(dk), static_cast<uint2*>(dv));
     } else {
       const long long n4 = (long long)s.B * s.L * s.Hkv * s.d / 4;
       acc_to_bf16_kernel<<<nsm * 8, 256, 0, stream>>>(

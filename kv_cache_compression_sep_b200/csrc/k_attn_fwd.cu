@@ -507,40 +507,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 // Row r < anchor_cnt[b] of kc/vc receives the K/V row of anchor r; rows from anchor_cnt[b] up to
 // the next multiple of 128 are zeroed so that the last (partly valid) anchor chunk holds finite
 // values (masked scores still multiply V in the P*V product).
+// One warp per compacted row (8 rows per CTA); CTAs past the last anchor tile exit at once.
 __global__ void __launch_bounds__(256) compact_anchors_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, const int32_t* __restrict__ anchor_idx,
-    const int32_t* __restrict__ anchor_cnt, int L, int rowvec, int rows_per_cta,
-    uint4* __restrict__ kc, uint4* __restrict__ vc) {
+    const int32_t* __restrict__ anchor_cnt, int L, int kv_ch, uint4* __restrict__ kc,
+    uint4* __restrict__ vc) {
   const int b = blockIdx.y;
-  const int cnt = anchor_cnt[b];
+  const int cnt = __ldg(anchor_cnt + b);
   const int pad_end = min(L, (cnt + 127) / 128 * 128);
-  const int r0 = blockIdx.x * rows_per_cta;
-  if (r0 >= pad_end) return;
-  const int rows = min(rows_per_cta, pad_end - r0);
-  const int32_t* idx = anchor_idx + (size_t)b * L;
-  for (int e = threadIdx.x; e < rows * rowvec; e += blockDim.x) {
-    const int r = r0 + e / rowvec, c = e % rowvec;
-    const size_t dst = ((size_t)b * L + r) * rowvec + c;
-    if (r < cnt) {
-      const size_t src = ((size_t)b * L + idx[r]) * rowvec + c;
-      kc[dst] = __ldg(k + src);
-      vc[dst] = __ldg(v + src);
-    } else {
-      kc[dst] = make_uint4(0, 0, 0, 0);
-      vc[dst] = make_uint4(0, 0, 0, 0);
-    }
-  }
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (i >= pad_end) return;
+  compact_anchor_row(k, v, anchor_idx, cnt, L, b, i, kv_ch, kc, vc, threadIdx.x & 31);
 }
 
 cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* anchor_idx,
                                    const int32_t* anchor_cnt, int B, int L, int Hkv, int d,
                                    void* kc, void* vc, cudaStream_t stream) {
-  const int rowvec = Hkv * d * 2 / 16;
-  const int rows_per_cta = 32;
-  dim3 grid((L + rows_per_cta - 1) / rows_per_cta, B);
+  const int kv_ch = Hkv * d * 2 / 16;
+  dim3 grid((L + 7) / 8, B);
   compact_anchors_kernel<<<grid, 256, 0, stream>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), anchor_idx, anchor_cnt, L,
-      rowvec, rows_per_cta, static_cast<uint4*>(kc), static_cast<uint4*>(vc));
+      kv_ch, static_cast<uint4*>(kc), static_cast<uint4*>(vc));
   return cudaGetLastError();
 }
 

@@ -10,6 +10,34 @@
 
 namespace sep {
 
+// Row i of batch b of the compacted anchor K / V (one warp; kv_ch = 16-byte chunks per row):
+// the K / V row of the i-th anchor when i < cnt, zeros up to the end of the anchors' last
+// 128-row tile. The caller takes rows i < min(L, roundup128(cnt)).
+__device__ __forceinline__ void compact_anchor_row(const uint4* __restrict__ k,
+                                                   const uint4* __restrict__ v,
+                                                   const int32_t* __restrict__ anchor_idx,
+                                                   int cnt, int L, int b, int i, int kv_ch,
+                                                   uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                                   int lane) {
+  const size_t row = (size_t)b * L + i;
+  uint4* dk = kc + row * kv_ch;
+  uint4* dv = vc + row * kv_ch;
+  if (i < cnt) {
+    const size_t src = ((size_t)b * L + __ldg(anchor_idx + row)) * kv_ch;
+    for (int c = lane; c < kv_ch; c += 32) {
+      const uint4 x = __ldg(k + src + c), y = __ldg(v + src + c);
+      dk[c] = x;
+      dv[c] = y;
+    }
+  } else {
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int c = lane; c < kv_ch; c += 32) {
+      dk[c] = z;
+      dv[c] = z;
+    }
+  }
+}
+
 __host__ __device__ __forceinline__ int window_lo_tile(int t, int n) {
   const long long k = (long long)t * 128 - n + 1;
   return k > 0 ? (int)(k / 128) : 0;

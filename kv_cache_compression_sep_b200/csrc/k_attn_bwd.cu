@@ -38,7 +38,7 @@ constexpr int kBoxBytes = 128 * 64 * 2;
 //   summed over the D / 8 lanes that hold them);
 //   row i of the compacted anchor K / V (i < roundup128(cnt));
 //   zero row i of the compact fp32 anchor partials (i < cnt, direct mode);
-//   and the two work-list counters (block 0).
+//   and the four work-list counters (block 0).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const uint4* __restrict__ o, const uint4* __restrict__ dout, const uint4* __restrict__ k,
@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
   const int b = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (blockIdx.x == 0 && b == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0;
+  if (blockIdx.x == 0 && b == 0 && threadIdx.x < 4) counters[threadIdx.x] = 0;
   if (i >= L) return;
   const size_t row = (size_t)b * L + i;
   const int nch = Hq * CPH;
@@ -518,7 +518,7 @@ __global__ void __launch_bounds__(1024) bwd_schedule_kernel(
     const int32_t* __restrict__ anchor_cnt, const int32_t* __restrict__ gather_end,
     const uint32_t* __restrict__ anchor_bits, int L, int n, int T, int W, int32_t* __restrict__ tile_prefix,
     WorkItem* __restrict__ anchor_items, WorkItem* __restrict__ window_items,
-    int32_t* __restrict__ counters /* [0] anchor items, [1] window items */) {
+    int32_t* __restrict__ counters /* [0] anchor items, [1] window items; [2], [3] dK/dV pass */) {
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   __shared__ int s_warp[32];
@@ -624,6 +624,8 @@ struct DkvBar {
   uint64_t s_full[2], pds_ready[2], mm_done[2];
   uint64_t acc_full, acc_free;
   uint64_t drain;
+  uint64_t item_full[4];  // ring of fetched work-item indices (producer -> MMA, softmax)
+  int item_x[4];
   float lse2[NST][128];
   float delta[NST][128];
   uint32_t tmem_base;
@@ -659,8 +661,7 @@ __device__ __forceinline__ DkvItem dkv_item(const BwdParams& p, const WorkItem* 
 template <int D>
 __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     sep_attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p, const WorkItem* __restrict__ aitems,
-                            const WorkItem* __restrict__ witems,
-                            const int32_t* __restrict__ counters,
+                            const WorkItem* __restrict__ witems, int32_t* __restrict__ counters,
                             const int32_t* __restrict__ tile_prefix, int direct) {
   using C = DkvCfg<D>;
   constexpr int NST = C::NST, KVB = C::KVB;
@@ -696,6 +697,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     mbar_init(&bar->acc_full, 1);
     mbar_init(&bar->acc_free, 256);
     mbar_init(&bar->drain, 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&bar->item_full[s], 1);
     bar->abort_flag = 0;
     fence_barrier_init();
   }
@@ -712,12 +714,23 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     // ---------------------------------------------------------------- producer (whole warp)
     int P = 0;
     bool ok = true;
-    for (int I = 0, x = blockIdx.x; ok && x < nitems; ++I, x += gridDim.x) {
-      const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+    // Items are taken one at a time from the global counter (counters[2]) once the K/V buffer
+    // they will use is free, and published to the other roles through the item ring; the
+    // first index >= nitems ends every role.
+    for (int I = 0; ok; ++I) {
       const int kb = I % KVB;
       bool okw = true;
       if (I >= KVB) okw = mbar_wait(&bar->kv_empty[kb], ((I - KVB) / KVB) & 1, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+      int x = 0;
+      if (lane == 0) {
+        x = min(atomicAdd(&counters[2], 1), nitems);
+        bar->item_x[I & 3] = x;
+        mbar_arrive(&bar->item_full[I & 3]);
+      }
+      x = __shfl_sync(0xffffffffu, x, 0);
+      if (x >= nitems) break;
+      const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar->kv_full[kb], 2 * C::TILE);
         const int krow = it.unit * 128;
@@ -772,26 +785,18 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t sQa = smem_u32(sQ), sdOa = smem_u32(sdO);
       bool ok = true;
-      // cursor over (item, pair): the pair P's item index and local pair index
+      // cursor over (item, pair): local item count I, its index x, pair q within it, and the
+      // CTA-wide pair count P
       struct Cur {
         int I, x, q, P;
         DkvItem it;
       };
-      auto first = [&]() {
-        Cur c;
-        c.I = 0; c.x = blockIdx.x; c.q = 0; c.P = 0;
+      auto load_item = [&](Cur& c) -> bool {  // c.I set: wait for the producer to publish it
+        if (!mbar_wait(&bar->item_full[c.I & 3], (c.I >> 2) & 1, p.err, abort_flag)) return false;
+        c.x = bar->item_x[c.I & 3];
+        c.q = 0;
         if (c.x < nitems) c.it = dkv_item(p, aitems, witems, n_anchor, c.x, G);
-        return c;
-      };
-      auto next = [&](Cur c) {
-        ++c.P;
-        if (++c.q >= c.it.npairs) {
-          c.q = 0;
-          ++c.I;
-          c.x += gridDim.x;
-          if (c.x < nitems) c.it = dkv_item(p, aitems, witems, n_anchor, c.x, G);
-        }
-        return c;
+        return true;
       };
       auto issue_S = [&](const Cur& c, int h) -> bool {
         const int kb = c.I % KVB, st = c.P % NST;
@@ -844,17 +849,29 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         }
         return true;
       };
-      Cur c = first();
-      if (c.x < nitems) ok = issue_S(c, 0) && issue_S(c, 1);
+      Cur c;
+      c.I = 0;
+      c.P = 0;
+      ok = load_item(c);
+      if (ok && c.x < nitems) ok = issue_S(c, 0) && issue_S(c, 1);
       while (ok && c.x < nitems) {
-        const Cur n = next(c);
-        const bool more = n.x < nitems;
-        const bool boundary_wait = (KVB == 1) && (n.q == 0);  // next pair starts a new item
-        if (!issue_G(c, 0)) { ok = false; break; }
-        if (more && !boundary_wait && !issue_S(n, 0)) { ok = false; break; }
-        if (!issue_G(c, 1)) { ok = false; break; }
-        if (more && boundary_wait && !issue_S(n, 0)) { ok = false; break; }
-        if (more && !issue_S(n, 1)) { ok = false; break; }
+        Cur n = c;
+        ++n.P;
+        if (c.q + 1 < c.it.npairs) {
+          ++n.q;
+          ok = issue_G(c, 0) && issue_S(n, 0) && issue_G(c, 1) && issue_S(n, 1);
+        } else if (KVB == 1) {
+          // the next item is published only after this item's epilogue (one K/V buffer)
+          ++n.I;
+          ok = issue_G(c, 0) && issue_G(c, 1) && load_item(n);
+          if (ok && n.x < nitems) ok = issue_S(n, 0) && issue_S(n, 1);
+        } else {
+          ++n.I;
+          ok = load_item(n);
+          const bool more = ok && n.x < nitems;
+          ok = ok && issue_G(c, 0) && (!more || issue_S(n, 0)) && issue_G(c, 1) &&
+               (!more || issue_S(n, 1));
+        }
         c = n;
       }
       tc_commit(&bar->drain);
@@ -868,7 +885,13 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     int P = 0;
-    for (int I = 0, x = blockIdx.x; ok && x < nitems; ++I, x += gridDim.x) {
+    for (int I = 0; ok; ++I) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar->item_full[I & 3], (I >> 2) & 1, p.err, abort_flag))) {
+        ok = false;
+        break;
+      }
+      const int x = bar->item_x[I & 3];
+      if (x >= nitems) break;
       const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
       const int kb = I % KVB;
       long long j = -1;  // key position (window items)
@@ -1059,6 +1082,15 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // the last CTA out rewinds the item counter, so that a later launch over the same work list
+  // (the staged form run again) starts from item 0
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&counters[3], 1) == (int)gridDim.x - 1) {
+      atomicExch(&counters[2], 0);
+      atomicExch(&counters[3], 0);
+    }
+  }
 }
 
 // Position-indexed fp32 accumulators to bf16 dK / dV (used when window items are segmented).
@@ -1097,7 +1129,7 @@ size_t bwd_sched_bytes(int B, int L) {
   const size_t T = (L + 127) / 128;
   const size_t cap = (size_t)B * T * ((T + kSegT - 1) / kSegT);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  return up(2 * sizeof(int32_t)) + up((size_t)B * T * sizeof(int32_t)) + 2 * up(cap * sizeof(WorkItem));
+  return up(4 * sizeof(int32_t)) + up((size_t)B * T * sizeof(int32_t)) + 2 * up(cap * sizeof(WorkItem));
 }
 
 static int sm_count_dev() {
@@ -1151,8 +1183,8 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   const size_t cap = (size_t)s.B * T * ((T + kSegT - 1) / kSegT);
   uint8_t* sw = static_cast<uint8_t*>(sched);
   int32_t* counters = reinterpret_cast<int32_t*>(sw);
-  int32_t* tile_prefix = reinterpret_cast<int32_t*>(sw + up(2 * sizeof(int32_t)));
-  WorkItem* aitems = reinterpret_cast<WorkItem*>(sw + up(2 * sizeof(int32_t)) + up((size_t)s.B * T * sizeof(int32_t)));
+  int32_t* tile_prefix = reinterpret_cast<int32_t*>(sw + up(4 * sizeof(int32_t)));
+  WorkItem* aitems = reinterpret_cast<WorkItem*>(sw + up(4 * sizeof(int32_t)) + up((size_t)s.B * T * sizeof(int32_t)));
   WorkItem* witems = aitems + up(cap * sizeof(WorkItem)) / sizeof(WorkItem);
   const size_t acc_bytes = (size_t)s.B * s.L * s.Hkv * s.d * sizeof(float);
 

@@ -142,7 +142,7 @@ class TrainDecodeStep:
         # decode bytes: retained K and V rows, the query and output, the new slot written
         self.bytes_dec = (occ * dc.Hkv * dc.d * 2 * 2 + 2 * dc.Hq * dc.d * 2 + dc.Hkv * dc.d * 2 * 2) * dc.S
         self.flops = self.flops_fwd + self.flops_bwd + self.flops_dec
-        self.launches = 12  # mask 2, fwd 2, bwd 6, update 1, decode 1
+        self.launches = 11  # mask 2, fwd 2, bwd 5 (prep, schedule, dQ, dK/dV, combine), update 1, decode 1
 
     def run(self):
         S, d, cfg = self.S, self.dev, self.cfg
@@ -340,11 +340,15 @@ def roofline_for(name, comps, step, peaks, peak_src):
 
 
 def load_traffic(name):
-    """DRAM bytes per launch from the committed ncu summary, if one covers this kernel."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(p):
-        with open(p) as fh:
-            return json.load(fh).get(name)
+    """DRAM bytes per launch from the committed ncu summary table, if a row covers this pass."""
+    p = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        for ln in fh:
+            cells = [c.strip() for c in ln.strip().strip("|").split("|")]
+            if len(cells) >= 3 and cells[0] == name and cells[2].isdigit():
+                return int(cells[2])
     return None
 
 

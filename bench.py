@@ -101,6 +101,28 @@ class ClockSampler:
                 "samples": len(self.rows)}
 
 
+# ---------------------------------------------------------------------------- ranks
+# Weak scaling: every rank runs the whole step on its own inputs (no data-path collective);
+# only the timing is combined, as the max over ranks.
+def rank_seed(seed, rank):
+    """Seed of a rank's synthetic inputs: the workload's seed for rank 0, distinct per rank."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x, device, world):
+    """Max of a per-rank float over all ranks (the step time the whole job waits for)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step_per_rank, world, steps, max_ms):
+    """Whole-job rate: the units all ranks processed divided by the slowest rank's time."""
+    return units_per_step_per_rank * world * steps / (max_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- native arm
 class TrainDecodeStep:
     """Buffers and one CUDA graph for the default step (training attention + decode)."""
@@ -109,7 +131,7 @@ class TrainDecodeStep:
         self.S = S
         cfg = workloads.PYTHIA160M
         self.cfg = cfg
-        inp = workloads.attn_inputs(dataclasses.replace(cfg, seed=cfg.seed + 1000 * rank))
+        inp = workloads.attn_inputs(dataclasses.replace(cfg, seed=rank_seed(cfg.seed, rank)))
         self.host = {k: inp[k].pin_memory() for k in ("sep", "q", "k", "v", "do")}
         self.dev = {k: v.to(dev) for k, v in inp.items() if v is not None}
         d = self.dev
@@ -125,10 +147,11 @@ class TrainDecodeStep:
         self.dc = dc
         self.cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, dc.s, dc.w, dc.theta, device=dev)
         fill = dc.c + 100
-        ch = workloads.decode_chunk(dc, 0, fill, device=dev)
+        dc_r = dataclasses.replace(dc, seed=rank_seed(dc.seed, rank))
+        ch = workloads.decode_chunk(dc_r, 0, fill, device=dev)
         for t in range(fill):
             self.cache.sepcache_update(ch["k"][t], ch["v"][t], ch["sep"][t])
-        self.pool = workloads.decode_chunk(dc, fill, 64, device=dev)
+        self.pool = workloads.decode_chunk(dc_r, fill, 64, device=dev)
         self.host_dec = {k: v[0].cpu().pin_memory() for k, v in self.pool.items()}
         self.step_in = {k: v[0].clone() for k, v in self.pool.items()}
         self.o_dec = torch.empty_like(self.step_in["q"])
@@ -248,12 +271,8 @@ def native(args, rank, world, dev):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = step.flops * world * args.steps / (max_ms * 1e-3) / 1e12
+    max_ms = max_over_ranks(sum(step_ms), dev, world)
+    value = job_throughput(step.flops, world, args.steps, max_ms) / 1e12
     assert S.sep_last_device_error() == 0
 
     if args.quick:  # timed step only (used under ncu)
@@ -353,47 +372,81 @@ def load_traffic(name):
 
 
 def e2e_run(step, args, dev, world):
-    """Same step through the public API with host buffers: H2D of the step's inputs, D2H of
-    its results (dQ, dK, dV and the decode output), all inside the timed region."""
-    S = step.S
-    h, d = step.host, step.dev
-    hd = step.host_dec
-    outs = {"dq": torch.empty_like(step.grads[0], device="cpu").pin_memory(),
-            "dk": torch.empty_like(step.grads[1], device="cpu").pin_memory(),
-            "dv": torch.empty_like(step.grads[2], device="cpu").pin_memory(),
-            "o_dec": torch.empty_like(step.o_dec, device="cpu").pin_memory()}
+    """Same step through the public API with host buffers: every step copies its inputs in from
+    pinned host memory and its results (dQ, dK, dV and the decode output) back out, all inside
+    the timed region. The copies of neighbouring steps overlap the compute: step k+1's inputs
+    go in on one stream and step k-1's results come out on another while step k computes on a
+    third (device inputs and outputs double-buffered)."""
+    S, cfg = step.S, step.cfg
+    h, hd = step.host, step.host_dec
+    x_in = [({k: torch.empty_like(step.dev[k]) for k in h},
+             {k: torch.empty_like(step.step_in[k]) for k in hd}) for _ in range(2)]
+    y_dev = [tuple(torch.empty_like(g) for g in step.grads) + (torch.empty_like(step.o_dec),)
+             for _ in range(2)]
+    y_host = [tuple(torch.empty_like(t, device="cpu").pin_memory() for t in y) for y in y_dev]
     h2d = sum(t.numel() * t.element_size() for t in list(h.values()) + list(hd.values()))
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    d2h = sum(t.numel() * t.element_size() for t in y_host[0])
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def compute(b):
+        xa, xd = x_in[b]
+        dq, dk, dv, od = y_dev[b]
+        S.sep_mask_build(xa["sep"], cfg.a, cfg.n, out=step.mask)
+        S.sep_attn_fwd(xa["q"], xa["k"], xa["v"], step.mask, out=step.o, lse=step.lse,
+                       workspace=step.ws_f)
+        S.sep_attn_bwd(xa["q"], xa["k"], xa["v"], step.o, step.lse, xa["do"], step.mask,
+                       workspace=step.ws_b, grads=(dq, dk, dv))
+        step.cache.sepcache_update(xd["k"], xd["v"], xd["sep"])
+        step.cache.sepcache_decode(xd["q"], out=od)
+
+    def pipeline(n, e_start=None, e_end=None):
+        started = [False, False]
+        for i in range(n + 2):
+            if i < n:  # inputs of step i into buffer i % 2, once step i-2 has finished with it
+                b = i % 2
+                with torch.cuda.stream(s_in):
+                    if started[b]:
+                        s_in.wait_event(comp_done[b])
+                    if i == 0 and e_start is not None:
+                        e_start.record(s_in)
+                    for k in h:
+                        x_in[b][0][k].copy_(h[k], non_blocking=True)
+                    for k in hd:
+                        x_in[b][1][k].copy_(hd[k], non_blocking=True)
+                    in_done[b].record(s_in)
+            if 1 <= i <= n:  # compute step i-1, once its inputs are in and buffer's results out
+                b = (i - 1) % 2
+                with torch.cuda.stream(s_comp):
+                    s_comp.wait_event(in_done[b])
+                    if started[b]:
+                        s_comp.wait_event(out_done[b])
+                    compute(b)
+                    comp_done[b].record(s_comp)
+                started[b] = True
+            if i >= 2:  # results of step i-2 out
+                b = (i - 2) % 2
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(comp_done[b])
+                    for src, dst in zip(y_dev[b], y_host[b]):
+                        dst.copy_(src, non_blocking=True)
+                    out_done[b].record(s_out)
+        if e_end is not None:
+            e_end.record(s_out)
+
     n = max(3, min(args.steps, 20))
-
-    def one():
-        for k in h:
-            d[k].copy_(h[k], non_blocking=True)
-        for k in hd:
-            step.step_in[k].copy_(hd[k], non_blocking=True)
-        step.run()
-        outs["dq"].copy_(step.grads[0], non_blocking=True)
-        outs["dk"].copy_(step.grads[1], non_blocking=True)
-        outs["dv"].copy_(step.grads[2], non_blocking=True)
-        outs["o_dec"].copy_(step.o_dec, non_blocking=True)
-
-    one()
+    pipeline(2)
     torch.cuda.synchronize()
-    st = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(n):
-        one()
-    e1.record(st)
+    pipeline(n, e0, e1)
     e1.synchronize()
     ms = e0.elapsed_time(e1) / n
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms = float(t.item())
-    return {"value": step.flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ms, dev, world)
+    return {"value": job_throughput(step.flops, world, 1, ms) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": n}
+            "steps": n, "overlap": "H2D of step k+1 and D2H of step k-1 overlap step k"}
 
 
 # ---------------------------------------------------------------------------- oracle arm

@@ -252,6 +252,23 @@ class SepCache:
                                   self.meta.data_ptr(), self.rope_cs.data_ptr())
         _check(_lib.sepcache_state_init(ctypes.byref(self._st), _stream()), "sepcache_state_init")
 
+    # checkpoint / resume: the whole state lives in these tensors (the cos/sin table is a pure
+    # function of c, d and theta and is rebuilt by the constructor)
+    _STATE = ("k_slots", "v_slots", "slot_pos", "slot_sep", "meta")
+
+    def state_dict(self):
+        """Host copies of every state tensor (stream-ordered after earlier calls)."""
+        return {k: getattr(self, k).to("cpu", copy=True) for k in self._STATE}
+
+    def load_state_dict(self, sd):
+        """Restores a state_dict() taken from a cache of the same shape."""
+        for k in self._STATE:
+            dst = getattr(self, k)
+            if tuple(sd[k].shape) != tuple(dst.shape) or sd[k].dtype != dst.dtype:
+                raise SepError(f"load_state_dict: {k} has shape {tuple(sd[k].shape)}, "
+                               f"expected {tuple(dst.shape)}")
+            dst.copy_(sd[k])
+
     def sepcache_update(self, k_new, v_new, sep_new):
         _cuda(k_new, torch.bfloat16, "k_new")
         _cuda(v_new, torch.bfloat16, "v_new")

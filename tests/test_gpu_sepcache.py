@@ -130,3 +130,39 @@ def test_sepcache_decode_config_full(S):
             check(t, o, f64(qn), seqs, kv)
     torch.cuda.synchronize()
     assert S.sep_last_device_error() == 0
+
+
+def test_checkpoint_resume_bit_identical(S):
+    """state_dict() after 300 steps, restored into a fresh cache, replays the next 100 steps
+    with bit-identical decode outputs and trajectory."""
+    import torch
+    Sq, Hq, Hkv, d, a, s, w = 3, 8, 2, 128, 4, 16, 40
+    g = torch.Generator().manual_seed(77)
+    steps = [(torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16),
+              torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16),
+              torch.randn(Sq, Hq, d, generator=g).to(torch.bfloat16),
+              (torch.rand(Sq, generator=g) < 0.2).to(torch.uint8)) for _ in range(400)]
+    a_cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, 500000.0)
+    for kn, vn, qn, sn in steps[:300]:
+        a_cache.sepcache_update(kn.cuda(), vn.cuda(), sn.cuda())
+    ckpt = a_cache.state_dict()
+
+    def run(cache):
+        outs = []
+        for kn, vn, qn, sn in steps[300:]:
+            cache.sepcache_update(kn.cuda(), vn.cuda(), sn.cuda())
+            lse = torch.empty(Sq, Hq, dtype=torch.float32, device="cuda")
+            o = cache.sepcache_decode(qn.cuda(), lse=lse)
+            outs.append((o.cpu(), lse.cpu()))
+        return outs, cache.sepcache_export_order()
+
+    ref_outs, ref_order = run(a_cache)
+    b_cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, 500000.0)
+    b_cache.load_state_dict(ckpt)
+    got_outs, got_order = run(b_cache)
+    torch.cuda.synchronize()
+    assert S.sep_last_device_error() == 0
+    for (o1, l1), (o2, l2) in zip(ref_outs, got_outs):
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    for x, y in zip(ref_order, got_order):
+        assert torch.equal(x.cpu(), y.cpu())

@@ -557,6 +557,22 @@ def single_row(args, dev):
                     "gbs_update_plus_decode": byts / (ms * 1e-3) / 1e9})
         del step
         return out
+    if args.workload == "cache-prefill":
+        # seed 64 caches (the decode configuration's capacities) from 8192-token prompts
+        dc, Lp = workloads.SEPCACHE_DECODE, 8192
+        cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, dc.s, dc.w, dc.theta, device=dev)
+        g0 = torch.Generator(device=dev).manual_seed(dc.seed)
+        k = torch.randn(dc.S, Lp, dc.Hkv, dc.d, generator=g0, device=dev).to(torch.bfloat16)
+        v = torch.randn(dc.S, Lp, dc.Hkv, dc.d, generator=g0, device=dev).to(torch.bfloat16)
+        sep = (torch.rand(dc.S, Lp, generator=g0, device=dev) < dc.p).to(torch.uint8)
+        g = capture(lambda: cache.sepcache_prefill(k, v, sep), reps=20)
+        ms = time_graph(g, args.steps, flush) / 20
+        occ = int(cache.state_dict()["meta"][:, 1:6:2].sum())  # initial + separators + window
+        byts = occ * dc.Hkv * dc.d * 2 * 2 * 2 + dc.S * Lp  # K/V rows read and written, flags
+        out.update({"prompt_len": Lp, "us": ms * 1e3, "occupied_slots": occ,
+                    "gbs": byts / (ms * 1e-3) / 1e9,
+                    "frac_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
+        return out
     cfg = {"llama-prefill": workloads.LLAMA3_8B_PREFILL, "long-context": workloads.LONG_CONTEXT,
            "long-context-dense": workloads.LONG_CONTEXT,
            "pythia-train": workloads.PYTHIA160M}[args.workload]
@@ -594,7 +610,7 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="train-decode",
                     choices=["train-decode", "pythia-train", "llama-prefill", "long-context",
-                             "long-context-dense", "decode"])
+                             "long-context-dense", "decode", "cache-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",

@@ -200,6 +200,19 @@ int sepcache_update(const SepCacheState* st, const sep_bf16* k_new, const sep_bf
                     const uint8_t* sep_new, sep_stream_t stream);
 
 /*
+ * sepcache_prefill - seed every sequence's cache with an L-token prompt in one call.
+ * Sets the state to the one L sepcache_update calls (tokens 0..L-1 in order) would leave on an
+ * empty cache, whatever the state was before; K/V rows of slots left unused are not touched.
+ * This is how a prompt processed by sep_attn_fwd (the prefill pass) hands its keys and values
+ * to streaming decode ("How SepLLM reorchestrates the language model...", "SepLLM's
+ * Architecture: Composing Efficiency": initial, separator and local-window blocks).
+ * k, v [S, L, Hkv, d] un-rotated (the layout sep_attn_fwd reads); sep [S, L] uint8. L >= 1;
+ * s <= 16384 (SEP_ERR_UNSUPPORTED otherwise).
+ */
+int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16* v,
+                     const uint8_t* sep, int L, sep_stream_t stream);
+
+/*
  * sepcache_decode - single-query attention of each sequence's newest token over its cache.
  * Logical order = [initial | separators oldest first | window oldest first]; the key of rank p
  * is rotated by RoPE(p) and the query by RoPE(m), m = occupied - 1 (its own rank).

@@ -255,6 +255,17 @@ int sepcache_update(const SepCacheState* st, const sep_bf16* k_new, const sep_bf
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16* v,
+                     const uint8_t* sep, int L, sep_stream_t stream) {
+  int e = check_cache(st);
+  if (e != SEP_OK) return e;
+  if (!k || !v || !sep || L < 1) return SEP_ERR_INVALID_ARG;
+  if (st->s > 16384) return SEP_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v)) return SEP_ERR_MISALIGNED;
+  return cuda_status(sep::launch_sepcache_prefill(*st, k, v, sep, L,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int sepcache_decode(const SepCacheState* st, const sep_bf16* q, sep_bf16* o, float* lse,
                     float scale, sep_stream_t stream) {
   int e = check_cache(st);

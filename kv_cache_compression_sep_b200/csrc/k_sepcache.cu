@@ -128,6 +128,153 @@ __global__ void __launch_bounds__(128) sepcache_update_kernel(
   }
 }
 
+// ------------------------------------------------------------------ prefill
+// State after appending the L prompt tokens of every sequence one at a time to an empty cache,
+// in one pass (the same rule as sepcache_update, solved in closed form):
+//   initial slots 0..min(a, L)-1 hold tokens 0..min(a, L)-1;
+//   the window ring holds the last min(w, L - a) tokens, token u at ring index (u - a) mod w,
+//   its head at (L - a) mod w once the ring has wrapped;
+//   the tokens u in [a, L - w) have left the window; the k-th separator among them (k = 0,
+//   1, ...) went to separator ring index k mod s, so the ring keeps the last min(s, count) of
+//   them, its head at count mod s once full (nothing is kept when s = 0).
+// One CTA per (sequence, KV head): each scans the flags (block-wide exclusive scan) to place the
+// kept separators, copies its head's K/V rows, and the head-0 CTA writes the metadata and the
+// slot maps. K/V rows of unused slots are left as they are.
+constexpr int kPrefillThreads = 256;
+constexpr int kPrefillItems = 16;
+
+__global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
+    int L, int Hkv, int d, int a, int s, int w, const uint4* __restrict__ k_in,
+    const uint4* __restrict__ v_in, const uint8_t* __restrict__ sep_in, uint4* __restrict__ k_slots,
+    uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
+    int32_t* __restrict__ meta) {
+  extern __shared__ int s_seppos[];  // [s]: position of the separator at each ring index
+  __shared__ int s_warp[kPrefillThreads / 32];
+  __shared__ int s_total;
+  const int seq = blockIdx.x, head = blockIdx.y;
+  const int c = a + s + w;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint8_t* flags = sep_in + (size_t)seq * L;
+  const int ninit = min(a, L);
+  const int nwin = max(0, min(w, L - a));
+  const int left_end = max(a, L - w);  // tokens in [a, left_end) have left the window
+
+  // ---- pass 1: how many separators left the window
+  int cnt = 0;
+  for (int u = a + tid; u < left_end; u += kPrefillThreads) cnt += flags[u] != 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  if (lane == 0) s_warp[warp] = cnt;
+  __syncthreads();
+  if (tid == 0) {
+    int tot = 0;
+    for (int x = 0; x < kPrefillThreads / 32; ++x) tot += s_warp[x];
+    s_total = tot;
+  }
+  __syncthreads();
+  const int count = (s > 0) ? s_total : 0;
+  const int sep_cnt = min(s, count);
+  const int first_kept = count - sep_cnt;
+
+  // ---- pass 2: exclusive scan; the kept separators record their positions by ring index
+  if (sep_cnt > 0) {
+    int carry = 0;
+    for (int base = a; base < left_end; base += kPrefillThreads * kPrefillItems) {
+      const int u0 = base + tid * kPrefillItems;
+      uint32_t bits = 0;
+#pragma unroll
+      for (int q = 0; q < kPrefillItems; ++q)
+        if (u0 + q < left_end && flags[u0 + q] != 0) bits |= 1u << q;
+      const int n = __popc(bits);
+      int incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      __syncthreads();
+      if (lane == 31) s_warp[warp] = incl;
+      __syncthreads();
+      int before = carry;
+      for (int x = 0; x < warp; ++x) before += s_warp[x];
+      int k = before + incl - n;  // index of this thread's first separator
+#pragma unroll
+      for (int q = 0; q < kPrefillItems; ++q) {
+        if (bits & (1u << q)) {
+          if (k >= first_kept) s_seppos[k % s] = u0 + q;
+          ++k;
+        }
+      }
+      int blk = 0;
+      for (int x = 0; x < kPrefillThreads / 32; ++x) blk += s_warp[x];
+      carry += blk;
+    }
+  }
+  __syncthreads();
+
+  // slot -> original position (-1: unused)
+  auto pos_of = [&](int slot) -> int {
+    if (slot < a) return slot < ninit ? slot : -1;
+    if (slot < a + s) {
+      const int r = slot - a;
+      return (count >= s || r < count) ? s_seppos[r] : -1;
+    }
+    const int r = slot - a - s;
+    if (nwin == w || r < nwin) {
+      const int first = L - nwin;  // oldest token in the window
+      const int r0 = (first - a) % w;
+      return first + (r - r0 + w) % w;
+    }
+    return -1;
+  };
+
+  // ---- metadata and slot maps (once per sequence)
+  if (head == 0) {
+    for (int slot = tid; slot < c; slot += kPrefillThreads) {
+      const int pos = pos_of(slot);
+      slot_pos[(size_t)seq * c + slot] = pos;
+      slot_sep[(size_t)seq * c + slot] = (pos >= 0 && flags[pos] != 0) ? 1 : 0;
+    }
+    if (tid == 0) {
+      int32_t* m = meta + (size_t)seq * SEPCACHE_META;
+      m[SEPCACHE_META_T] = L;
+      m[SEPCACHE_META_NINIT] = ninit;
+      m[SEPCACHE_META_SEP_HEAD] = (count >= s && s > 0) ? count % s : 0;
+      m[SEPCACHE_META_SEP_CNT] = sep_cnt;
+      m[SEPCACHE_META_WIN_HEAD] = (L - a >= w) ? (L - a) % w : 0;
+      m[SEPCACHE_META_WIN_CNT] = nwin;
+    }
+  }
+  // ---- this head's K/V rows of the occupied slots (one warp per row, 16-byte vectors)
+  const int vec = d / 8;
+  const size_t dst_base = ((size_t)seq * Hkv + head) * c;
+  for (int slot = warp; slot < c; slot += kPrefillThreads / 32) {
+    const int pos = pos_of(slot);
+    if (pos < 0) continue;
+    const size_t src = (((size_t)seq * L + pos) * Hkv + head) * vec;
+    const size_t dst = (dst_base + slot) * vec;
+    for (int e = lane; e < vec; e += 32) {
+      k_slots[dst + e] = __ldg(k_in + src + e);
+      v_slots[dst + e] = __ldg(v_in + src + e);
+    }
+  }
+}
+
+cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, const void* v,
+                                    const uint8_t* sep, int L, cudaStream_t stream) {
+  const size_t smem = (size_t)max(st.s, 1) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(sepcache_prefill_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  sepcache_prefill_kernel<<<dim3(st.S, st.Hkv), kPrefillThreads, smem, stream>>>(
+      L, st.Hkv, st.d, st.a, st.s, st.w, static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), sep, reinterpret_cast<uint4*>(st.k_slots),
+      reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta);
+  return cudaGetLastError();
+}
+
 // Slot holding logical rank r (r < occupied).
 __device__ __forceinline__ int rank_to_slot(int r, int ninit, int sep_head, int sep_cnt,
                                             int win_head, int a, int s, int w) {

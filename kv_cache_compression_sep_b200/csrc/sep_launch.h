@@ -58,6 +58,8 @@ cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream);
 cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new,
                                    const void* v_new, const uint8_t* sep_new,
                                    cudaStream_t stream);
+cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, const void* v,
+                                    const uint8_t* sep, int L, cudaStream_t stream);
 cudaError_t launch_sepcache_decode(const SepCacheState& st, const void* q, void* o, float* lse,
                                    float scale, cudaStream_t stream);
 cudaError_t launch_sepcache_export(const SepCacheState& st, int32_t* pos_out, int32_t* count,

@@ -43,6 +43,7 @@ def _load():
         "sepcache_state_init": (I, [P, P]),
         "sepcache_update": (I, [P, P, P, P, P]),
         "sepcache_decode": (I, [P, P, P, P, F, P]),
+        "sepcache_prefill": (I, [P, P, P, P, I, P]),
         "sepcache_export_order": (I, [P, P, P, P]),
         "sep_last_device_error": (I, []),
         "sep_status_string": (ctypes.c_char_p, [I]),
@@ -251,6 +252,15 @@ class SepCache:
                                   self.slot_pos.data_ptr(), self.slot_sep.data_ptr(),
                                   self.meta.data_ptr(), self.rope_cs.data_ptr())
         _check(_lib.sepcache_state_init(ctypes.byref(self._st), _stream()), "sepcache_state_init")
+
+    def sepcache_prefill(self, k, v, sep):
+        """Seeds every sequence with a prompt: k, v [S, L, Hkv, d] bf16, sep [S, L] uint8."""
+        _cuda(k, torch.bfloat16, "k")
+        _cuda(v, torch.bfloat16, "v")
+        _cuda(sep, torch.uint8, "sep")
+        L = k.shape[1]
+        _check(_lib.sepcache_prefill(ctypes.byref(self._st), _ptr(k), _ptr(v), _ptr(sep), L,
+                                     _stream()), "sepcache_prefill")
 
     # checkpoint / resume: the whole state lives in these tensors (the cos/sin table is a pure
     # function of c, d and theta and is rebuilt by the constructor)

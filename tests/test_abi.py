@@ -129,3 +129,17 @@ def test_cache_rejects_bad_state(lib):
     assert f(ctypes.byref(st(k_slots=258)), P(256), P(256), P(256), None) == SEP_ERR_MISALIGNED
     assert f(ctypes.byref(st(rope_theta=0.0)), P(256), P(256), P(256), None) == SEP_ERR_INVALID_ARG
     assert f(ctypes.byref(st()), P(258), P(256), P(256), None) == SEP_ERR_MISALIGNED
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    f = lib.sepcache_prefill
+    f.restype = ctypes.c_int
+    P, I = ctypes.c_void_p, ctypes.c_int
+    st = _CacheState(S=2, Hq=8, Hkv=2, d=128, a=4, s=8, w=16, rope_theta=1e4, k_slots=256,
+                     v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_cs=256)
+    assert f(ctypes.byref(st), P(256), P(256), P(256), I(0), None) == SEP_ERR_INVALID_ARG
+    assert f(ctypes.byref(st), None, P(256), P(256), I(8), None) == SEP_ERR_INVALID_ARG
+    assert f(ctypes.byref(st), P(264), P(256), P(256), I(8), None) == SEP_ERR_MISALIGNED
+    big = _CacheState(S=2, Hq=8, Hkv=2, d=128, a=4, s=20000, w=16, rope_theta=1e4, k_slots=256,
+                      v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_cs=256)
+    assert f(ctypes.byref(big), P(256), P(256), P(256), I(8), None) == SEP_ERR_UNSUPPORTED

@@ -166,3 +166,49 @@ def test_checkpoint_resume_bit_identical(S):
         assert torch.equal(o1, o2) and torch.equal(l1, l2)
     for x, y in zip(ref_order, got_order):
         assert torch.equal(x.cpu(), y.cpu())
+
+
+@pytest.mark.parametrize("Sq,Hq,Hkv,d,a,s,w,L,p", [
+    (2, 8, 2, 128, 4, 6, 20, 3, 0.3),        # prompt shorter than the initial block
+    (2, 8, 2, 128, 4, 6, 20, 15, 0.3),       # window not yet full
+    (3, 8, 2, 128, 4, 6, 20, 200, 0.3),      # window wrapped, separator FIFO overflowed
+    (2, 4, 4, 64, 0, 3, 7, 100, 0.5),        # no initial block
+    (2, 8, 1, 128, 2, 0, 9, 60, 0.3),        # s = 0: separators dropped
+    (1, 16, 2, 64, 1, 2, 1, 40, 0.6),        # window of one slot
+    (2, 32, 8, 128, 4, 64, 732, 3000, 0.1),  # the decode configuration's capacities
+])
+def test_prefill_equals_sequential_updates(S, Sq, Hq, Hkv, d, a, s, w, L, p):
+    """sepcache_prefill leaves the state L sepcache_update calls leave (bit-identical), whose
+    trajectory is the oracle's; a decode step after either gives identical outputs."""
+    import torch
+    g = torch.Generator().manual_seed(L * 7 + w)
+    k = torch.randn(Sq, L, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(Sq, L, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    sep = (torch.rand(Sq, L, generator=g) < p).to(torch.uint8).cuda()
+    seq_cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, 500000.0)
+    for t in range(L):
+        seq_cache.sepcache_update(k[:, t].contiguous(), v[:, t].contiguous(), sep[:, t].contiguous())
+    pre_cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, 500000.0)
+    pre_cache.sepcache_prefill(k, v, sep)
+    torch.cuda.synchronize()
+    assert S.sep_last_device_error() == 0
+    for name in ("meta", "slot_pos", "slot_sep", "k_slots", "v_slots"):
+        assert torch.equal(getattr(seq_cache, name), getattr(pre_cache, name)), name
+    pos, cnt = pre_cache.sepcache_export_order()
+    pos, cnt = pos.cpu().numpy(), cnt.cpu().numpy()
+    flags = sep.cpu().numpy()
+    for sq in range(Sq):
+        sim = C.SepCacheSim(a, s, w)
+        for t in range(L):
+            sim.append(bool(flags[sq, t]))
+        order = sim.order()
+        assert int(cnt[sq]) == len(order)
+        assert pos[sq, : len(order)].tolist() == list(order)
+    q = torch.randn(Sq, Hq, d, generator=g).to(torch.bfloat16).cuda()
+    kn = torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    sn = torch.zeros(Sq, dtype=torch.uint8, device="cuda")
+    outs = []
+    for cache in (seq_cache, pre_cache):
+        cache.sepcache_update(kn, kn, sn)
+        outs.append(cache.sepcache_decode(q))
+    assert torch.equal(outs[0], outs[1])

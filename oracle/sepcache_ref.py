@@ -7,15 +7,22 @@ Separator Cache that keeps only separator KV of older tokens, with total capacit
 say positions are taken inside the cache, not in the original text.
 
 Readings where the pages are silent (listed again in the design doc):
-* Fixed partitions c = a + s + w; the Past Window Cache has size 0, so compression happens
-  one token at a time: when the window overflows, its oldest token moves to the separator
-  cache if it is a separator and is evicted otherwise; when the separator cache overflows,
-  its oldest entry is evicted. The first a tokens go to the initial cache whatever their flag.
+* Without a usage threshold (c = None): fixed partitions a + s + w and a Past Window Cache of
+  size 0, so compression happens one token at a time: when the window overflows, its oldest
+  token moves to the separator cache if it is a separator and is evicted otherwise; when the
+  separator cache overflows, its oldest entry is evicted.
+* With a usage threshold c (> a + s + w): a token leaving the window goes to the Past Window
+  Cache; right after an append that makes initial + separators + past + window reach c, the
+  past window's separators move to the separator cache oldest first (which evicts its oldest
+  entries beyond s) and the rest of the past window is dropped. The usage after a step is
+  therefore always below c.
+* The first a tokens go to the initial cache whatever their flag.
 * Per step: the update happens first, then the new token's query attends to every retained
   slot, itself included.
 * Positional-encoding shifting: the position of a retained key is its rank in the logical
-  order [initial | separators oldest first | window oldest first]; the query's position is
-  its own rank (occupied - 1). Keys are kept un-rotated and rotated afresh at every step.
+  order [initial | separators oldest first | past window oldest first | window oldest first];
+  the query's position is its own rank (occupied - 1). Keys are kept un-rotated and rotated
+  afresh at every step.
 * RoPE convention: rotate-half pairs (k, k + d/2) with angle p * theta^(-2k/d).
 """
 
@@ -32,13 +39,23 @@ class SepCacheSim:
     Holds original token positions only; the K/V content is looked up by position.
     """
 
-    def __init__(self, a, s, w):
+    def __init__(self, a, s, w, c=None):
         assert a >= 0 and s >= 0 and w >= 1
-        self.a, self.s, self.w = a, s, w
+        assert c is None or c > a + s + w
+        self.a, self.s, self.w, self.c = a, s, w, c
         self.initial = []
         self.seps = deque()
+        self.past = []
         self.window = deque()
         self.t = 0
+
+    def usage(self):
+        return len(self.initial) + len(self.seps) + len(self.past) + len(self.window)
+
+    def _to_separators(self, pos):
+        self.seps.append(pos)
+        if len(self.seps) > self.s:
+            self.seps.popleft()
 
     def append(self, is_sep):
         """Add the next token (original position self.t) and compress if over capacity."""
@@ -50,14 +67,21 @@ class SepCacheSim:
         self.window.append((tok, bool(is_sep)))
         if len(self.window) > self.w:
             old, old_sep = self.window.popleft()
-            if old_sep:
-                self.seps.append(old)
-                if len(self.seps) > self.s:
-                    self.seps.popleft()
+            if self.c is None:
+                if old_sep:
+                    self._to_separators(old)
+            else:
+                self.past.append((old, old_sep))
+        if self.c is not None and self.usage() >= self.c:
+            for p, p_sep in self.past:
+                if p_sep:
+                    self._to_separators(p)
+            self.past = []
 
     def order(self):
         """Retained original positions in logical order; a key's rank is its in-cache position."""
-        return list(self.initial) + list(self.seps) + [p for p, _ in self.window]
+        return (list(self.initial) + list(self.seps) + [p for p, _ in self.past] +
+                [p for p, _ in self.window])
 
 
 def rope_rotate(x, pos, theta):

@@ -111,3 +111,45 @@ def test_decode_without_eviction_is_causal_rope_attention():
     np.testing.assert_allclose(o, ref, atol=1e-12)
     s = 0.3 * np.einsum("khd,hd->hk", np.repeat(kr, G, axis=1), qr)
     np.testing.assert_allclose(lse, np.log(np.exp(s).sum(1)), atol=1e-12)
+
+
+# ---------------------------------------------------------------- Past Window Cache (usage c)
+def test_golden_trajectory_past_window():
+    g = load_golden("sepcache_past_a1_s2_w2_c7.txt")
+    sim = C.SepCacheSim(g["a"][0], g["s"][0], g["w"][0], g["c"][0])
+    seps = set(g["sep"])
+    for t in sorted(g["step"]):
+        sim.append(t in seps)
+        assert sim.order() == g["step"][t], t
+        assert sim.usage() < g["c"][0]
+
+
+@pytest.mark.parametrize("a,s,w,c,p", [(4, 64, 256, 800, 0.1), (0, 3, 5, 20, 0.3),
+                                       (2, 0, 4, 12, 0.5), (1, 2, 1, 5, 0.9), (3, 1, 2, 7, 0.0)])
+def test_past_window_invariants(a, s, w, c, p):
+    rng = np.random.default_rng(a * 100 + s + c)
+    steps = 3000
+    flags = rng.random(steps) < p
+    sim = C.SepCacheSim(a, s, w, c)
+    ref = C.SepCacheSim(a, s, w)  # the one-token-at-a-time rule
+    for t in range(steps):
+        sim.append(flags[t])
+        ref.append(flags[t])
+        order = sim.order()
+        assert len(order) < c
+        assert order == sorted(order) and len(set(order)) == len(order)
+        assert order[-1] == t
+        n_init = min(t + 1, a)
+        assert order[:n_init] == list(range(n_init))
+        n_win = min(t + 1 - n_init, w)
+        assert order[len(order) - n_win:] == list(range(t + 1 - n_win, t + 1))
+        # middle = separators (all flagged, at most s) then the past window, a contiguous run
+        # of the tokens that left the window since the last compression
+        n_past = len(sim.past)
+        past = order[len(order) - n_win - n_past:len(order) - n_win]
+        assert past == list(range(t + 1 - n_win - n_past, t + 1 - n_win))
+        mid = order[n_init:len(order) - n_win - n_past]
+        assert len(mid) <= s and all(flags[j] for j in mid)
+        # right after a compression the retained set is the one-token-at-a-time rule's
+        if n_past == 0:
+            assert order == ref.order(), t

@@ -557,6 +557,48 @@ def single_row(args, dev):
                     "gbs_update_plus_decode": byts / (ms * 1e-3) / 1e9})
         del step
         return out
+    if args.workload == "decode-past":
+        # SepCache with a Past Window: a=4, s=64, w=256, compressed when the usage reaches
+        # c=800; R consecutive steps (distinct inputs) replayed from the same starting state
+        dc, R, c_use, w_p = workloads.SEPCACHE_DECODE, 512, 800, 256
+        cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, dc.s, w_p, dc.theta, device=dev,
+                           c=c_use)
+        warm = workloads.decode_chunk(dc, 0, 2048, device=dev)
+        for t in range(2048):
+            cache.sepcache_update(warm["k"][t], warm["v"][t], warm["sep"][t])
+        pool = workloads.decode_chunk(dc, 2048, R, device=dev)
+        o = torch.empty_like(pool["q"][0])
+        state0 = cache.state_dict()
+        occ = []
+        for t in range(R):  # untimed pass: the occupancy each step reads
+            cache.sepcache_update(pool["k"][t], pool["v"][t], pool["sep"][t])
+            cache.sepcache_decode(pool["q"][t], out=o)
+            m = cache.meta.cpu()
+            occ.append(int((m[:, 1] + m[:, 3] + m[:, 5] + m[:, 6]).sum()))
+
+        def steps():
+            for t in range(R):
+                cache.sepcache_update(pool["k"][t], pool["v"][t], pool["sep"][t])
+                cache.sepcache_decode(pool["q"][t], out=o)
+        cache.load_state_dict(state0)
+        g = capture(steps)
+        times = []
+        st = torch.cuda.current_stream()
+        for _ in range(max(3, args.steps)):
+            cache.load_state_dict(state0)  # also evicts the cache lines of the previous replay
+            flush_l2(flush)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            g.replay()
+            e1.record(st)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.mean(times) / R
+        byts = (sum(occ) / R * dc.Hkv * dc.d * 4 + dc.S * (4 * dc.Hq * dc.d + 4 * dc.Hkv * dc.d))
+        out.update({"a": dc.a, "s": dc.s, "w": w_p, "c": c_use,
+                    "mean_occupancy": sum(occ) / R / dc.S, "us_per_step": ms * 1e3,
+                    "tokens_per_s": dc.S / (ms * 1e-3), "gbs_update_plus_decode": byts / (ms * 1e-3) / 1e9})
+        return out
     if args.workload == "cache-prefill":
         # seed 64 caches (the decode configuration's capacities) from 8192-token prompts
         dc, Lp = workloads.SEPCACHE_DECODE, 8192
@@ -610,7 +652,7 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="train-decode",
                     choices=["train-decode", "pythia-train", "llama-prefill", "long-context",
-                             "long-context-dense", "decode", "cache-prefill"])
+                             "long-context-dense", "decode", "decode-past", "cache-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",

@@ -151,19 +151,22 @@ int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const se
                        void* workspace, size_t workspace_bytes, sep_stream_t stream);
 
 /*
- * SepCache: streaming KV cache of S independent sequences with capacity c = a + s + w slots
- * per sequence: a initial slots, s separator slots (FIFO), w local-window slots (FIFO)
- * ("SepLLM's Architecture: Composing Efficiency", beiduofen.top). Keys are stored without
+ * SepCache: streaming KV cache of S independent sequences ("SepLLM's Architecture: Composing
+ * Efficiency", beiduofen.top): a initial slots, a separator FIFO of s slots, a local-window
+ * FIFO of w slots and, when the usage threshold c is non-zero, a Past Window of P = c - a - w
+ * slots that holds the tokens leaving the window until the total usage reaches c. With c = 0
+ * there is no Past Window and compression is one token at a time. Keys are stored without
  * rotary embedding; sepcache_decode applies RoPE at in-cache positions (positional-encoding
  * shifting, SepLLM project card, "Limitations & Caveats").
  *
- * Every pointer below is caller-owned device memory; the struct itself lives on the host and
- * is read by each call. Sizes in elements:
- *   k_slots, v_slots  S * Hkv * c * d bf16   slot-major per (sequence, KV head)
- *   slot_pos          S * c int32             original position held by each slot (-1 empty)
- *   slot_sep          S * c uint8             separator flag of each slot's token
+ * Slots per sequence: n = a + s + P + w (P = 0 when c = 0), in this order: initial, separator
+ * ring, past window, window ring. Every pointer below is caller-owned device memory; the
+ * struct itself lives on the host and is read by each call. Sizes in elements:
+ *   k_slots, v_slots  S * Hkv * n * d bf16   slot-major per (sequence, KV head)
+ *   slot_pos          S * n int32             original position held by each slot (-1 empty)
+ *   slot_sep          S * n uint8             separator flag of each slot's token
  *   meta              S * SEPCACHE_META int32 per-sequence counters (see below)
- *   rope_cs           c * d float             cos/sin table of in-cache positions 0..c-1
+ *   rope_cs           n * d float             cos/sin table of in-cache positions 0..n-1
  */
 #define SEPCACHE_META 8
 /* meta[seq * SEPCACHE_META + ...] */
@@ -173,10 +176,12 @@ int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const se
 #define SEPCACHE_META_SEP_CNT 3   /* separator FIFO: entries */
 #define SEPCACHE_META_WIN_HEAD 4  /* window FIFO: ring index of the oldest entry */
 #define SEPCACHE_META_WIN_CNT 5   /* window FIFO: entries */
+#define SEPCACHE_META_PAST_CNT 6  /* past window: entries (c > 0) */
 
 typedef struct SepCacheState {
   int32_t S, Hq, Hkv, d;     /* sequences, query heads, KV heads, head dim (d = 128 or 64) */
-  int32_t a, s, w;           /* initial / separator / window capacities, c = a + s + w */
+  int32_t a, s, w;           /* initial / separator / window capacities */
+  int32_t c;                 /* usage threshold of the Past Window (0: none; else > a + s + w) */
   float rope_theta;          /* RoPE base: angle of pair k at position p = p * theta^(-2k/d) */
   sep_bf16* k_slots;
   sep_bf16* v_slots;
@@ -193,8 +198,12 @@ int sepcache_state_init(const SepCacheState* st, sep_stream_t stream);
  * sepcache_update - append one token to every sequence (one kernel).
  * k_new, v_new [S, Hkv, d] un-rotated; sep_new [S] uint8. Token t of a sequence goes to
  * initial slot t when t < a; otherwise to the window. If the window then holds more than w
- * tokens its oldest token leaves: into the separator FIFO if it is a separator, else it is
- * dropped; if the separator FIFO then holds more than s entries its oldest is dropped.
+ * tokens its oldest token leaves. With c = 0 it goes into the separator FIFO if it is a
+ * separator and is dropped otherwise. With c > 0 it goes to the Past Window, and when the
+ * total usage (initial + separators + past + window) then reaches c the Past Window is
+ * compressed: its separators enter the separator FIFO oldest first, the rest is dropped.
+ * Whenever the separator FIFO holds more than s entries its oldest are dropped.
+ * With c > 0, min(s, c - a - w) must be at most 4096 (SEP_ERR_UNSUPPORTED otherwise).
  */
 int sepcache_update(const SepCacheState* st, const sep_bf16* k_new, const sep_bf16* v_new,
                     const uint8_t* sep_new, sep_stream_t stream);
@@ -207,15 +216,16 @@ int sepcache_update(const SepCacheState* st, const sep_bf16* k_new, const sep_bf
  * to streaming decode ("How SepLLM reorchestrates the language model...", "SepLLM's
  * Architecture: Composing Efficiency": initial, separator and local-window blocks).
  * k, v [S, L, Hkv, d] un-rotated (the layout sep_attn_fwd reads); sep [S, L] uint8. L >= 1;
- * s <= 16384 (SEP_ERR_UNSUPPORTED otherwise).
+ * s <= 16384 and c = 0 (SEP_ERR_UNSUPPORTED otherwise).
  */
 int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16* v,
                      const uint8_t* sep, int L, sep_stream_t stream);
 
 /*
  * sepcache_decode - single-query attention of each sequence's newest token over its cache.
- * Logical order = [initial | separators oldest first | window oldest first]; the key of rank p
- * is rotated by RoPE(p) and the query by RoPE(m), m = occupied - 1 (its own rank).
+ * Logical order = [initial | separators oldest first | past window oldest first | window
+ * oldest first]; the key of rank p is rotated by RoPE(p) and the query by RoPE(m),
+ * m = occupied - 1 (its own rank).
  * q [S, Hq, d] un-rotated; o [S, Hq, d] bf16; lse [S, Hq] fp32 natural log (nullable).
  * Call after sepcache_update of the same step.
  */

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 
@@ -236,6 +237,9 @@ static int check_cache(const SepCacheState* st) {
   if (!aligned16(st->k_slots) || !aligned16(st->v_slots) || !aligned16(st->rope_cs))
     return SEP_ERR_MISALIGNED;
   if (!(st->rope_theta > 0.f)) return SEP_ERR_INVALID_ARG;
+  // usage threshold of the Past Window: 0 (none) or above the three fixed blocks
+  if (st->c < 0 || (st->c > 0 && st->c <= st->a + st->s + st->w)) return SEP_ERR_INVALID_ARG;
+  if (st->c > 0 && std::min(st->s, st->c - st->a - st->w) > 4096) return SEP_ERR_UNSUPPORTED;
   return SEP_OK;
 }
 
@@ -260,7 +264,7 @@ int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16*
   int e = check_cache(st);
   if (e != SEP_OK) return e;
   if (!k || !v || !sep || L < 1) return SEP_ERR_INVALID_ARG;
-  if (st->s > 16384) return SEP_ERR_UNSUPPORTED;
+  if (st->s > 16384 || st->c != 0) return SEP_ERR_UNSUPPORTED;
   if (!aligned16(k) || !aligned16(v)) return SEP_ERR_MISALIGNED;
   return cuda_status(sep::launch_sepcache_prefill(*st, k, v, sep, L,
                                                   reinterpret_cast<cudaStream_t>(stream)));

@@ -3,14 +3,18 @@
 //
 // Cache blocks ("How SepLLM reorchestrates the language model...", beiduofen.top, section
 // "SepLLM's Architecture: Composing Efficiency"): a initial slots, a separator FIFO of s slots,
-// a local-window FIFO of w slots. When the window overflows, its oldest token moves to the
-// separator FIFO if it is a separator and is dropped otherwise; the separator FIFO drops its
-// oldest entry when full. Positions are ranks inside the cache (SepLLM project card,
-// "Limitations & Caveats": streaming needs positional-encoding shifting), so a key is rotated
-// by RoPE(rank) at every step and the query by RoPE(occupied - 1).
+// a local-window FIFO of w slots and, with a usage threshold c > 0, a Past Window of
+// P = c - a - w slots. When the window overflows, its oldest token leaves: with c = 0 it moves
+// to the separator FIFO if it is a separator and is dropped otherwise; with c > 0 it goes to
+// the Past Window, which is compressed (its separators to the FIFO, the rest dropped) by the
+// step that makes the total usage reach c. The separator FIFO drops its oldest entries when
+// full. Positions are ranks inside the cache (SepLLM project card, "Limitations & Caveats":
+// streaming needs positional-encoding shifting), so a key is rotated by RoPE(rank) at every
+// step and the query by RoPE(occupied - 1).
 //
-// Slot storage per (sequence, KV head) is [c][d] with c = a + s + w: slots 0..a-1 initial,
-// a..a+s-1 separator ring, a+s..c-1 window ring. Keys are stored without rotation.
+// Slot storage per (sequence, KV head) is [n][d], n = a + s + P + w: initial slots, the
+// separator ring, the past window (a plain array, emptied by each compression), the window
+// ring. Keys are stored without rotation.
 //
 // Decode: one CTA per (sequence, KV head), all of them resident at once (4 per SM), so the
 // whole cache streams in a single wave. Each CTA streams its ranks through a shared-memory ring
@@ -50,81 +54,165 @@ __global__ void sepcache_init_kernel(int S, int c, int d, double theta, int32_t*
 }
 
 // ------------------------------------------------------------------ update
-// One CTA per sequence. Thread 0 plans the move, all threads copy rows (16-byte vectors).
-__global__ void __launch_bounds__(128) sepcache_update_kernel(
-    int Hkv, int d, int a, int s, int w, uint4* __restrict__ k_slots, uint4* __restrict__ v_slots,
-    int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep, int32_t* __restrict__ meta,
-    const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+// One CTA per sequence. Thread 0 plans the step, all threads copy rows (16-byte vectors). With a
+// Past Window (P > 0) the step that makes the usage reach c then compresses it: a block-wide
+// scan numbers the past window's separators k = 0, 1, ... (oldest first); the FIFO keeps the
+// last s of its current entries followed by them, so separator k lands at ring index
+// (sep_head + sep_cnt + k) mod s and is kept when it is among the last s (k >= nnew - s).
+constexpr int kUpdateThreads = 128;
+
+__global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
+    int Hkv, int d, int a, int s, int w, int P, int c, uint4* __restrict__ k_slots,
+    uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
+    int32_t* __restrict__ meta, const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
     const uint8_t* __restrict__ sep_new) {
+  extern __shared__ int2 s_moves[];  // compression: (past slot, separator slot), min(s, P) at most
   const int seq = blockIdx.x;
-  const int c = a + s + w;
+  const int ns = a + s + P + w;       // slots per sequence
+  const int win_base = a + s + P;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* m = meta + (size_t)seq * SEPCACHE_META;
-  __shared__ int plan[4];  // slot_new, move_from, move_to, t
-  if (threadIdx.x == 0) {
+  // slot_new, move_from, move_to, t, compress, past_cnt, sep_head, sep_cnt
+  __shared__ int plan[8];
+  __shared__ int s_warp[kUpdateThreads / 32];
+  if (tid == 0) {
     const int t = m[SEPCACHE_META_T];
     int slot_new, move_from = -1, move_to = -1;
+    int ninit = m[SEPCACHE_META_NINIT];
+    int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
+    int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
+    int past_cnt = (P > 0) ? m[SEPCACHE_META_PAST_CNT] : 0;
     if (t < a) {
       slot_new = t;
-      m[SEPCACHE_META_NINIT] = t + 1;
+      ninit = t + 1;
+    } else if (win_cnt < w) {
+      slot_new = win_base + (win_head + win_cnt) % w;
+      ++win_cnt;
     } else {
-      int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
-      if (win_cnt < w) {
-        slot_new = a + s + (win_head + win_cnt) % w;
-        m[SEPCACHE_META_WIN_CNT] = win_cnt + 1;
-      } else {
-        // window full: its oldest token leaves and the new token takes its slot
-        const int old_slot = a + s + win_head;
-        if (slot_sep[(size_t)seq * c + old_slot] && s > 0) {
-          int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
-          int to;
-          if (sep_cnt < s) {
-            to = a + (sep_head + sep_cnt) % s;
-            m[SEPCACHE_META_SEP_CNT] = sep_cnt + 1;
-          } else {  // separator FIFO full: the oldest separator is dropped
-            to = a + sep_head;
-            m[SEPCACHE_META_SEP_HEAD] = (sep_head + 1) % s;
-          }
-          move_from = old_slot;
-          move_to = to;
+      // window full: its oldest token leaves and the new token takes its slot
+      const int old_slot = win_base + win_head;
+      if (P > 0) {
+        move_from = old_slot;
+        move_to = a + s + past_cnt;
+        ++past_cnt;
+      } else if (slot_sep[(size_t)seq * ns + old_slot] && s > 0) {
+        if (sep_cnt < s) {
+          move_to = a + (sep_head + sep_cnt) % s;
+          ++sep_cnt;
+        } else {  // separator FIFO full: the oldest separator is dropped
+          move_to = a + sep_head;
+          sep_head = (sep_head + 1) % s;
         }
-        slot_new = old_slot;
-        m[SEPCACHE_META_WIN_HEAD] = (win_head + 1) % w;
+        move_from = old_slot;
       }
+      slot_new = old_slot;
+      win_head = (win_head + 1) % w;
     }
+    const bool compress = P > 0 && ninit + sep_cnt + past_cnt + win_cnt >= c;
     m[SEPCACHE_META_T] = t + 1;
+    m[SEPCACHE_META_NINIT] = ninit;
+    m[SEPCACHE_META_SEP_HEAD] = sep_head;
+    m[SEPCACHE_META_SEP_CNT] = sep_cnt;
+    m[SEPCACHE_META_WIN_HEAD] = win_head;
+    m[SEPCACHE_META_WIN_CNT] = win_cnt;
+    if (P > 0) m[SEPCACHE_META_PAST_CNT] = past_cnt;
     plan[0] = slot_new;
     plan[1] = move_from;
     plan[2] = move_to;
     plan[3] = t;
+    plan[4] = compress ? 1 : 0;
+    plan[5] = past_cnt;
+    plan[6] = sep_head;
+    plan[7] = sep_cnt;
   }
   __syncthreads();
   const int slot_new = plan[0], move_from = plan[1], move_to = plan[2], t = plan[3];
   const int vec = d / 8;  // 16-byte vectors per row
-  const size_t seq_rows = (size_t)seq * Hkv * c;
-  if (move_from >= 0) {
-    for (int e = threadIdx.x; e < Hkv * vec; e += blockDim.x) {
+  const size_t seq_rows = (size_t)seq * Hkv * ns;
+  auto copy_row = [&](int from, int to) {  // all heads, all threads
+    for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
       const int hh = e / vec, q = e % vec;
-      const size_t src = (seq_rows + (size_t)hh * c + move_from) * vec + q;
-      const size_t dst = (seq_rows + (size_t)hh * c + move_to) * vec + q;
+      const size_t src = (seq_rows + (size_t)hh * ns + from) * vec + q;
+      const size_t dst = (seq_rows + (size_t)hh * ns + to) * vec + q;
       k_slots[dst] = k_slots[src];
       v_slots[dst] = v_slots[src];
     }
-    if (threadIdx.x == 0) {
-      slot_pos[(size_t)seq * c + move_to] = slot_pos[(size_t)seq * c + move_from];
-      slot_sep[(size_t)seq * c + move_to] = 1;
+  };
+  if (move_from >= 0) {
+    copy_row(move_from, move_to);
+    if (tid == 0) {
+      slot_pos[(size_t)seq * ns + move_to] = slot_pos[(size_t)seq * ns + move_from];
+      slot_sep[(size_t)seq * ns + move_to] = slot_sep[(size_t)seq * ns + move_from];
     }
     __syncthreads();
   }
-  for (int e = threadIdx.x; e < Hkv * vec; e += blockDim.x) {
+  for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
     const int hh = e / vec, q = e % vec;
-    const size_t dst = (seq_rows + (size_t)hh * c + slot_new) * vec + q;
+    const size_t dst = (seq_rows + (size_t)hh * ns + slot_new) * vec + q;
     const size_t src = ((size_t)seq * Hkv + hh) * vec + q;
     k_slots[dst] = k_new[src];
     v_slots[dst] = v_new[src];
   }
-  if (threadIdx.x == 0) {
-    slot_pos[(size_t)seq * c + slot_new] = t;
-    slot_sep[(size_t)seq * c + slot_new] = sep_new[seq] != 0;
+  if (tid == 0) {
+    slot_pos[(size_t)seq * ns + slot_new] = t;
+    slot_sep[(size_t)seq * ns + slot_new] = sep_new[seq] != 0;
+  }
+  if (!plan[4]) return;
+
+  // ---- compression of the past window [a + s, a + s + past_cnt)
+  __syncthreads();
+  const int past_cnt = plan[5], sep_head = plan[6], sep_cnt = plan[7];
+  const uint8_t* pflag = slot_sep + (size_t)seq * ns + a + s;
+  int cnt = 0;
+  for (int i = tid; i < past_cnt; i += kUpdateThreads) cnt += pflag[i] != 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  if (lane == 0) s_warp[warp] = cnt;
+  __syncthreads();
+  int nnew = 0;
+  for (int x = 0; x < kUpdateThreads / 32; ++x) nnew += s_warp[x];
+  const int kfirst = (s > 0) ? max(0, nnew - s) : nnew;  // the first new separator kept
+  int carry = 0;
+  for (int base = 0; base < past_cnt; base += kUpdateThreads) {
+    const int i = base + tid;
+    const int f = (i < past_cnt && pflag[i] != 0) ? 1 : 0;
+    int incl = f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    __syncthreads();
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int k = carry + incl - f;
+    for (int x = 0; x < warp; ++x) k += s_warp[x];
+    if (f && k >= kfirst)
+      s_moves[k - kfirst] = make_int2(a + s + i, a + (sep_head + sep_cnt + k) % s);
+    for (int x = 0; x < kUpdateThreads / 32; ++x) carry += s_warp[x];
+  }
+  __syncthreads();
+  const int nkept = nnew - kfirst;
+  for (int j = 0; j < nkept; ++j) {
+    const int2 mv = s_moves[j];
+    copy_row(mv.x, mv.y);
+    if (tid == 0) {
+      slot_pos[(size_t)seq * ns + mv.y] = slot_pos[(size_t)seq * ns + mv.x];
+      slot_sep[(size_t)seq * ns + mv.y] = 1;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < past_cnt; i += kUpdateThreads) {  // the past window is empty again
+    slot_pos[(size_t)seq * ns + a + s + i] = -1;
+    slot_sep[(size_t)seq * ns + a + s + i] = 0;
+  }
+  if (tid == 0) {
+    const int total = sep_cnt + nnew;
+    if (s > 0) {
+      m[SEPCACHE_META_SEP_HEAD] = (total > s) ? (sep_head + total - s) % s : sep_head;
+      m[SEPCACHE_META_SEP_CNT] = min(total, s);
+    }
+    m[SEPCACHE_META_PAST_CNT] = 0;
   }
 }
 
@@ -277,12 +365,15 @@ cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, cons
 
 // Slot holding logical rank r (r < occupied).
 __device__ __forceinline__ int rank_to_slot(int r, int ninit, int sep_head, int sep_cnt,
-                                            int win_head, int a, int s, int w) {
+                                            int past_cnt, int win_head, int a, int s, int P,
+                                            int w) {
   if (r < ninit) return r;
   r -= ninit;
   if (r < sep_cnt) return a + (sep_head + r) % s;
   r -= sep_cnt;
-  return a + s + (win_head + r) % w;
+  if (r < past_cnt) return a + s + r;
+  r -= past_cnt;
+  return a + s + P + (win_head + r) % w;
 }
 
 // N consecutive bf16 (N = 2 or 4, 4- or 8-byte aligned) to fp32.
@@ -340,7 +431,7 @@ struct DecSmem {
 
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
-    sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int w,
+    sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int P, int w,
                            const __nv_bfloat16* __restrict__ k_slots,
                            const __nv_bfloat16* __restrict__ v_slots,
                            const int32_t* __restrict__ meta, const float2* __restrict__ rope_cs,
@@ -349,7 +440,7 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
   constexpr int HP = D / 32;       // rotation pairs per lane
   constexpr int HALF = D / 2;
   const int kvh = blockIdx.x, seq = blockIdx.y;
-  const int c = a + s + w;
+  const int c = a + s + P + w;  // slots per sequence (and rows of the cos/sin table)
   const int tid = threadIdx.x, lane16 = tid & 15, hw = tid >> 4, warp = tid >> 5;
   extern __shared__ __align__(128) uint8_t dsm_raw[];
   DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
@@ -358,7 +449,8 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
   const int ninit = m[SEPCACHE_META_NINIT];
   const int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
   const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
-  const int occ = ninit + sep_cnt + win_cnt;
+  const int past_cnt = (P > 0) ? m[SEPCACHE_META_PAST_CNT] : 0;
+  const int occ = ninit + sep_cnt + past_cnt + win_cnt;
   const int mq = occ - 1;  // the query's own rank
   const int r0 = 0, r1 = occ;
   const int nchunks = r1 > r0 ? (r1 - r0 + kChunk - 1) / kChunk : 0;
@@ -371,7 +463,7 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
     const int rows = min(kChunk, r1 - c0);
     mbar_arrive_expect_tx(&sm.full[st], (uint32_t)(rows * D * 2 * 2));
     // ranks map to slots piecewise contiguously: initial block, then the separator ring, then
-    // the window ring; a run ends at a block boundary or where a ring wraps
+    // the past window, then the window ring; a run ends at a block boundary or a ring wrap
     int r = c0;
     const int end = c0 + rows;
     while (r < end) {
@@ -383,9 +475,12 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
         const int x = (sep_head + (r - ninit)) % s;
         slot = a + x;
         len = min(min(end, ninit + sep_cnt) - r, s - x);
+      } else if (r < ninit + sep_cnt + past_cnt) {
+        slot = a + s + (r - ninit - sep_cnt);
+        len = min(end, ninit + sep_cnt + past_cnt) - r;
       } else {
-        const int x = (win_head + (r - ninit - sep_cnt)) % w;
-        slot = a + s + x;
+        const int x = (win_head + (r - ninit - sep_cnt - past_cnt)) % w;
+        slot = a + s + P + x;
         len = min(end - r, w - x);
       }
       const size_t src = (row_base + slot) * D;
@@ -602,27 +697,33 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
 }
 
 // ------------------------------------------------------------------ export order
-__global__ void sepcache_export_kernel(int a, int s, int w, const int32_t* __restrict__ meta,
+__global__ void sepcache_export_kernel(int a, int s, int P, int w,
+                                       const int32_t* __restrict__ meta,
                                        const int32_t* __restrict__ slot_pos,
                                        int32_t* __restrict__ pos_out, int32_t* __restrict__ count) {
   const int seq = blockIdx.x;
-  const int c = a + s + w;
+  const int c = a + s + P + w;
   const int32_t* m = meta + (size_t)seq * SEPCACHE_META;
   const int ninit = m[SEPCACHE_META_NINIT];
   const int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
   const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
-  const int occ = ninit + sep_cnt + win_cnt;
+  const int past_cnt = (P > 0) ? m[SEPCACHE_META_PAST_CNT] : 0;
+  const int occ = ninit + sep_cnt + past_cnt + win_cnt;
   for (int r = threadIdx.x; r < c; r += blockDim.x) {
     pos_out[(size_t)seq * c + r] =
-        r < occ ? slot_pos[(size_t)seq * c +
-                           rank_to_slot(r, ninit, sep_head, sep_cnt, win_head, a, s, w)]
+        r < occ ? slot_pos[(size_t)seq * c + rank_to_slot(r, ninit, sep_head, sep_cnt, past_cnt,
+                                                          win_head, a, s, P, w)]
                 : -1;
   }
   if (threadIdx.x == 0) count[seq] = occ;
 }
 
+// Past Window slots and slots per sequence of a cache state.
+static int past_slots(const SepCacheState& st) { return st.c > 0 ? st.c - st.a - st.w : 0; }
+static int cache_slots(const SepCacheState& st) { return st.a + st.s + past_slots(st) + st.w; }
+
 cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream) {
-  const int c = st.a + st.s + st.w;
+  const int c = cache_slots(st);
   sepcache_init_kernel<<<64, 256, 0, stream>>>(st.S, c, st.d, (double)st.rope_theta, st.meta,
                                                st.slot_pos, st.slot_sep, st.rope_cs);
   return cudaGetLastError();
@@ -630,8 +731,10 @@ cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream) {
 
 cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new, const void* v_new,
                                    const uint8_t* sep_new, cudaStream_t stream) {
-  sepcache_update_kernel<<<st.S, 128, 0, stream>>>(
-      st.Hkv, st.d, st.a, st.s, st.w, reinterpret_cast<uint4*>(st.k_slots),
+  const int P = past_slots(st);
+  const size_t smem = (size_t)max(1, min(st.s, P)) * sizeof(int2);  // compression moves
+  sepcache_update_kernel<<<st.S, kUpdateThreads, smem, stream>>>(
+      st.Hkv, st.d, st.a, st.s, st.w, P, st.c, reinterpret_cast<uint4*>(st.k_slots),
       reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta,
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), sep_new);
   return cudaGetLastError();
@@ -653,7 +756,8 @@ static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void*
   }
   dim3 grid(st.Hkv, st.S);
   sepcache_decode_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(
-      st.Hq, st.Hkv, st.a, st.s, st.w, reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
+      st.Hq, st.Hkv, st.a, st.s, past_slots(st), st.w,
+      reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
       reinterpret_cast<const __nv_bfloat16*>(st.v_slots), st.meta,
       reinterpret_cast<const float2*>(st.rope_cs), static_cast<const __nv_bfloat16*>(q),
       static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f, device_error_word());
@@ -679,8 +783,8 @@ cudaError_t launch_sepcache_decode(const SepCacheState& st, const void* q, void*
 
 cudaError_t launch_sepcache_export(const SepCacheState& st, int32_t* pos_out, int32_t* count,
                                    cudaStream_t stream) {
-  sepcache_export_kernel<<<st.S, 256, 0, stream>>>(st.a, st.s, st.w, st.meta, st.slot_pos,
-                                                   pos_out, count);
+  sepcache_export_kernel<<<st.S, 256, 0, stream>>>(st.a, st.s, past_slots(st), st.w, st.meta,
+                                                   st.slot_pos, pos_out, count);
   return cudaGetLastError();
 }
 

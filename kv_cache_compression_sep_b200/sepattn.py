@@ -69,7 +69,7 @@ class _SepMask(ctypes.Structure):
 class _SepCacheState(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("a", ctypes.c_int32), ("s", ctypes.c_int32),
-                ("w", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("w", ctypes.c_int32), ("c", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
                 ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]
@@ -232,22 +232,26 @@ def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=Non
 class SepCache:
     """SepCache state for S sequences, held in torch-allocated device memory.
 
-    Capacities: a initial slots, s separator slots, w window slots (c = a + s + w).
+    Capacities: a initial slots, s separator slots, w window slots; c = 0 compresses one token
+    at a time, c > a + s + w adds a Past Window that is compressed when the usage reaches c.
+    Slots per sequence: n = a + s + w, plus c - a - w past-window slots when c > 0.
     Methods map one-to-one to sepcache_update / sepcache_decode / sepcache_export_order.
     """
 
-    def __init__(self, S, Hq, Hkv, d, a, s, w, rope_theta, device="cuda"):
+    def __init__(self, S, Hq, Hkv, d, a, s, w, rope_theta, device="cuda", c=0):
         self.S, self.Hq, self.Hkv, self.d, self.a, self.s, self.w = S, Hq, Hkv, d, a, s, w
-        self.c = a + s + w
+        self.c = int(c)
+        self.past = c - a - w if c > 0 else 0
+        self.n = a + s + self.past + w
         self.rope_theta = float(rope_theta)
         dev = torch.device(device)
-        self.k_slots = torch.zeros(S, Hkv, self.c, d, dtype=torch.bfloat16, device=dev)
-        self.v_slots = torch.zeros(S, Hkv, self.c, d, dtype=torch.bfloat16, device=dev)
-        self.slot_pos = torch.empty(S, self.c, dtype=torch.int32, device=dev)
-        self.slot_sep = torch.empty(S, self.c, dtype=torch.uint8, device=dev)
+        self.k_slots = torch.zeros(S, Hkv, self.n, d, dtype=torch.bfloat16, device=dev)
+        self.v_slots = torch.zeros(S, Hkv, self.n, d, dtype=torch.bfloat16, device=dev)
+        self.slot_pos = torch.empty(S, self.n, dtype=torch.int32, device=dev)
+        self.slot_sep = torch.empty(S, self.n, dtype=torch.uint8, device=dev)
         self.meta = torch.empty(S, META, dtype=torch.int32, device=dev)
-        self.rope_cs = torch.empty(self.c, d, dtype=torch.float32, device=dev)
-        self._st = _SepCacheState(S, Hq, Hkv, d, a, s, w, self.rope_theta,
+        self.rope_cs = torch.empty(self.n, d, dtype=torch.float32, device=dev)
+        self._st = _SepCacheState(S, Hq, Hkv, d, a, s, w, self.c, self.rope_theta,
                                   self.k_slots.data_ptr(), self.v_slots.data_ptr(),
                                   self.slot_pos.data_ptr(), self.slot_sep.data_ptr(),
                                   self.meta.data_ptr(), self.rope_cs.data_ptr())
@@ -295,7 +299,7 @@ class SepCache:
         return o
 
     def sepcache_export_order(self):
-        pos = torch.empty(self.S, self.c, dtype=torch.int32, device=self.k_slots.device)
+        pos = torch.empty(self.S, self.n, dtype=torch.int32, device=self.k_slots.device)
         cnt = torch.empty(self.S, dtype=torch.int32, device=self.k_slots.device)
         _check(_lib.sepcache_export_order(ctypes.byref(self._st), _ptr(pos), _ptr(cnt),
                                           _stream()), "sepcache_export_order")

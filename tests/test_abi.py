@@ -104,7 +104,7 @@ def test_workspace_sizes_grow_with_shape(lib):
 class _CacheState(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("a", ctypes.c_int32), ("s", ctypes.c_int32),
-                ("w", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("w", ctypes.c_int32), ("c", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
                 ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]
@@ -129,6 +129,10 @@ def test_cache_rejects_bad_state(lib):
     assert f(ctypes.byref(st(k_slots=258)), P(256), P(256), P(256), None) == SEP_ERR_MISALIGNED
     assert f(ctypes.byref(st(rope_theta=0.0)), P(256), P(256), P(256), None) == SEP_ERR_INVALID_ARG
     assert f(ctypes.byref(st()), P(258), P(256), P(256), None) == SEP_ERR_MISALIGNED
+    # Past Window threshold: 0 or above a + s + w
+    assert f(ctypes.byref(st(c=28)), P(256), P(256), P(256), None) == SEP_ERR_INVALID_ARG
+    assert f(ctypes.byref(st(c=-1)), P(256), P(256), P(256), None) == SEP_ERR_INVALID_ARG
+    assert f(ctypes.byref(st(c=20000, s=5000)), P(256), P(256), P(256), None) == SEP_ERR_UNSUPPORTED
 
 
 def test_prefill_rejects_bad_arguments(lib):

@@ -21,19 +21,25 @@ def S():
     return sepattn
 
 
-@pytest.mark.parametrize("Sq,Hq,Hkv,d,a,s,w,steps,p", [
-    (3, 8, 2, 128, 4, 6, 20, 120, 0.2),
-    (2, 4, 4, 64, 0, 3, 7, 60, 0.5),
-    (2, 8, 1, 128, 2, 0, 9, 50, 0.3),     # s = 0: StreamingLLM with shifting
-    (1, 16, 2, 64, 1, 2, 1, 30, 0.6),     # window of one slot
-    (2, 32, 8, 128, 4, 64, 300, 500, 0.1),
+@pytest.mark.parametrize("Sq,Hq,Hkv,d,a,s,w,steps,p,c", [
+    (3, 8, 2, 128, 4, 6, 20, 120, 0.2, 0),
+    (2, 4, 4, 64, 0, 3, 7, 60, 0.5, 0),
+    (2, 8, 1, 128, 2, 0, 9, 50, 0.3, 0),     # s = 0: StreamingLLM with shifting
+    (1, 16, 2, 64, 1, 2, 1, 30, 0.6, 0),     # window of one slot
+    (2, 32, 8, 128, 4, 64, 300, 500, 0.1, 0),
+    # Past Window Cache, compressed when the usage reaches c
+    (3, 8, 2, 128, 4, 6, 20, 200, 0.2, 45),
+    (2, 4, 4, 64, 0, 3, 7, 120, 0.5, 14),
+    (2, 8, 1, 128, 2, 0, 9, 80, 0.3, 20),    # s = 0: compression drops the past window
+    (1, 16, 2, 64, 1, 2, 1, 60, 0.6, 7),     # window of one slot
+    (2, 32, 8, 128, 4, 64, 256, 900, 0.1, 800),
 ])
-def test_small_every_step(S, Sq, Hq, Hkv, d, a, s, w, steps, p):
+def test_small_every_step(S, Sq, Hq, Hkv, d, a, s, w, steps, p, c):
     import torch
     theta = 500000.0
-    g = torch.Generator().manual_seed(Sq * 1000 + w)
-    cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, theta)
-    sims = [C.SepCacheSim(a, s, w) for _ in range(Sq)]
+    g = torch.Generator().manual_seed(Sq * 1000 + w + c)
+    cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, theta, c=c)
+    sims = [C.SepCacheSim(a, s, w, c if c > 0 else None) for _ in range(Sq)]
     K, V = [], []
     for t in range(steps):
         kn = torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16)

@@ -127,3 +127,44 @@ def decode_attention(q, k_ret, v_ret, theta, scale):
         o[h] = (e / l) @ v_ret[:, kh, :]
         lse[h] = mx + np.log(l)
     return o, lse
+
+
+# ---------------------------------------------------------------- decode without shifting
+# Training-free use of the separator mask at inference ([AS] "Key results": training-free
+# Llama-3-8B with the cache keeping initial, separator and neighbour tokens): no positional
+# shifting, so every retained key keeps its original position. Reading: such a cache stores
+# each key rotated once at its original position, in the storage type (bf16), as an ordinary
+# rotary KV cache does; only the query is rotated at decode time, at its own position t.
+def bf16_round(x):
+    """Round to the nearest bfloat16 (ties to even), returned as fp64."""
+    import torch
+    return torch.as_tensor(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).double().numpy()
+
+
+def stored_rotated_key(k, pos, theta):
+    """A key as the cache stores it without shifting: RoPE(k, pos) in fp64, rounded to bf16."""
+    return bf16_round(rope_rotate(k, pos, theta))
+
+
+def decode_attention_original_positions(q, k_stored, v_ret, t, theta, scale):
+    """Single-query attention over retained keys already rotated at their original positions
+    (k_stored [n_ret, Hkv, d]); the query q [Hq, d] is rotated at its own position t.
+    Returns o [Hq, d] and lse [Hq] (natural log), fp64."""
+    q = np.asarray(q, dtype=np.float64)
+    k_stored = np.asarray(k_stored, dtype=np.float64)
+    v_ret = np.asarray(v_ret, dtype=np.float64)
+    Hq, d = q.shape
+    Hkv = k_stored.shape[1]
+    G = Hq // Hkv
+    qr = rope_rotate(q, np.full((Hq,), t), theta)
+    o = np.zeros((Hq, d))
+    lse = np.zeros(Hq)
+    for h in range(Hq):
+        kh = h // G
+        s = scale * (k_stored[:, kh, :] @ qr[h])
+        mx = s.max()
+        e = np.exp(s - mx)
+        l = e.sum()
+        o[h] = (e / l) @ v_ret[:, kh, :]
+        lse[h] = mx + np.log(l)
+    return o, lse

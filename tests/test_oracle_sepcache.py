@@ -153,3 +153,50 @@ def test_past_window_invariants(a, s, w, c, p):
         # right after a compression the retained set is the one-token-at-a-time rule's
         if n_past == 0:
             assert order == ref.order(), t
+
+
+# ---------------------------------------------------------------- decode without shifting
+def test_original_positions_decode_is_the_mask_row():
+    """With every separator retained (s large) and w = n, decode at step t without shifting is
+    row t of the separator-sparse attention over RoPE'd queries and stored (rotated, bf16) keys."""
+    rng = np.random.default_rng(5)
+    a, n, L, Hq, Hkv, d, theta = 3, 6, 60, 4, 2, 8, 500000.0
+    sep = (rng.random(L) < 0.25).astype(np.uint8)
+    q = rng.standard_normal((L, Hq, d))
+    k = rng.standard_normal((L, Hkv, d))
+    v = rng.standard_normal((L, Hkv, d))
+    pos = np.arange(L)
+    k_st = C.stored_rotated_key(k, pos[:, None], theta)
+    q_rot = C.rope_rotate(q, pos[:, None], theta)
+    sim = C.SepCacheSim(a, L, n)
+    for t in range(L):
+        sim.append(bool(sep[t]))
+        order = sim.order()
+        o, lse = C.decode_attention_original_positions(q[t], k_st[order], v[order], t, theta,
+                                                       d ** -0.5)
+        ro, rl = R.attn_fwd_rows(q_rot[None], k_st[None], v[None], sep[None], a, n, d ** -0.5,
+                                 0, [t])
+        np.testing.assert_allclose(o, ro[0], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, rl[0], rtol=1e-12, atol=1e-12)
+
+
+def test_original_positions_before_eviction_is_causal_rope_attention():
+    rng = np.random.default_rng(6)
+    L, Hq, Hkv, d, theta = 20, 4, 4, 16, 10000.0
+    q = rng.standard_normal((Hq, d))
+    k = rng.standard_normal((L, Hkv, d))
+    v = rng.standard_normal((L, Hkv, d))
+    k_st = C.stored_rotated_key(k, np.arange(L)[:, None], theta)
+    o, lse = C.decode_attention_original_positions(q, k_st, v, L - 1, theta, d ** -0.5)
+    qr = C.rope_rotate(q, np.full((Hq,), L - 1), theta)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(qr)[:, None, :], torch.from_numpy(k_st).permute(1, 0, 2),
+        torch.from_numpy(v).permute(1, 0, 2), scale=d ** -0.5)
+    np.testing.assert_allclose(o, ref[:, 0].numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_bf16_round_ties_to_even():
+    # 1 + 2^-8 lies halfway between bf16 neighbours 1 and 1 + 2^-7: ties go to the even one (1)
+    assert C.bf16_round(1.0 + 2 ** -8) == 1.0
+    assert C.bf16_round(1.0 + 3 * 2 ** -8) == 1.0 + 2 ** -6
+    assert C.bf16_round(1.0 + 2 ** -8 + 2 ** -20) == 1.0 + 2 ** -7

@@ -599,6 +599,34 @@ def single_row(args, dev):
                     "mean_occupancy": sum(occ) / R / dc.S, "us_per_step": ms * 1e3,
                     "tokens_per_s": dc.S / (ms * 1e-3), "gbs_update_plus_decode": byts / (ms * 1e-3) / 1e9})
         return out
+    if args.workload == "decode-noshift":
+        # training-free use without positional shifting: initial a=4, every separator (s large)
+        # and the n=256 neighbours, keys at their original positions; 64 sequences seeded from
+        # 8192-token prompts, then steady decode steps
+        dc, Lp, n_win, s_all = workloads.SEPCACHE_DECODE, 8192, 256, 2048
+        cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, s_all, n_win, dc.theta, device=dev,
+                           original_positions=True)
+        g0 = torch.Generator(device=dev).manual_seed(dc.seed)
+        k = torch.randn(dc.S, Lp, dc.Hkv, dc.d, generator=g0, device=dev).to(torch.bfloat16)
+        v = torch.randn(dc.S, Lp, dc.Hkv, dc.d, generator=g0, device=dev).to(torch.bfloat16)
+        sep = (torch.rand(dc.S, Lp, generator=g0, device=dev) < dc.p).to(torch.uint8)
+        cache.sepcache_prefill(k, v, sep)
+        del k, v
+        pool = workloads.decode_chunk(dc, 0, 64, device=dev)
+        o = torch.empty_like(pool["q"][0])
+        x = {kk: vv[0].clone() for kk, vv in pool.items()}
+        x["sep"].zero_()  # steady state: the window slides, the separator set stays as prompted
+        g = capture(lambda: (cache.sepcache_update(x["k"], x["v"], x["sep"]),
+                             cache.sepcache_decode(x["q"], out=o)), reps=50)
+        ms = time_graph(g, args.steps, flush) / 50
+        m = cache.meta.cpu()
+        occ = int((m[:, 1] + m[:, 3] + m[:, 5]).sum())
+        T = int(m[:, 0].float().mean())
+        byts = occ * dc.Hkv * dc.d * 4 + dc.S * (4 * dc.Hq * dc.d + 4 * dc.Hkv * dc.d)
+        out.update({"a": dc.a, "n": n_win, "prompt_len": Lp, "mean_occupancy": occ / dc.S,
+                    "r_kv": occ / dc.S / T, "us_per_step": ms * 1e3,
+                    "tokens_per_s": dc.S / (ms * 1e-3), "gbs_update_plus_decode": byts / (ms * 1e-3) / 1e9})
+        return out
     if args.workload == "cache-prefill":
         # seed 64 caches (the decode configuration's capacities) from 8192-token prompts
         dc, Lp = workloads.SEPCACHE_DECODE, 8192
@@ -652,7 +680,8 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="train-decode",
                     choices=["train-decode", "pythia-train", "llama-prefill", "long-context",
-                             "long-context-dense", "decode", "decode-past", "cache-prefill"])
+                             "long-context-dense", "decode", "decode-past", "decode-noshift",
+                             "cache-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true",

@@ -182,6 +182,9 @@ typedef struct SepCacheState {
   int32_t S, Hq, Hkv, d;     /* sequences, query heads, KV heads, head dim (d = 128 or 64) */
   int32_t a, s, w;           /* initial / separator / window capacities */
   int32_t c;                 /* usage threshold of the Past Window (0: none; else > a + s + w) */
+  int32_t original_positions; /* 0: positional-encoding shifting, keys stored un-rotated and
+                                 rotated at their in-cache rank by every decode; 1: no
+                                 shifting, keys stored rotated at their original positions */
   float rope_theta;          /* RoPE base: angle of pair k at position p = p * theta^(-2k/d) */
   sep_bf16* k_slots;
   sep_bf16* v_slots;
@@ -225,7 +228,9 @@ int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16*
  * sepcache_decode - single-query attention of each sequence's newest token over its cache.
  * Logical order = [initial | separators oldest first | past window oldest first | window
  * oldest first]; the key of rank p is rotated by RoPE(p) and the query by RoPE(m),
- * m = occupied - 1 (its own rank).
+ * m = occupied - 1 (its own rank). With original_positions = 1 (training-free use without
+ * shifting) the keys were rotated at their original positions when they entered the cache,
+ * and the query is rotated at its own original position T - 1.
  * q [S, Hq, d] un-rotated; o [S, Hq, d] bf16; lse [S, Hq] fp32 natural log (nullable).
  * Call after sepcache_update of the same step.
  */

@@ -53,6 +53,36 @@ __global__ void sepcache_init_kernel(int S, int c, int d, double theta, int32_t*
   }
 }
 
+// Key rotation for a cache without positional shifting: the 16-byte chunks x (dims k0..k0+7)
+// and y (dims k0+d/2..k0+d/2+7) of one key row rotated at original position pos, the angle of
+// pair k being pos * theta^(-2k/d) as in the cos/sin table; fp64 arithmetic, rounded to bf16.
+__device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, int pos, int d,
+                                                   double theta) {
+  uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&xs[q]);
+    const __nv_bfloat162 ya = *reinterpret_cast<const __nv_bfloat162*>(&ys[q]);
+    double xv[2] = {(double)__low2float(xa), (double)__high2float(xa)};
+    double yv[2] = {(double)__low2float(ya), (double)__high2float(ya)};
+    __nv_bfloat16 xo[2], yo[2];
+#pragma unroll
+    for (int z = 0; z < 2; ++z) {
+      const int k = k0 + 2 * q + z;
+      double sn, cs;
+      sincos((double)pos * pow(theta, -2.0 * (double)k / (double)d), &sn, &cs);
+      xo[z] = __double2bfloat16(xv[z] * cs - yv[z] * sn);
+      yo[z] = __double2bfloat16(yv[z] * cs + xv[z] * sn);
+    }
+    const __nv_bfloat162 xp = __halves2bfloat162(xo[0], xo[1]);
+    const __nv_bfloat162 yp = __halves2bfloat162(yo[0], yo[1]);
+    xs[q] = *reinterpret_cast<const uint32_t*>(&xp);
+    ys[q] = *reinterpret_cast<const uint32_t*>(&yp);
+  }
+  x = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+  y = make_uint4(ys[0], ys[1], ys[2], ys[3]);
+}
+
 // ------------------------------------------------------------------ update
 // One CTA per sequence. Thread 0 plans the step, all threads copy rows (16-byte vectors). With a
 // Past Window (P > 0) the step that makes the usage reach c then compresses it: a block-wide
@@ -62,7 +92,8 @@ __global__ void sepcache_init_kernel(int S, int c, int d, double theta, int32_t*
 constexpr int kUpdateThreads = 128;
 
 __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
-    int Hkv, int d, int a, int s, int w, int P, int c, uint4* __restrict__ k_slots,
+    int Hkv, int d, int a, int s, int w, int P, int c, int orig, double theta,
+    uint4* __restrict__ k_slots,
     uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
     int32_t* __restrict__ meta, const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
     const uint8_t* __restrict__ sep_new) {
@@ -146,12 +177,19 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
     }
     __syncthreads();
   }
-  for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
-    const int hh = e / vec, q = e % vec;
+  const int hv = vec / 2;  // chunks per RoPE half
+  for (int e = tid; e < Hkv * hv; e += kUpdateThreads) {  // K: chunk q and its partner q + hv
+    const int hh = e / hv, q = e % hv;
     const size_t dst = (seq_rows + (size_t)hh * ns + slot_new) * vec + q;
     const size_t src = ((size_t)seq * Hkv + hh) * vec + q;
-    k_slots[dst] = k_new[src];
-    v_slots[dst] = v_new[src];
+    uint4 x = k_new[src], y = k_new[src + hv];
+    if (orig) rope_rotate_chunks(x, y, 8 * q, t, d, theta);
+    k_slots[dst] = x;
+    k_slots[dst + hv] = y;
+  }
+  for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
+    const int hh = e / vec, q = e % vec;
+    v_slots[(seq_rows + (size_t)hh * ns + slot_new) * vec + q] = v_new[((size_t)seq * Hkv + hh) * vec + q];
   }
   if (tid == 0) {
     slot_pos[(size_t)seq * ns + slot_new] = t;
@@ -232,7 +270,8 @@ constexpr int kPrefillThreads = 256;
 constexpr int kPrefillItems = 16;
 
 __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
-    int L, int Hkv, int d, int a, int s, int w, const uint4* __restrict__ k_in,
+    int L, int Hkv, int d, int a, int s, int w, int orig, double theta,
+    const uint4* __restrict__ k_in,
     const uint4* __restrict__ v_in, const uint8_t* __restrict__ sep_in, uint4* __restrict__ k_slots,
     uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
     int32_t* __restrict__ meta) {
@@ -341,10 +380,13 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
     if (pos < 0) continue;
     const size_t src = (((size_t)seq * L + pos) * Hkv + head) * vec;
     const size_t dst = (dst_base + slot) * vec;
-    for (int e = lane; e < vec; e += 32) {
-      k_slots[dst + e] = __ldg(k_in + src + e);
-      v_slots[dst + e] = __ldg(v_in + src + e);
+    for (int e = lane; e < vec / 2; e += 32) {  // K: chunk e and its RoPE partner
+      uint4 x = __ldg(k_in + src + e), y = __ldg(k_in + src + e + vec / 2);
+      if (orig) rope_rotate_chunks(x, y, 8 * e, pos, d, theta);
+      k_slots[dst + e] = x;
+      k_slots[dst + e + vec / 2] = y;
     }
+    for (int e = lane; e < vec; e += 32) v_slots[dst + e] = __ldg(v_in + src + e);
   }
 }
 
@@ -357,7 +399,8 @@ cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, cons
     if (e != cudaSuccess) return e;
   }
   sepcache_prefill_kernel<<<dim3(st.S, st.Hkv), kPrefillThreads, smem, stream>>>(
-      L, st.Hkv, st.d, st.a, st.s, st.w, static_cast<const uint4*>(k),
+      L, st.Hkv, st.d, st.a, st.s, st.w, st.original_positions, (double)st.rope_theta,
+      static_cast<const uint4*>(k),
       static_cast<const uint4*>(v), sep, reinterpret_cast<uint4*>(st.k_slots),
       reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta);
   return cudaGetLastError();
@@ -429,14 +472,17 @@ struct DecSmem {
   int abort_flag;
 };
 
-template <int D, int G>
+// ORIG: keys were stored rotated at their original positions (no positional shifting): no
+// rotation of keys here, and the query is rotated at its own original position T - 1.
+template <int D, int G, bool ORIG>
 __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
     sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int P, int w,
                            const __nv_bfloat16* __restrict__ k_slots,
                            const __nv_bfloat16* __restrict__ v_slots,
                            const int32_t* __restrict__ meta, const float2* __restrict__ rope_cs,
                            const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ o,
-                           float* __restrict__ lse, float scale_log2, unsigned* err) {
+                           float* __restrict__ lse, float scale_log2, double theta,
+                           unsigned* err) {
   constexpr int HP = D / 32;       // rotation pairs per lane
   constexpr int HALF = D / 2;
   const int kvh = blockIdx.x, seq = blockIdx.y;
@@ -512,10 +558,23 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
 
   {
     // ---------------------------------------------------------------- consumers
-    // query heads of this KV head, rotated by RoPE(mq) and scaled by scale*log2(e)
+    // query heads of this KV head, rotated by RoPE(mq) (by RoPE(T - 1) without shifting) and
+    // scaled by scale*log2(e)
     float qr[G][2 * HP];
     {
-      const float2* cs = rope_cs + (size_t)max(mq, 0) * HALF;
+      float2 qcs[HP];
+#pragma unroll
+      for (int e = 0; e < HP; ++e) {
+        const int k = lane16 * HP + e;
+        if constexpr (ORIG) {
+          double sn, cs;
+          sincos((double)(m[SEPCACHE_META_T] - 1) * pow(theta, -2.0 * (double)k / (double)D), &sn,
+                 &cs);
+          qcs[e] = make_float2((float)cs, (float)sn);
+        } else {
+          qcs[e] = rope_cs[(size_t)max(mq, 0) * HALF + k];
+        }
+      }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const __nv_bfloat16* qh = q + ((size_t)seq * Hq + kvh * G + g) * D;
@@ -523,7 +582,7 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
         for (int e = 0; e < HP; ++e) {
           const int k = lane16 * HP + e;
           const float x1 = __bfloat162float(qh[k]), x2 = __bfloat162float(qh[k + HALF]);
-          const float2 rr = cs[k];
+          const float2 rr = qcs[e];
           qr[g][e] = (x1 * rr.x - x2 * rr.y) * scale_log2;
           qr[g][HP + e] = (x2 * rr.x + x1 * rr.y) * scale_log2;
         }
@@ -573,17 +632,19 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
         for (int g = 0; g < G; ++g) part[g] = 0.f;
 #pragma unroll
         for (int e = 0; e < HP; ++e) {
-          const float y1 = k1[e] * cr[e] - k2[e] * sr[e];
-          const float y2 = k2[e] * cr[e] + k1[e] * sr[e];
+          const float y1 = ORIG ? k1[e] : k1[e] * cr[e] - k2[e] * sr[e];
+          const float y2 = ORIG ? k2[e] : k2[e] * cr[e] + k1[e] * sr[e];
 #pragma unroll
           for (int g = 0; g < G; ++g) part[g] = fmaf(qr[g][e], y1, fmaf(qr[g][HP + e], y2, part[g]));
         }
+        if constexpr (!ORIG) {
 #pragma unroll
-        for (int e = 0; e < HP; ++e) {
-          const float cn = cr[e] * cd[e] - sr[e] * sd[e];
-          const float sn = sr[e] * cd[e] + cr[e] * sd[e];
-          cr[e] = cn;
-          sr[e] = sn;
+          for (int e = 0; e < HP; ++e) {
+            const float cn = cr[e] * cd[e] - sr[e] * sd[e];
+            const float sn = sr[e] * cd[e] + cr[e] * sd[e];
+            cr[e] = cn;
+            sr[e] = sn;
+          }
         }
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -734,13 +795,14 @@ cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new, c
   const int P = past_slots(st);
   const size_t smem = (size_t)max(1, min(st.s, P)) * sizeof(int2);  // compression moves
   sepcache_update_kernel<<<st.S, kUpdateThreads, smem, stream>>>(
-      st.Hkv, st.d, st.a, st.s, st.w, P, st.c, reinterpret_cast<uint4*>(st.k_slots),
+      st.Hkv, st.d, st.a, st.s, st.w, P, st.c, st.original_positions, (double)st.rope_theta,
+      reinterpret_cast<uint4*>(st.k_slots),
       reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta,
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), sep_new);
   return cudaGetLastError();
 }
 
-template <int D, int G>
+template <int D, int G, bool ORIG>
 static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void* o, float* lse,
                                    float scale, cudaStream_t stream) {
   constexpr size_t smem = sizeof(DecSmem<D>);
@@ -749,18 +811,19 @@ static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void*
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(sepcache_decode_kernel<D, G>,
+    e = cudaFuncSetAttribute(sepcache_decode_kernel<D, G, ORIG>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   dim3 grid(st.Hkv, st.S);
-  sepcache_decode_kernel<D, G><<<grid, kDecThreads, smem, stream>>>(
+  sepcache_decode_kernel<D, G, ORIG><<<grid, kDecThreads, smem, stream>>>(
       st.Hq, st.Hkv, st.a, st.s, past_slots(st), st.w,
       reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
       reinterpret_cast<const __nv_bfloat16*>(st.v_slots), st.meta,
       reinterpret_cast<const float2*>(st.rope_cs), static_cast<const __nv_bfloat16*>(q),
-      static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f, device_error_word());
+      static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f, (double)st.rope_theta,
+      device_error_word());
   return cudaGetLastError();
 }
 
@@ -768,7 +831,9 @@ cudaError_t launch_sepcache_decode(const SepCacheState& st, const void* q, void*
                                    float scale, cudaStream_t stream) {
   const int G = st.Hq / st.Hkv;
 #define SEP_DEC_CASE(DD, GG) \
-  if (st.d == DD && G == GG) return launch_decode_t<DD, GG>(st, q, o, lse, scale, stream);
+  if (st.d == DD && G == GG)                                                             \
+    return st.original_positions ? launch_decode_t<DD, GG, true>(st, q, o, lse, scale, stream) \
+                                 : launch_decode_t<DD, GG, false>(st, q, o, lse, scale, stream);
   SEP_DEC_CASE(128, 1)
   SEP_DEC_CASE(128, 2)
   SEP_DEC_CASE(128, 4)

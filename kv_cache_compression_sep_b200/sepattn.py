@@ -69,7 +69,8 @@ class _SepMask(ctypes.Structure):
 class _SepCacheState(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("a", ctypes.c_int32), ("s", ctypes.c_int32),
-                ("w", ctypes.c_int32), ("c", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("w", ctypes.c_int32), ("c", ctypes.c_int32),
+                ("original_positions", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
                 ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]
@@ -235,10 +236,13 @@ class SepCache:
     Capacities: a initial slots, s separator slots, w window slots; c = 0 compresses one token
     at a time, c > a + s + w adds a Past Window that is compressed when the usage reaches c.
     Slots per sequence: n = a + s + w, plus c - a - w past-window slots when c > 0.
+    original_positions=True: no positional shifting (keys stored rotated at their original
+    positions, the query rotated at its own position).
     Methods map one-to-one to sepcache_update / sepcache_decode / sepcache_export_order.
     """
 
-    def __init__(self, S, Hq, Hkv, d, a, s, w, rope_theta, device="cuda", c=0):
+    def __init__(self, S, Hq, Hkv, d, a, s, w, rope_theta, device="cuda", c=0,
+                 original_positions=False):
         self.S, self.Hq, self.Hkv, self.d, self.a, self.s, self.w = S, Hq, Hkv, d, a, s, w
         self.c = int(c)
         self.past = c - a - w if c > 0 else 0
@@ -251,7 +255,9 @@ class SepCache:
         self.slot_sep = torch.empty(S, self.n, dtype=torch.uint8, device=dev)
         self.meta = torch.empty(S, META, dtype=torch.int32, device=dev)
         self.rope_cs = torch.empty(self.n, d, dtype=torch.float32, device=dev)
-        self._st = _SepCacheState(S, Hq, Hkv, d, a, s, w, self.c, self.rope_theta,
+        self.original_positions = bool(original_positions)
+        self._st = _SepCacheState(S, Hq, Hkv, d, a, s, w, self.c, int(self.original_positions),
+                                  self.rope_theta,
                                   self.k_slots.data_ptr(), self.v_slots.data_ptr(),
                                   self.slot_pos.data_ptr(), self.slot_sep.data_ptr(),
                                   self.meta.data_ptr(), self.rope_cs.data_ptr())

@@ -104,7 +104,8 @@ def test_workspace_sizes_grow_with_shape(lib):
 class _CacheState(ctypes.Structure):
     _fields_ = [("S", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("a", ctypes.c_int32), ("s", ctypes.c_int32),
-                ("w", ctypes.c_int32), ("c", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+                ("w", ctypes.c_int32), ("c", ctypes.c_int32),
+                ("original_positions", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
                 ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]

@@ -218,3 +218,63 @@ def test_prefill_equals_sequential_updates(S, Sq, Hq, Hkv, d, a, s, w, L, p):
         cache.sepcache_update(kn, kn, sn)
         outs.append(cache.sepcache_decode(q))
     assert torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("Sq,Hq,Hkv,d,a,s,w,steps,p", [
+    (2, 8, 2, 128, 4, 300, 32, 300, 0.2),    # every separator retained, w = n
+    (3, 4, 4, 64, 1, 4, 9, 150, 0.4),        # separator FIFO overflows
+    (2, 32, 8, 128, 4, 64, 200, 400, 0.1),
+])
+def test_original_positions_every_step(S, Sq, Hq, Hkv, d, a, s, w, steps, p):
+    """Without positional shifting: trajectory bit-exact and decode within the forward
+    tolerances of the oracle (keys stored rotated at original positions in bf16)."""
+    import torch
+    theta = 500000.0
+    g = torch.Generator().manual_seed(steps + s)
+    cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, theta, original_positions=True)
+    sims = [C.SepCacheSim(a, s, w) for _ in range(Sq)]
+    Kst, V = [], []
+    for t in range(steps):
+        kn = torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16)
+        vn = torch.randn(Sq, Hkv, d, generator=g).to(torch.bfloat16)
+        qn = torch.randn(Sq, Hq, d, generator=g).to(torch.bfloat16)
+        sn = (torch.rand(Sq, generator=g) < p).to(torch.uint8)
+        Kst.append(C.stored_rotated_key(f64(kn), t, theta))
+        V.append(f64(vn))
+        cache.sepcache_update(kn.cuda(), vn.cuda(), sn.cuda())
+        lse = torch.empty(Sq, Hq, dtype=torch.float32, device="cuda")
+        o = cache.sepcache_decode(qn.cuda(), lse=lse)
+        if t % 7 and t < steps - 1:
+            for sq in range(Sq):
+                sims[sq].append(bool(sn[sq]))
+            continue
+        pos, cnt = cache.sepcache_export_order()
+        pos, cnt = pos.cpu().numpy(), cnt.cpu().numpy()
+        for sq in range(Sq):
+            sims[sq].append(bool(sn[sq]))
+            order = sims[sq].order()
+            assert pos[sq, : int(cnt[sq])].tolist() == order, (t, sq)
+            kr = np.stack([Kst[j][sq] for j in order])
+            vr = np.stack([V[j][sq] for j in order])
+            ro, rl = C.decode_attention_original_positions(f64(qn[sq]), kr, vr, t, theta, d ** -0.5)
+            check_out(f64(o[sq]), ro, f"step {t} seq {sq}")
+            assert np.abs(f64(lse[sq]) - rl).max() < 2e-3
+    assert S.sep_last_device_error() == 0
+
+
+def test_original_positions_prefill_equals_updates(S):
+    import torch
+    Sq, Hq, Hkv, d, a, s, w, L = 2, 8, 2, 128, 4, 64, 40, 500
+    g = torch.Generator().manual_seed(9)
+    k = torch.randn(Sq, L, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(Sq, L, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    sep = (torch.rand(Sq, L, generator=g) < 0.15).to(torch.uint8).cuda()
+    seq_cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, 500000.0, original_positions=True)
+    for t in range(L):
+        seq_cache.sepcache_update(k[:, t].contiguous(), v[:, t].contiguous(), sep[:, t].contiguous())
+    pre_cache = S.SepCache(Sq, Hq, Hkv, d, a, s, w, 500000.0, original_positions=True)
+    pre_cache.sepcache_prefill(k, v, sep)
+    torch.cuda.synchronize()
+    assert S.sep_last_device_error() == 0
+    for name in ("meta", "slot_pos", "slot_sep", "k_slots", "v_slots"):
+        assert torch.equal(getattr(seq_cache, name), getattr(pre_cache, name)), name

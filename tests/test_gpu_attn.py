@@ -105,6 +105,33 @@ def test_fixed_interval_anchors(S):
     check_grad(f64(dv), dvr)
 
 
+def test_varlen_right_padded(S):
+    """Variable lengths through right padding: rows below each sequence's length equal the
+    unpadded sequence's attention (causal: real rows never read padded keys), and with dO zero
+    on padded rows the gradients of the real rows and keys equal the unpadded ones."""
+    import torch
+    lens, L, Hq, Hkv, d, a, n = (300, 517), 517, 4, 2, 64, 4, 64
+    inp = _inputs(77, len(lens), L, Hq, Hkv, d, 0.15)
+    for b, lb in enumerate(lens):
+        inp["do"][b, lb:] = 0
+    dev = _to_dev(inp)
+    mask, o, lse = _fwd(S, dev, a, n)
+    dq, dk, dv = S.sep_attn_bwd(dev["q"], dev["k"], dev["v"], o, lse, dev["do"], mask)
+    torch.cuda.synchronize()
+    assert S.sep_last_device_error() == 0
+    for b, lb in enumerate(lens):
+        sl = lambda t: f64(t[b:b + 1, :lb])  # noqa: E731
+        sep = inp["sep"][b:b + 1, :lb].numpy()
+        Or, LSEr = R.attn_fwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sep, a, n, d ** -0.5)
+        check_out(f64(o[b:b + 1, :lb]), Or, f"O seq {b}")
+        check_lse(f64(lse[b:b + 1, :, :lb]), LSEr, f"LSE seq {b}")
+        dqr, dkr, dvr = R.attn_bwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["do"]), sep, a,
+                                   n, d ** -0.5)
+        check_grad(f64(dq[b:b + 1, :lb]), dqr, f"dQ seq {b}")
+        check_grad(f64(dk[b:b + 1, :lb]), dkr, f"dK seq {b}")
+        check_grad(f64(dv[b:b + 1, :lb]), dvr, f"dV seq {b}")
+
+
 def _cfg_inputs(name):
     import workloads
     cfg = workloads.ATTN_CONFIGS[name]

@@ -459,6 +459,53 @@ __device__ __forceinline__ void load_bf16_vec_smem(const __nv_bfloat16* p, float
 // first stages; afterwards the last warp to finish reading a stage refills it with the chunk
 // kStages further on, so no thread waits to issue. Half-warp hw handles ranks r0 + hw + 16k;
 // lane16 owns HP rotation pairs (k, k + d/2), k = lane16 * HP + e, of every row it reads.
+// Half-warp reduction of the G per-query partial dot products of one key row: the first
+// log2(G) butterfly levels halve what a lane holds (it keeps one half, adding its partner's copy
+// of it, and sends the other half), the remaining levels sum a single value. Afterwards lane
+// l16 holds the full score of query own_query<G>(l16): 2G + 3 - log2(G) shuffles and adds
+// instead of 4G for one reduction per query.
+template <int G>
+__host__ __device__ constexpr int log2_of() {
+  return G >= 16 ? 4 : G >= 8 ? 3 : G >= 4 ? 2 : G >= 2 ? 1 : 0;
+}
+template <int G>
+__device__ __forceinline__ float halfwarp_reduce_own(float (&v)[G], int lane16) {
+  constexpr int LG = log2_of<G>();
+  static_assert((1 << LG) == G && G <= 16, "G must be a power of two <= 16");
+#pragma unroll
+  for (int l = 0; l < LG; ++l) {
+    const int off = 8 >> l, h = (G >> l) >> 1;
+    const bool upper = (lane16 & off) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h];
+      const float keep = upper ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int l = LG; l < 4; ++l) r += __shfl_xor_sync(0xffffffffu, r, 8 >> l);
+  return r;
+}
+// The query whose score lane l16 holds after halfwarp_reduce_own, and a lane holding query g.
+template <int G>
+__device__ __forceinline__ int own_query(int lane16) {
+  int g = 0;
+#pragma unroll
+  for (int l = 0; l < log2_of<G>(); ++l)
+    if (lane16 & (8 >> l)) g += G >> (l + 1);
+  return g;
+}
+template <int G>
+__device__ __forceinline__ int lane_of_query(int g) {
+  int src = 0;
+#pragma unroll
+  for (int l = 0; l < log2_of<G>(); ++l)
+    if (g & (G >> (l + 1))) src |= 8 >> l;
+  return src;
+}
+
 constexpr int kChunk = 16;
 constexpr int kStages = 4;
 constexpr int kConsumerWarps = kDecThreads / 32;
@@ -547,11 +594,10 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
   __syncthreads();
 
   // per-head softmax state (consumers)
-  float mrun[G], lrun[G], acc[G][2 * HP];
+  // softmax state of this lane's own query (see halfwarp_reduce_own); V sums of every query
+  float m_own = -INFINITY, l_own = 0.f, acc[G][2 * HP];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    mrun[g] = -INFINITY;
-    lrun[g] = 0.f;
 #pragma unroll
     for (int e = 0; e < 2 * HP; ++e) acc[g][e] = 0.f;
   }
@@ -646,29 +692,32 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
             sr[e] = sn;
           }
         }
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-          for (int off = 8; off > 0; off >>= 1) part[g] += __shfl_xor_sync(0xffffffffu, part[g], off);
-        }
-        if (valid) {
+        // this lane's query score; the online softmax of that query only, its probability
+        // then broadcast to the lanes of the half-warp for the V accumulation of every query
+        const float sc = halfwarp_reduce_own<G>(part, lane16);
+        const bool need = valid && sc > m_own + 8.0f;  // lazy rescale (max grew by > 2^8)
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2(m_own - sc) : 1.0f;
+          if (need) {
+            l_own *= alpha;
+            m_own = sc;
+          }
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float sc = part[g];
-            if (sc > mrun[g] + 8.0f) {
-              const float alpha = ex2(mrun[g] - sc);
-              lrun[g] *= alpha;
+            const float ag = __shfl_sync(0xffffffffu, alpha, lane_of_query<G>(g), 16);
 #pragma unroll
-              for (int e = 0; e < 2 * HP; ++e) acc[g][e] *= alpha;
-              mrun[g] = sc;
-            }
-            const float pg = ex2(sc - mrun[g]);
-            lrun[g] += pg;
+            for (int e = 0; e < 2 * HP; ++e) acc[g][e] *= ag;
+          }
+        }
+        const float p_own = valid ? ex2(sc - m_own) : 0.f;
+        l_own += p_own;
 #pragma unroll
-            for (int e = 0; e < HP; ++e) {
-              acc[g][e] = fmaf(pg, v1[e], acc[g][e]);
-              acc[g][HP + e] = fmaf(pg, v2[e], acc[g][HP + e]);
-            }
+        for (int g = 0; g < G; ++g) {
+          const float pg = __shfl_sync(0xffffffffu, p_own, lane_of_query<G>(g), 16);
+#pragma unroll
+          for (int e = 0; e < HP; ++e) {
+            acc[g][e] = fmaf(pg, v1[e], acc[g][e]);
+            acc[g][HP + e] = fmaf(pg, v2[e], acc[g][HP + e]);
           }
         }
       }
@@ -692,6 +741,13 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
     }
   }
 
+  // every query's softmax state from the lanes that own it
+  float mrun[G], lrun[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    mrun[g] = __shfl_sync(0xffffffffu, m_own, lane_of_query<G>(g), 16);
+    lrun[g] = __shfl_sync(0xffffffffu, l_own, lane_of_query<G>(g), 16);
+  }
   // ---- combine the two half-warps of each warp (lanes l and l^16 hold the same columns)
 #pragma unroll
   for (int g = 0; g < G; ++g) {

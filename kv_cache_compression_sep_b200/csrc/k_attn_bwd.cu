@@ -614,7 +614,7 @@ struct DkvCfg {
   static constexpr int SMEM_TILES = TILE * (2 * KVB + 2 * NST);
   static constexpr int COL_S0 = 0;     // half h: S^T at 128h, dP^T at 128h + 64
   static constexpr int COL_DV = 256, COL_DK = 256 + D;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, storer
 };
 
 template <int NST, int KVB>
@@ -623,6 +623,7 @@ struct DkvBar {
   uint64_t q_full[NST], q_empty[NST];
   uint64_t s_full[2], pds_ready[2], mm_done[2];
   uint64_t acc_full, acc_free;
+  uint64_t staged[KVB];   // the item's dK/dV rows are in the K/V buffer (softmax -> storer)
   uint64_t drain;
   uint64_t item_full[4];  // ring of fetched work-item indices (producer -> MMA, softmax)
   int item_x[4];
@@ -696,6 +697,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     }
     mbar_init(&bar->acc_full, 1);
     mbar_init(&bar->acc_free, 256);
+    for (int s = 0; s < KVB; ++s) mbar_init(&bar->staged[s], 256);
     mbar_init(&bar->drain, 1);
     for (int s = 0; s < 4; ++s) mbar_init(&bar->item_full[s], 1);
     bar->abort_flag = 0;
@@ -877,7 +879,31 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }
-  } else {
+  } else if (warp == 10) {
+    // ---------------------------------------------------------------- dK/dV storer
+    // Per item, once the softmax warps have staged it: the bf16 rows of a direct-mode window
+    // item leave by TMA store from the item's K/V buffer; then the buffer is released.
+    if (lane == 0) {
+      for (int I = 0;; ++I) {
+        if (!mbar_wait(&bar->item_full[I & 3], (I >> 2) & 1, p.err, abort_flag)) break;
+        const int x = bar->item_x[I & 3];
+        if (x >= nitems) break;
+        const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+        const int kb = I % KVB;
+        if (!mbar_wait(&bar->staged[kb], (I / KVB) & 1, p.err, abort_flag)) break;
+        if (direct && it.window) {
+          for (int z = 0; z < C::KB; ++z) {
+            tma_store_4d(&p.tmdV, sV + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
+            tma_store_4d(&p.tmdK, sK + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
+          }
+          bulk_commit_group();
+          bulk_wait_read_all();  // the buffer may now take a later item's K / V
+        }
+        mbar_arrive(&bar->kv_empty[kb]);
+      }
+      bulk_wait_all();  // dK / dV stores complete before the CTA exits
+    }
+  } else if (warp < 8) {
     // ---------------------------------------------------------------- softmax warpgroups
     const int h = threadIdx.x >> 7;      // query half owned by this warpgroup
     const int krow = threadIdx.x & 127;  // key row = TMEM lane
@@ -1061,20 +1087,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       tc_fence_before();
       mbar_arrive(&bar->acc_free);  // the next item may overwrite dV / dK
       if (stage_row) fence_proxy_async_smem();
-      asm volatile("bar.sync 5, 256;" ::: "memory");
-      if (threadIdx.x == 0) {
-        if (direct && it.window) {
-          for (int z = 0; z < C::KB; ++z) {
-            tma_store_4d(&p.tmdV, sV + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
-            tma_store_4d(&p.tmdK, sK + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
-          }
-          bulk_commit_group();
-          bulk_wait_read_all();
-        }
-        mbar_arrive(&bar->kv_empty[kb]);
-      }
+      mbar_arrive(&bar->staged[kb]);  // the storer writes the rows out and frees the buffer
     }
-    if (threadIdx.x == 0) bulk_wait_all();
     tc_fence_before();
   }
   __syncthreads();

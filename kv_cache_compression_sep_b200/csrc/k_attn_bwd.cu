@@ -56,12 +56,28 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
   const int nch = Hq * CPH;
   const uint4* po = o + row * nch;
   const uint4* pd = dout + row * nch;
-  for (int c0 = 0; c0 < nch; c0 += 32) {
-    const int c = c0 + lane;
-    float acc = 0.f;
-    if (c < nch) {
-      const uint4 x = __ldg(po + c), y = __ldg(pd + c);
-      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+  // groups of up to kRounds 32-chunk rounds: every load of a group is issued before any of
+  // its reductions, so a warp keeps several 16-byte loads of O and dO in flight
+  constexpr int kRounds = 4;
+  for (int g0 = 0; g0 < nch; g0 += 32 * kRounds) {
+    uint4 xv[kRounds], yv[kRounds];
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+      const int c = g0 + 32 * r + lane;
+      if (c < nch) {
+        xv[r] = __ldg(po + c);
+        yv[r] = __ldg(pd + c);
+      } else {
+        xv[r] = yv[r] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRounds; ++r) {
+      const int c = g0 + 32 * r + lane;
+      if (g0 + 32 * r >= nch) break;  // warp-uniform
+      const uint32_t xs[4] = {xv[r].x, xv[r].y, xv[r].z, xv[r].w};
+      const uint32_t ys[4] = {yv[r].x, yv[r].y, yv[r].z, yv[r].w};
+      float acc = 0.f;
 #pragma unroll
       for (int z = 0; z < 4; ++z) {
         const __nv_bfloat162 a2 = *reinterpret_cast<const __nv_bfloat162*>(&xs[z]);
@@ -69,10 +85,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
         acc = fmaf(__low2float(a2), __low2float(b2), acc);
         acc = fmaf(__high2float(a2), __high2float(b2), acc);
       }
-    }
 #pragma unroll
-    for (int off = CPH / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (c < nch && (lane % CPH) == 0) delta[((size_t)b * Hq + c / CPH) * L + i] = acc;
+      for (int off = CPH / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (c < nch && (lane % CPH) == 0) delta[((size_t)b * Hq + c / CPH) * L + i] = acc;
+    }
   }
   const int cnt = __ldg(anchor_cnt + b);
   if (i < min(L, (cnt + 127) / 128 * 128))

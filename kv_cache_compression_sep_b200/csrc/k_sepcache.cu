@@ -106,13 +106,22 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
   // slot_new, move_from, move_to, t, compress, past_cnt, sep_head, sep_cnt
   __shared__ int plan[8];
   __shared__ int s_warp[kUpdateThreads / 32];
+  // the metadata and the flag of the window's oldest slot, loaded in parallel
+  __shared__ int s_meta[SEPCACHE_META];
+  __shared__ int s_oldsep;
+  if (tid < SEPCACHE_META) s_meta[tid] = m[tid];
+  if (tid == 32) {
+    const int wh = m[SEPCACHE_META_WIN_HEAD];
+    s_oldsep = slot_sep[(size_t)seq * ns + win_base + wh];
+  }
+  __syncthreads();
   if (tid == 0) {
-    const int t = m[SEPCACHE_META_T];
+    const int t = s_meta[SEPCACHE_META_T];
     int slot_new, move_from = -1, move_to = -1;
-    int ninit = m[SEPCACHE_META_NINIT];
-    int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
-    int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
-    int past_cnt = (P > 0) ? m[SEPCACHE_META_PAST_CNT] : 0;
+    int ninit = s_meta[SEPCACHE_META_NINIT];
+    int sep_head = s_meta[SEPCACHE_META_SEP_HEAD], sep_cnt = s_meta[SEPCACHE_META_SEP_CNT];
+    int win_head = s_meta[SEPCACHE_META_WIN_HEAD], win_cnt = s_meta[SEPCACHE_META_WIN_CNT];
+    int past_cnt = (P > 0) ? s_meta[SEPCACHE_META_PAST_CNT] : 0;
     if (t < a) {
       slot_new = t;
       ninit = t + 1;
@@ -126,7 +135,7 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
         move_from = old_slot;
         move_to = a + s + past_cnt;
         ++past_cnt;
-      } else if (slot_sep[(size_t)seq * ns + old_slot] && s > 0) {
+      } else if (s_oldsep && s > 0) {  // the flag of old_slot = win_base + win_head
         if (sep_cnt < s) {
           move_to = a + (sep_head + sep_cnt) % s;
           ++sep_cnt;

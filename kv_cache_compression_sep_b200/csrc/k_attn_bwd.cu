@@ -9,17 +9,18 @@
 // dK, dV summed over the query heads of a KV head.
 //
 // Kernels, in stream order:
-//   1. prep: compacted anchor K/V rows (shared with the forward), zeroed fp32 anchor partials,
-//      Delta = rowsum(dO * O).
-//   2. dQ (query-major, one CTA per (query tile, query head, batch); same key tiles as the
-//      forward): S = Q K^T and dP = dO V^T into TMEM, dS = P (dP - Delta) written back to TMEM
-//      as bf16, dQ += dS K (A from TMEM, B = K MN-major).
-//   3. dK/dV (key-major): one CTA per window key tile u (query tiles t with lo(t) <= u <= t) or
-//      per (anchor chunk c, segment of query tiles that gather it). Per (query tile, query head):
+//   1. prep (one warp per position): compacted anchor K/V rows (as the forward), zeroed fp32
+//      anchor partials, Delta = rowsum(dO * O); then the dK/dV work list (bwd_schedule_kernel).
+//   2. dQ (query-major, persistent over the forward's item order and key tiles): S = Q K^T and
+//      dP = dO V^T into TMEM, dS = P (dP - Delta) written back to TMEM as bf16,
+//      dQ += dS K (A from TMEM, B = K MN-major); a storer warp writes the dQ tile.
+//   3. dK/dV (key-major, persistent, items fetched dynamically): work items are window key
+//      tiles u (query tiles t with lo(t) <= u <= t) and (anchor chunk c, segment of query tiles
+//      that gather it). Per (query tile, query head), in two 64-row query halves:
 //      S^T = K Q^T, dP^T = V dO^T into TMEM; P^T and dS^T back to TMEM as bf16;
 //      dV += P^T dO, dK += dS^T Q. Non-anchor keys of a window tile get their complete gradient
-//      and are written as bf16; anchor keys are summed in fp32 (window part + every gathered
-//      part) in a compact [B, anchors, Hkv, d] buffer.
+//      and leave as bf16 through a storer warp's TMA store; anchor keys are summed in fp32
+//      (window part + every gathered part) in a compact [B, anchors, Hkv, d] buffer.
 //   4. combine: anchor partials to bf16 dK/dV at the anchors' positions.
 #include <cuda_runtime.h>
 

@@ -5,7 +5,7 @@
 // iff j <= i && (i - j < n || f[j]), f = initial-or-separator ("SepLLM: Accelerate Large
 // Language Models ...", atlas.scime.ai summary, "Approach").
 //
-// One CTA per (query tile t of 128 rows, query head h, batch b). Its keys are split in two
+// Work item = (query tile t of 128 rows, query head h, batch b). Its keys are split in two
 // disjoint parts that together hold every kept key exactly once:
 //   * window tiles u = t, t-1, ..., lo(t), lo(t) = max(0, 128t - n + 1) / 128: whole 128-key
 //     tiles loaded by TMA in tile mode; FULL tiles need no mask, PARTIAL tiles apply keep()
@@ -15,13 +15,14 @@
 //     too arrive as TMA tiles.
 // Skipped tiles are never loaded.
 //
-// Warp roles (192 threads): warps 0-3 softmax (thread = query row = TMEM lane), warp 4 TMA
-// producer, warp 5 TMEM allocator + MMA issuer (one thread). Per key tile j:
-//   S_j = Q K_j^T                  (tcgen05.mma, A and B K-major in smem, D in TMEM S[j%2])
+// Persistent CTAs, one per SM, 352 threads: warps 0-7 softmax (two warps per query row, each
+// owning 64 key columns; thread = row = TMEM lane), warp 8 TMA producer, warp 9 TMEM allocator
+// and MMA issuer (one thread), warp 10 O storer. Per key tile j:
+//   S_j = Q K_j^T                  (tcgen05.mma, A and B K-major in smem, D in TMEM)
 //   P_j = exp2(S_j*c - m)          (softmax warps: tcgen05.ld S, online max with lazy
-//                                   rescale of O, tcgen05.st of bf16 P into TMEM P[j%2])
+//                                   rescale of O, tcgen05.st of bf16 P into TMEM)
 //   O  += P_j V_j                  (tcgen05.mma, A = P from TMEM, B = V MN-major in smem)
-// S_{j+1} is issued before PV_j so the tensor core works while softmax runs.
+// S_{j+1} is issued before PV_j so the tensor core works while the softmax runs.
 #include <cuda_runtime.h>
 
 #include <algorithm>

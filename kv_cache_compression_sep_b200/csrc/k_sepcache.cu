@@ -428,23 +428,6 @@ __device__ __forceinline__ int rank_to_slot(int r, int ninit, int sep_head, int 
   return a + s + P + (win_head + r) % w;
 }
 
-// N consecutive bf16 (N = 2 or 4, 4- or 8-byte aligned) to fp32.
-template <int N>
-__device__ __forceinline__ void load_bf16_vec(const __nv_bfloat16* p, float (&out)[N]) {
-  if constexpr (N == 4) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-    out[0] = __low2float(x); out[1] = __high2float(x);
-    out[2] = __low2float(y); out[3] = __high2float(y);
-  } else {
-    static_assert(N == 2, "two or four elements per lane");
-    const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(p));
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u);
-    out[0] = __low2float(x); out[1] = __high2float(x);
-  }
-}
-
 // N consecutive bf16 from shared memory (4- or 8-byte aligned) to fp32.
 template <int N>
 __device__ __forceinline__ void load_bf16_vec_smem(const __nv_bfloat16* p, float (&out)[N]) {

@@ -265,6 +265,4 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
-
 }  // namespace sep

@@ -61,32 +61,4 @@ __device__ __forceinline__ uint32_t window_keep_word(int w, long long i, long lo
   return range_word(lo > 0 ? lo : 0, hi, w) | (fbits & range_word(0, hi, w));
 }
 
-// Anchor flags of keys base..base+31 as a bit word (sep[j] != 0 or j < a); keys >= L read as 0.
-__device__ __forceinline__ uint32_t anchor_bits32(const uint8_t* __restrict__ sep_row,
-                                                  long long base, int L, int a) {
-  uint32_t bits = 0;
-  if (base + 32 <= L && ((reinterpret_cast<uintptr_t>(sep_row + base) & 15) == 0)) {
-    const uint4* p = reinterpret_cast<const uint4*>(sep_row + base);
-    const uint4 x0 = __ldg(p), x1 = __ldg(p + 1);
-    const uint32_t wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const uint32_t v = wv[q];
-      const uint32_t nib = (uint32_t)((v & 0xffu) != 0) | ((uint32_t)(((v >> 8) & 0xffu) != 0) << 1) |
-                           ((uint32_t)(((v >> 16) & 0xffu) != 0) << 2) |
-                           ((uint32_t)(((v >> 24) & 0xffu) != 0) << 3);
-      bits |= nib << (4 * q);
-    }
-  } else {
-    for (int c = 0; c < 32; ++c) {
-      const long long j = base + c;
-      if (j < L && sep_row[j] != 0) bits |= 1u << c;
-    }
-  }
-  const long long na = (long long)a - base;  // keys j < a are anchors
-  if (na > 0) bits |= (na >= 32) ? 0xffffffffu : ((1u << na) - 1u);
-  if (base + 32 > L) bits &= range_word(0, (long long)L - 1 - base, 0);
-  return bits;
-}
-
 }  // namespace sep

@@ -586,19 +586,24 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
   __syncthreads();
 
   // per-head softmax state (consumers)
-  // softmax state of this lane's own query (see halfwarp_reduce_own); V sums of every query
-  float m_own = -INFINITY, l_own = 0.f, acc[G][2 * HP];
+  // softmax state of this lane's own query (see halfwarp_reduce_own); V sums of every query,
+  // as pairs of consecutive elements for the packed fp32x2 arithmetic (lo: elements
+  // lane16 * HP + 2i, +1; hi: the same plus d/2)
+  static_assert(HP % 2 == 0, "rotation pairs per lane come in twos");
+  constexpr int HP2 = HP / 2;
+  float m_own = -INFINITY, l_own = 0.f;
+  float2 acc_lo[G][HP2], acc_hi[G][HP2];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
 #pragma unroll
-    for (int e = 0; e < 2 * HP; ++e) acc[g][e] = 0.f;
+    for (int i = 0; i < HP2; ++i) acc_lo[g][i] = acc_hi[g][i] = make_float2(0.f, 0.f);
   }
 
   {
     // ---------------------------------------------------------------- consumers
     // query heads of this KV head, rotated by RoPE(mq) (by RoPE(T - 1) without shifting) and
     // scaled by scale*log2(e)
-    float qr[G][2 * HP];
+    float2 q_lo[G][HP2], q_hi[G][HP2];
     {
       float2 qcs[HP];
 #pragma unroll
@@ -616,29 +621,39 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const __nv_bfloat16* qh = q + ((size_t)seq * Hq + kvh * G + g) * D;
+        float qa[HP], qb[HP];
 #pragma unroll
         for (int e = 0; e < HP; ++e) {
           const int k = lane16 * HP + e;
           const float x1 = __bfloat162float(qh[k]), x2 = __bfloat162float(qh[k + HALF]);
           const float2 rr = qcs[e];
-          qr[g][e] = (x1 * rr.x - x2 * rr.y) * scale_log2;
-          qr[g][HP + e] = (x2 * rr.x + x1 * rr.y) * scale_log2;
+          qa[e] = (x1 * rr.x - x2 * rr.y) * scale_log2;
+          qb[e] = (x2 * rr.x + x1 * rr.y) * scale_log2;
+        }
+#pragma unroll
+        for (int i = 0; i < HP2; ++i) {
+          q_lo[g][i] = make_float2(qa[2 * i], qa[2 * i + 1]);
+          q_hi[g][i] = make_float2(qb[2 * i], qb[2 * i + 1]);
         }
       }
     }
-    // cos/sin of this half-warp's current rank, advanced by kHalfWarps per step
-    float cr[HP], sr[HP], cd[HP], sd[HP];
+    // cos/sin of this half-warp's current rank, advanced by kHalfWarps per step (pairs of
+    // consecutive frequencies; nsd = -sin of the step)
+    float2 cr[HP2], sr[HP2], cd[HP2], sd[HP2], nsd[HP2];
     {
       const int rf = r0 + hw;
 #pragma unroll
-      for (int e = 0; e < HP; ++e) {
-        const int k = lane16 * HP + e;
+      for (int i = 0; i < HP2; ++i) {
+        const int k = lane16 * HP + 2 * i;
         const float2 v0 = (rf < r1) ? rope_cs[(size_t)rf * HALF + k] : make_float2(1.f, 0.f);
-        cr[e] = v0.x;
-        sr[e] = v0.y;
-        const float2 stp = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
-        cd[e] = stp.x;
-        sd[e] = stp.y;
+        const float2 v1 = (rf < r1) ? rope_cs[(size_t)rf * HALF + k + 1] : make_float2(1.f, 0.f);
+        cr[i] = make_float2(v0.x, v1.x);
+        sr[i] = make_float2(v0.y, v1.y);
+        const float2 t0 = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
+        const float2 t1 = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k + 1];
+        cd[i] = make_float2(t0.x, t1.x);
+        sd[i] = make_float2(t0.y, t1.y);
+        nsd[i] = make_float2(-t0.y, -t1.y);
       }
     }
     bool ok = true;
@@ -665,23 +680,32 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
 #pragma unroll
           for (int e = 0; e < HP; ++e) k1[e] = k2[e] = v1[e] = v2[e] = 0.f;
         }
+        // rotate (y1, y2) = RoPE(rank) (k1, k2) and form the G partial dot products, two
+        // frequencies per packed instruction
+        float2 part2[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) part2[g] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < HP2; ++i) {
+          const float2 x1 = make_float2(k1[2 * i], k1[2 * i + 1]);
+          const float2 x2 = make_float2(k2[2 * i], k2[2 * i + 1]);
+          float2 y1 = x1, y2 = x2;
+          if constexpr (!ORIG) {
+            y1 = f2_sub(f2_mul(x1, cr[i]), f2_mul(x2, sr[i]));
+            y2 = f2_fma(x2, cr[i], f2_mul(x1, sr[i]));
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) part2[g] = f2_fma(q_lo[g][i], y1, f2_fma(q_hi[g][i], y2, part2[g]));
+        }
         float part[G];
 #pragma unroll
-        for (int g = 0; g < G; ++g) part[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < HP; ++e) {
-          const float y1 = ORIG ? k1[e] : k1[e] * cr[e] - k2[e] * sr[e];
-          const float y2 = ORIG ? k2[e] : k2[e] * cr[e] + k1[e] * sr[e];
-#pragma unroll
-          for (int g = 0; g < G; ++g) part[g] = fmaf(qr[g][e], y1, fmaf(qr[g][HP + e], y2, part[g]));
-        }
+        for (int g = 0; g < G; ++g) part[g] = part2[g].x + part2[g].y;
         if constexpr (!ORIG) {
 #pragma unroll
-          for (int e = 0; e < HP; ++e) {
-            const float cn = cr[e] * cd[e] - sr[e] * sd[e];
-            const float sn = sr[e] * cd[e] + cr[e] * sd[e];
-            cr[e] = cn;
-            sr[e] = sn;
+          for (int i = 0; i < HP2; ++i) {
+            const float2 cn = f2_fma(cr[i], cd[i], f2_mul(sr[i], nsd[i]));
+            sr[i] = f2_fma(sr[i], cd[i], f2_mul(cr[i], sd[i]));
+            cr[i] = cn;
           }
         }
         // this lane's query score; the online softmax of that query only, its probability
@@ -697,8 +721,12 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
 #pragma unroll
           for (int g = 0; g < G; ++g) {
             const float ag = __shfl_sync(0xffffffffu, alpha, lane_of_query<G>(g), 16);
+            const float2 ag2 = make_float2(ag, ag);
 #pragma unroll
-            for (int e = 0; e < 2 * HP; ++e) acc[g][e] *= ag;
+            for (int i = 0; i < HP2; ++i) {
+              acc_lo[g][i] = f2_mul(acc_lo[g][i], ag2);
+              acc_hi[g][i] = f2_mul(acc_hi[g][i], ag2);
+            }
           }
         }
         const float p_own = valid ? ex2(sc - m_own) : 0.f;
@@ -706,10 +734,11 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float pg = __shfl_sync(0xffffffffu, p_own, lane_of_query<G>(g), 16);
+          const float2 pg2 = make_float2(pg, pg);
 #pragma unroll
-          for (int e = 0; e < HP; ++e) {
-            acc[g][e] = fmaf(pg, v1[e], acc[g][e]);
-            acc[g][HP + e] = fmaf(pg, v2[e], acc[g][HP + e]);
+          for (int i = 0; i < HP2; ++i) {
+            acc_lo[g][i] = f2_fma(pg2, make_float2(v1[2 * i], v1[2 * i + 1]), acc_lo[g][i]);
+            acc_hi[g][i] = f2_fma(pg2, make_float2(v2[2 * i], v2[2 * i + 1]), acc_hi[g][i]);
           }
         }
       }
@@ -733,6 +762,17 @@ __global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
     }
   }
 
+  float acc[G][2 * HP];  // V sums, elements lane16 * HP + e (e < HP) and the same plus d/2
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int i = 0; i < HP2; ++i) {
+      acc[g][2 * i] = acc_lo[g][i].x;
+      acc[g][2 * i + 1] = acc_lo[g][i].y;
+      acc[g][HP + 2 * i] = acc_hi[g][i].x;
+      acc[g][HP + 2 * i + 1] = acc_hi[g][i].y;
+    }
+  }
   // every query's softmax state from the lanes that own it
   float mrun[G], lrun[G];
 #pragma unroll

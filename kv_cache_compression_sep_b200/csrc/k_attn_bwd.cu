@@ -644,7 +644,7 @@ struct DkvBar {
   uint64_t drain;
   uint64_t item_full[4];  // ring of fetched work-item indices (producer -> MMA, softmax)
   int item_x[4];
-  float lse2[NST][128];
+  float nlse2[NST][128];  // -log2-domain LSE of each query of the stage (-inf past L)
   float delta[NST][128];
   uint32_t tmem_base;
   int abort_flag;
@@ -782,7 +782,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
           const int col = lane * 4 + z;
           const long long i = (long long)t * 128 + col;
           const bool v = i < p.L;
-          bar->lse2[st][col] = v ? __ldg(p.lse + base + i) * 1.4426950408889634f : INFINITY;
+          bar->nlse2[st][col] = v ? -__ldg(p.lse + base + i) * 1.4426950408889634f : -INFINITY;
           bar->delta[st][col] = v ? __ldg(p.delta + base + i) : 0.f;
         }
         mbar_arrive(&bar->q_full[st]);
@@ -995,7 +995,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         }
         tc_fence_after();
         const uint32_t aS = tmem + lane_off + 128 * h, aP = aS + 64;
-        const float* lse2 = &bar->lse2[st][64 * h];
+        const float* nlse2 = &bar->nlse2[st][64 * h];
         const float* dl = &bar->delta[st][64 * h];
         // two 32-column chunks; packed chunk c lands in columns 16c..16c+15, already read
 #pragma unroll
@@ -1005,19 +1005,21 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
           tmem_ld32(aP + 32 * ch, dp);
           tmem_ld_wait();
           uint32_t pk[16], dk16[16];
+          // two queries per packed fp32x2 instruction: x = S * scale*log2(e) - lse2,
+          // P = exp2(x) on kept pairs, dS = P (dP - Delta)
+          const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
-            float pv[2], dv2[2];
-#pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const int col = 32 * ch + c + z;
-              const bool kp = (keep[ch] >> (c + z)) & 1u;
-              const float pr = kp ? ex2(fmaf(__uint_as_float(sv[c + z]), sl2, -lse2[col])) : 0.f;
-              pv[z] = pr;
-              dv2[z] = pr * (__uint_as_float(dp[c + z]) - dl[col]);
-            }
-            pk[c >> 1] = pack_bf16x2(pv[0], pv[1]);
-            dk16[c >> 1] = pack_bf16x2(dv2[0], dv2[1]);
+            const int col = 32 * ch + c;
+            const float2 x = f2_fma(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                    sl2x2, *reinterpret_cast<const float2*>(nlse2 + col));
+            const float2 dd = f2_sub(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                     *reinterpret_cast<const float2*>(dl + col));
+            const float p0 = ((keep[ch] >> c) & 1u) ? ex2(x.x) : 0.f;
+            const float p1 = ((keep[ch] >> (c + 1)) & 1u) ? ex2(x.y) : 0.f;
+            const float2 ds = f2_mul(make_float2(p0, p1), dd);
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+            dk16[c >> 1] = pack_bf16x2(ds.x, ds.y);
           }
           asm volatile(
               "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "

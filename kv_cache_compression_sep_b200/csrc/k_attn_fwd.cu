@@ -415,17 +415,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         // ---- P = exp2(S * scale*log2e - m), partial row sum (8 chains), packed to bf16 pairs
         // in place over the already consumed S registers (pair c/2 <= c)
-        float sum8[8];
+        // two columns per packed fp32x2 instruction (scale and subtract, and the row sums)
+        float2 sum4[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) sum8[q] = 0.f;
+        for (int q = 0; q < 4; ++q) sum4[q] = make_float2(0.f, 0.f);
+        const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const float e0 = ex2(fmaf(__uint_as_float(s[c]), sl2, -m_use));
-          const float e1 = ex2(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
-          sum8[(c >> 1) & 7] += e0 + e1;
-          s[c >> 1] = pack_bf16x2(e0, e1);
+          const float2 x = f2_fma(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                  sl2x2, nm2);
+          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          sum4[(c >> 1) & 3] = f2_add(sum4[(c >> 1) & 3], e);
+          s[c >> 1] = pack_bf16x2(e.x, e.y);
         }
-        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        l_run += ((sum4[0].x + sum4[0].y) + (sum4[1].x + sum4[1].y)) +
+                 ((sum4[2].x + sum4[2].y) + (sum4[3].x + sum4[3].y));
         // P and O: the previous tile's P V must be complete (it read P and accumulated O)
         if (g > 0 &&
             !__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {

@@ -6,7 +6,7 @@ and to its n most recent neighbours. [BD] "SepLLM's Architecture" writes the att
 O = M(A, V, M_b) with a binary n x n mask M_b. This file writes that out as plain masked
 softmax attention in float64, plus its analytic gradients, with no blocking or fusion.
 
-Readings where the pages are silent (listed again in the design doc):
+Readings where the pages are silent:
 * "n neighbours" = the n most recent tokens including the query itself: i - n < j <= i.
 * "initial tokens" = positions j < a; every kept pair is causal (j <= i).
 * A zero in M_b is a logit of -inf (the pair is dropped from the softmax).

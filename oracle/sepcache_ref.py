@@ -6,7 +6,7 @@ Separator Cache that keeps only separator KV of older tokens, with total capacit
 "Limitations & Caveats" and [AS] "Measured effects" (removing positional-encoding shifting)
 say positions are taken inside the cache, not in the original text.
 
-Readings where the pages are silent (listed again in the design doc):
+Readings where the pages are silent:
 * Without a usage threshold (c = None): fixed partitions a + s + w and a Past Window Cache of
   size 0, so compression happens one token at a time: when the window overflows, its oldest
   token moves to the separator cache if it is a separator and is evicted otherwise; when the

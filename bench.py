@@ -319,14 +319,8 @@ def native(args, rank, world, dev):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, separator flags as configured)",
-        "config": {"workload": "pythia160m-train-attention + sepcache-decode step",
-                   "train": {"B": 8, "Hq": 12, "Hkv": 12, "L": 2048, "d": 64, "a": 4, "n": 64,
-                             "flags": "geometric(mean 10) segments"},
-                   "decode": {"S": 64, "Hq": 32, "Hkv": 8, "d": 128, "c": 800, "a": 4, "s": 64,
-                              "w": 732, "theta": 5e5, "occupancy": 800},
-                   "global_batch": 8 * world, "seq_len": 2048, "parallelism": f"dp{world}",
-                   "l2": "flushed between timed steps (256 MiB write)",
-                   "step": "one CUDA graph: mask build, fwd, bwd, cache update, decode"},
+        "config": step_config(world, "flushed between timed steps (256 MiB write)",
+                              "one CUDA graph: mask build, fwd, bwd, cache update, decode"),
         "roofline": roof,
         "components": comp_out,
         "e2e": e2e,
@@ -505,6 +499,18 @@ def cpu_baseline(seconds):
             "seconds": dt}
 
 
+def step_config(world, l2, step):
+    """The default step's configuration, shared by both arms (the reference arm runs a sample
+    of the same step)."""
+    return {"workload": "pythia160m-train-attention + sepcache-decode step",
+            "train": {"B": 8, "Hq": 12, "Hkv": 12, "L": 2048, "d": 64, "a": 4, "n": 64,
+                      "flags": "geometric(mean 10) segments"},
+            "decode": {"S": 64, "Hq": 32, "Hkv": 8, "d": 128, "c": 800, "a": 4, "s": 64,
+                       "w": 732, "theta": 5e5, "occupancy": 800},
+            "global_batch": 8 * world, "seq_len": 2048, "parallelism": f"dp{world}",
+            "l2": l2, "step": step}
+
+
 def reference(args, rank, world):
     if rank != 0:
         return None
@@ -525,7 +531,9 @@ def reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "pythia160m-train-attention + sepcache-decode step (sample)"},
+            "config": step_config(world, "host CPU run (no GPU L2)",
+                                  "a bounded sample of the step on the host cores "
+                                  "(cpu_baseline.sample)"),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,

@@ -629,7 +629,7 @@ struct DkvCfg {
   static constexpr int KVB = (D == 128) ? 1 : 2;  // K/V buffers (items in flight)
   static constexpr int NST = (D == 128) ? 2 : 3;  // Q/dO stages (pairs in flight)
   static constexpr int SMEM_TILES = TILE * (2 * KVB + 2 * NST);
-  static constexpr int COL_S0 = 0;     // half h: S^T at 128h, dP^T at 128h + 64
+  // TMEM columns: half h holds S^T at 128h and dP^T at 128h + 64
   static constexpr int COL_DV = 256, COL_DK = 256 + D;
   static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, storer
 };

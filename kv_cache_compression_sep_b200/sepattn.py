@@ -89,9 +89,26 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _cuda(t, dtype, name):
-    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
-        raise SepError(f"{name} must be a contiguous CUDA {dtype} tensor")
+def _cuda(t, dtype, name, shape=None):
+    """t must be a contiguous CUDA tensor of this dtype and, if given, this shape. The checks
+    run before any launch: a buffer of the wrong size would be read or written out of bounds
+    by the kernels, which trust the sizes passed to the library."""
+    if not isinstance(t, torch.Tensor):
+        raise SepError(f"{name} must be a torch.Tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise SepError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise SepError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise SepError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise SepError(f"{name} must be on a CUDA device (there is no CPU path)")
+
+
+def _dims(t, ndim, name):
+    if not isinstance(t, torch.Tensor) or t.dim() != ndim:
+        raise SepError(f"{name} must be a {ndim}-D tensor")
+    return tuple(t.shape)
 
 
 def sep_last_device_error() -> int:
@@ -121,11 +138,18 @@ class SepMask:
 def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = TILE,
                    out: SepMask | None = None) -> SepMask:
     """Mask artefacts of `sep` [B, L] uint8; `out` reuses the buffers of an earlier result."""
+    B, L = _dims(sep, 2, "sep")
     _cuda(sep, torch.uint8, "sep")
-    B, L = sep.shape
-    T, U = -(-L // bm), -(-L // bn)
+    T, U = -(-L // max(bm, 1)), -(-L // max(bn, 1))
     dev = sep.device
     if out is not None:
+        for name, dtype, shape in (("anchor_idx", torch.int32, (B, L)),
+                                   ("anchor_cnt", torch.int32, (B,)),
+                                   ("anchor_bits", torch.int32, (B, -(-L // 32))),
+                                   ("gather_end", torch.int32, (B, T)),
+                                   ("tile_map", torch.int8, (B, T, U)),
+                                   ("kept", torch.int64, (B,))):
+            _cuda(getattr(out, name), dtype, f"out.{name}", shape)
         out.sep, out.a, out.n = sep, a, n
     else:
         out = SepMask(sep=sep,
@@ -149,7 +173,25 @@ def sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d) -> int:
     return int(_lib.sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d))
 
 
+def _attn_inputs(q, k, v, mask):
+    """Shapes of q [B, L, Hq, d] and k, v [B, L, Hkv, d], checked against each other and the
+    mask's flags [B, L]."""
+    B, L, Hq, d = _dims(q, 4, "q")
+    Hkv = _dims(k, 4, "k")[2]
+    if tuple(mask.sep.shape) != (B, L):
+        raise SepError(f"mask was built for flags of shape {tuple(mask.sep.shape)}, "
+                       f"q needs {(B, L)}")
+    if Hkv < 1 or Hq % Hkv != 0:
+        raise SepError(f"Hq = {Hq} is not a multiple of Hkv = {Hkv}")
+    _cuda(k, torch.bfloat16, "k", (B, L, Hkv, d))
+    _cuda(v, torch.bfloat16, "v", (B, L, Hkv, d))
+    _cuda(q, torch.bfloat16, "q")
+    return B, L, Hq, Hkv, d
+
+
 def _workspace(nbytes, device, ws):
+    if ws is not None:
+        _cuda(ws, torch.uint8, "workspace")
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
     return ws
@@ -161,13 +203,12 @@ def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspa
 
     stage=None runs the whole call; stage=0/1 runs sep_attn_fwd_stage (timing one pass).
     """
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _cuda(t, torch.bfloat16, name)
-    B, L, Hq, d = q.shape
-    Hkv = k.shape[2]
+    B, L, Hq, Hkv, d = _attn_inputs(q, k, v, mask)
     scale = d ** -0.5 if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device) if lse is None else lse
+    _cuda(o, torch.bfloat16, "out", (B, L, Hq, d))
+    _cuda(lse, torch.float32, "lse", (B, Hq, L))
     nbytes = sep_attn_fwd_workspace_size(B, L, Hkv, d)
     ws = _workspace(nbytes, q.device, workspace)
     mc = mask._c()
@@ -187,13 +228,12 @@ def sep_attn_fwd_noalloc(q, k, v, mask: SepMask, scale=None, out=None, lse=None)
     Problems whose compacted anchors exceed SEP_NOALLOC_SCRATCH_BYTES raise SepError
     (SEP_ERR_SCRATCH_LIMIT). Calls that may overlap in time share the scratch and race.
     """
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _cuda(t, torch.bfloat16, name)
-    B, L, Hq, d = q.shape
-    Hkv = k.shape[2]
+    B, L, Hq, Hkv, d = _attn_inputs(q, k, v, mask)
     scale = d ** -0.5 if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device) if lse is None else lse
+    _cuda(o, torch.bfloat16, "out", (B, L, Hq, d))
+    _cuda(lse, torch.float32, "lse", (B, Hq, L))
     mc = mask._c()
     _check(_lib.sep_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale),
                                      mask.a, mask.n, ctypes.byref(mc), _ptr(o), _ptr(lse),
@@ -207,16 +247,18 @@ def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=Non
 
     stage=None runs the whole call; stage=0/1/2 runs sep_attn_bwd_stage (timing one pass).
     """
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
-        _cuda(t, torch.bfloat16, name)
-    _cuda(lse, torch.float32, "lse")
-    B, L, Hq, d = q.shape
-    Hkv = k.shape[2]
+    B, L, Hq, Hkv, d = _attn_inputs(q, k, v, mask)
+    _cuda(o, torch.bfloat16, "o", (B, L, Hq, d))
+    _cuda(dout, torch.bfloat16, "dout", (B, L, Hq, d))
+    _cuda(lse, torch.float32, "lse", (B, Hq, L))
     scale = d ** -0.5 if scale is None else scale
     if grads is None:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     else:
         dq, dk, dv = grads
+    _cuda(dq, torch.bfloat16, "dq", (B, L, Hq, d))
+    _cuda(dk, torch.bfloat16, "dk", (B, L, Hkv, d))
+    _cuda(dv, torch.bfloat16, "dv", (B, L, Hkv, d))
     nbytes = sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d)
     ws = _workspace(nbytes, q.device, workspace)
     mc = mask._c()
@@ -249,6 +291,9 @@ class SepCache:
         self.n = a + s + self.past + w
         self.rope_theta = float(rope_theta)
         dev = torch.device(device)
+        if dev.type != "cuda":
+            raise SepError(f"SepCache state must live on a CUDA device, not {dev} "
+                           "(there is no CPU path)")
         self.k_slots = torch.zeros(S, Hkv, self.n, d, dtype=torch.bfloat16, device=dev)
         self.v_slots = torch.zeros(S, Hkv, self.n, d, dtype=torch.bfloat16, device=dev)
         self.slot_pos = torch.empty(S, self.n, dtype=torch.int32, device=dev)
@@ -265,10 +310,10 @@ class SepCache:
 
     def sepcache_prefill(self, k, v, sep):
         """Seeds every sequence with a prompt: k, v [S, L, Hkv, d] bf16, sep [S, L] uint8."""
-        _cuda(k, torch.bfloat16, "k")
-        _cuda(v, torch.bfloat16, "v")
-        _cuda(sep, torch.uint8, "sep")
-        L = k.shape[1]
+        L = _dims(k, 4, "k")[1]
+        _cuda(k, torch.bfloat16, "k", (self.S, L, self.Hkv, self.d))
+        _cuda(v, torch.bfloat16, "v", (self.S, L, self.Hkv, self.d))
+        _cuda(sep, torch.uint8, "sep", (self.S, L))
         _check(_lib.sepcache_prefill(ctypes.byref(self._st), _ptr(k), _ptr(v), _ptr(sep), L,
                                      _stream()), "sepcache_prefill")
 
@@ -290,16 +335,19 @@ class SepCache:
             dst.copy_(sd[k])
 
     def sepcache_update(self, k_new, v_new, sep_new):
-        _cuda(k_new, torch.bfloat16, "k_new")
-        _cuda(v_new, torch.bfloat16, "v_new")
-        _cuda(sep_new, torch.uint8, "sep_new")
+        _cuda(k_new, torch.bfloat16, "k_new", (self.S, self.Hkv, self.d))
+        _cuda(v_new, torch.bfloat16, "v_new", (self.S, self.Hkv, self.d))
+        _cuda(sep_new, torch.uint8, "sep_new", (self.S,))
         _check(_lib.sepcache_update(ctypes.byref(self._st), _ptr(k_new), _ptr(v_new),
                                     _ptr(sep_new), _stream()), "sepcache_update")
 
     def sepcache_decode(self, q, scale=None, out=None, lse=None):
-        _cuda(q, torch.bfloat16, "q")
+        _cuda(q, torch.bfloat16, "q", (self.S, self.Hq, self.d))
         scale = self.d ** -0.5 if scale is None else scale
         o = torch.empty_like(q) if out is None else out
+        _cuda(o, torch.bfloat16, "out", (self.S, self.Hq, self.d))
+        if lse is not None:
+            _cuda(lse, torch.float32, "lse", (self.S, self.Hq))
         _check(_lib.sepcache_decode(ctypes.byref(self._st), _ptr(q), _ptr(o), _ptr(lse),
                                     float(scale), _stream()), "sepcache_decode")
         return o

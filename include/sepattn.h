@@ -155,9 +155,16 @@ int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const se
  * Efficiency", beiduofen.top): a initial slots, a separator FIFO of s slots, a local-window
  * FIFO of w slots and, when the usage threshold c is non-zero, a Past Window of P = c - a - w
  * slots that holds the tokens leaving the window until the total usage reaches c. With c = 0
- * there is no Past Window and compression is one token at a time. Keys are stored without
- * rotary embedding; sepcache_decode applies RoPE at in-cache positions (positional-encoding
- * shifting, SepLLM project card, "Limitations & Caveats").
+ * there is no Past Window and compression is one token at a time. Keys are seen at their
+ * positions inside the cache (positional-encoding shifting, SepLLM project card, "Limitations &
+ * Caveats"): the key of rank p at RoPE(p), the newest token's query at RoPE(occupied - 1).
+ *
+ * Storage of the keys: every key is stored rotated once, in bf16, by RoPE(u) where u is a
+ * counter that differs from its rank by an offset shared by its whole block: its original
+ * position t for initial, past-window and window keys, and its admission index A (the A-th
+ * separator admitted to the FIFO since the cache was empty) for separators. A key is rotated by
+ * RoPE(t) when it is appended and by RoPE(A - t) more when it enters the separator FIFO;
+ * decode rotates the query once per block. Rotation angles are formed in fp64.
  *
  * Slots per sequence: n = a + s + P + w (P = 0 when c = 0), in this order: initial, separator
  * ring, past window, window ring. Every pointer below is caller-owned device memory; the
@@ -166,7 +173,7 @@ int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const se
  *   slot_pos          S * n int32             original position held by each slot (-1 empty)
  *   slot_sep          S * n uint8             separator flag of each slot's token
  *   meta              S * SEPCACHE_META int32 per-sequence counters (see below)
- *   rope_cs           n * d float             cos/sin table of in-cache positions 0..n-1
+ *   rope_freq         d / 2 double            RoPE inverse frequencies theta^(-2k/d)
  */
 #define SEPCACHE_META 8
 /* meta[seq * SEPCACHE_META + ...] */
@@ -177,29 +184,32 @@ int sep_attn_bwd_stage(int stage, const sep_bf16* q, const sep_bf16* k, const se
 #define SEPCACHE_META_WIN_HEAD 4  /* window FIFO: ring index of the oldest entry */
 #define SEPCACHE_META_WIN_CNT 5   /* window FIFO: entries */
 #define SEPCACHE_META_PAST_CNT 6  /* past window: entries (c > 0) */
+#define SEPCACHE_META_SEP_ADMIT 7 /* separators admitted to the FIFO so far (the FIFO holds
+                                     admission indices SEP_ADMIT - SEP_CNT .. SEP_ADMIT - 1) */
 
 typedef struct SepCacheState {
-  int32_t S, Hq, Hkv, d;     /* sequences, query heads, KV heads, head dim (d = 128 or 64) */
+  int32_t S, Hq, Hkv, d;     /* sequences, query heads, KV heads, head dim (d = 128 or 64);
+                                Hq / Hkv query heads share a KV head, 1 to 8 of them */
   int32_t a, s, w;           /* initial / separator / window capacities */
   int32_t c;                 /* usage threshold of the Past Window (0: none; else > a + s + w) */
-  int32_t original_positions; /* 0: positional-encoding shifting, keys stored un-rotated and
-                                 rotated at their in-cache rank by every decode; 1: no
-                                 shifting, keys stored rotated at their original positions */
+  int32_t original_positions; /* 0: positional-encoding shifting (ranks inside the cache);
+                                 1: no shifting, every key and the query at their original
+                                 positions (keys stay at RoPE(t) in every block) */
   float rope_theta;          /* RoPE base: angle of pair k at position p = p * theta^(-2k/d) */
   sep_bf16* k_slots;
   sep_bf16* v_slots;
   int32_t* slot_pos;
   uint8_t* slot_sep;
   int32_t* meta;
-  float* rope_cs;
+  double* rope_freq;
 } SepCacheState;
 
-/* Empties every sequence (meta and slot_pos) and fills rope_cs. Call once before use. */
+/* Empties every sequence (meta and slot_pos) and fills rope_freq. Call once before use. */
 int sepcache_state_init(const SepCacheState* st, sep_stream_t stream);
 
 /*
  * sepcache_update - append one token to every sequence (one kernel).
- * k_new, v_new [S, Hkv, d] un-rotated; sep_new [S] uint8. Token t of a sequence goes to
+ * k_new, v_new [S, Hkv, d] without rotary embedding; sep_new [S] uint8. Token t of a sequence goes to
  * initial slot t when t < a; otherwise to the window. If the window then holds more than w
  * tokens its oldest token leaves. With c = 0 it goes into the separator FIFO if it is a
  * separator and is dropped otherwise. With c > 0 it goes to the Past Window, and when the
@@ -218,8 +228,11 @@ int sepcache_update(const SepCacheState* st, const sep_bf16* k_new, const sep_bf
  * This is how a prompt processed by sep_attn_fwd (the prefill pass) hands its keys and values
  * to streaming decode ("How SepLLM reorchestrates the language model...", "SepLLM's
  * Architecture: Composing Efficiency": initial, separator and local-window blocks).
- * k, v [S, L, Hkv, d] un-rotated (the layout sep_attn_fwd reads); sep [S, L] uint8. L >= 1;
- * s <= 16384 and c = 0 (SEP_ERR_UNSUPPORTED otherwise).
+ * With a Past Window (c > 0) the compressions the updates would have made are replayed run by
+ * run: each run of c - a - w - (separators held) tokens that has left the window is one
+ * compression, so the call costs one block-wide count per run.
+ * k, v [S, L, Hkv, d] without rotary embedding (the layout sep_attn_fwd reads); sep [S, L]
+ * uint8. L >= 1; s <= 16384 (SEP_ERR_UNSUPPORTED otherwise).
  */
 int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16* v,
                      const uint8_t* sep, int L, sep_stream_t stream);
@@ -227,10 +240,10 @@ int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16*
 /*
  * sepcache_decode - single-query attention of each sequence's newest token over its cache.
  * Logical order = [initial | separators oldest first | past window oldest first | window
- * oldest first]; the key of rank p is rotated by RoPE(p) and the query by RoPE(m),
- * m = occupied - 1 (its own rank). With original_positions = 1 (training-free use without
- * shifting) the keys were rotated at their original positions when they entered the cache,
- * and the query is rotated at its own original position T - 1.
+ * oldest first]; the key of rank p is seen at RoPE(p) and the query at RoPE(m),
+ * m = occupied - 1 (its own rank): the stored keys are read as they are and the query is rotated
+ * once per block by RoPE(m - offset of the block). With original_positions = 1 (training-free
+ * use without shifting) keys and query are at their original positions (query at T - 1).
  * q [S, Hq, d] un-rotated; o [S, Hq, d] bf16; lse [S, Hq] fp32 natural log (nullable).
  * Call after sepcache_update of the same step.
  */
@@ -245,6 +258,19 @@ int sepcache_export_order(const SepCacheState* st, int32_t* pos_out, int32_t* co
 /* Reads and clears the sticky device error word of the current device (synchronises the
  * device). Returns SEP_OK or the first SEP_ERR_* a kernel recorded. */
 int sep_last_device_error(void);
+
+/*
+ * sep_set_wait_limit_ns - test hook for the device-side failure path.
+ *
+ * Every wait of the kernels on a pipeline barrier is bounded; when one runs out the kernel
+ * records SEP_ERR_TIMEOUT in the sticky device error word, lets the copies and tensor-core work
+ * it issued finish, frees its tensor memory and returns. This call sets the limit of the
+ * pipeline waits of the attention forward kernels launched afterwards, process-wide (ns = 0
+ * restores the default of 1.5 s); waits that drain issued work always keep 1.5 s. A very short
+ * limit makes a normal launch give up part-way, which is how a test exercises that path
+ * without any fault. Returns SEP_OK.
+ */
+int sep_set_wait_limit_ns(unsigned long long ns);
 
 /* Human-readable name of a status code. */
 const char* sep_status_string(int status);
@@ -264,7 +290,10 @@ const char* sep_status_string(int status);
  * above SEP_NOALLOC_SCRATCH_BYTES returns SEP_ERR_SCRATCH_LIMIT before any device work.
  * Setup: the first call on each device (with that device current) looks up the array's device
  * address with cudaGetSymbolAddress, which loads the library's module on that device; make that
- * first call before any stream capture. A failed lookup returns SEP_ERR_CUDA.
+ * first call before any stream capture. A failed lookup returns SEP_ERR_CUDA. The address is
+ * cached per device for the life of the process: after cudaDeviceReset (or anything else that
+ * destroys and recreates the device's primary context) it is stale, so this call must not be
+ * used again in that process.
  * Zeroing: none is needed; the compaction writes every row the attention kernel reads (the
  * anchors, then zero rows up to the end of their last 128-row tile).
  * Concurrency: every call on a device shares the one array. Calls that may overlap in time

@@ -5,11 +5,17 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
 #include "../../include/sepattn.h"
 #include "sep_launch.h"
+
+namespace sep {
+static std::atomic<unsigned long long> g_pipeline_wait_ns{kDefaultPipelineWaitNs};
+unsigned long long pipeline_wait_limit_ns() { return g_pipeline_wait_ns.load(); }
+}  // namespace sep
 
 namespace {
 
@@ -230,11 +236,11 @@ static int check_cache(const SepCacheState* st) {
   if (st->Hq % st->Hkv != 0) return SEP_ERR_INVALID_ARG;
   const int G = st->Hq / st->Hkv;
   if (st->d != 64 && st->d != 128) return SEP_ERR_UNSUPPORTED;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return SEP_ERR_UNSUPPORTED;
+  if (G > 8) return SEP_ERR_UNSUPPORTED;
   if (!st->k_slots || !st->v_slots || !st->slot_pos || !st->slot_sep || !st->meta ||
-      !st->rope_cs)
+      !st->rope_freq)
     return SEP_ERR_INVALID_ARG;
-  if (!aligned16(st->k_slots) || !aligned16(st->v_slots) || !aligned16(st->rope_cs))
+  if (!aligned16(st->k_slots) || !aligned16(st->v_slots) || !aligned16(st->rope_freq))
     return SEP_ERR_MISALIGNED;
   if (!(st->rope_theta > 0.f)) return SEP_ERR_INVALID_ARG;
   // usage threshold of the Past Window: 0 (none) or above the three fixed blocks
@@ -264,7 +270,7 @@ int sepcache_prefill(const SepCacheState* st, const sep_bf16* k, const sep_bf16*
   int e = check_cache(st);
   if (e != SEP_OK) return e;
   if (!k || !v || !sep || L < 1) return SEP_ERR_INVALID_ARG;
-  if (st->s > 16384 || st->c != 0) return SEP_ERR_UNSUPPORTED;
+  if (st->s > 16384) return SEP_ERR_UNSUPPORTED;
   if (!aligned16(k) || !aligned16(v)) return SEP_ERR_MISALIGNED;
   return cuda_status(sep::launch_sepcache_prefill(*st, k, v, sep, L,
                                                   reinterpret_cast<cudaStream_t>(stream)));
@@ -316,6 +322,11 @@ int sep_attn_fwd_noalloc(const sep_bf16* q, const sep_bf16* k, const sep_bf16* v
   if (!scratch) return SEP_ERR_CUDA;
   return attn_fwd_impl(3, q, k, v, B, L, Hq, Hkv, d, scale, a, n, mask, o, lse, scratch,
                        (size_t)SEP_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int sep_set_wait_limit_ns(unsigned long long ns) {
+  sep::g_pipeline_wait_ns.store(ns ? ns : sep::kDefaultPipelineWaitNs);
+  return SEP_OK;
 }
 
 const char* sep_status_string(int status) {

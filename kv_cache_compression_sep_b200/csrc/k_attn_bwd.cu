@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int g = 0;
+      int kq = 0, kd = 0;  // items whose Q / dO load was issued
       bool ok = true;
       int ge_cur = bwd_item_ge(p, blockIdx.x);
       for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
           ok = false;
           break;
         }
+        kq = k + 1;
         mbar_arrive_expect_tx(&bar->q_full[qb], C::TILE);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_4d(sQ + qb * C::TILE + kb * kBoxBytes, &p.tmQ, &bar->q_full[qb], kb * 64, it.h,
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
               ok = false;
               break;
             }
+            kd = k + 1;
             mbar_arrive_expect_tx(&bar->do_full[db], C::TILE);
             for (int kb = 0; kb < C::KB; ++kb)
               tma_load_4d(sdO + db * C::TILE + kb * kBoxBytes, &p.tmdO, &bar->do_full[db],
@@ -301,10 +304,16 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         }
       }
       if (!ok) {
+        // drain: the loads of the last NST key tiles, Q and dO tiles that may be in flight
+        // (older phases completed already, so their waits return at once)
         for (int gg = max(0, g - NST); gg < g; ++gg) {
           mbar_wait(&bar->k_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
           mbar_wait(&bar->v_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
         }
+        for (int kk = max(0, kq - 2); kk < kq; ++kk)
+          mbar_wait(&bar->q_full[kk & 1], (kk >> 1) & 1, nullptr, nullptr);
+        for (int kk = max(0, kd - DOB); kk < kd; ++kk)
+          mbar_wait(&bar->do_full[kk % DOB], (kk / DOB) & 1, nullptr, nullptr);
       }
     }
   } else if (warp == 9) {
@@ -732,6 +741,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
   if (warp == 8) {
     // ---------------------------------------------------------------- producer (whole warp)
     int P = 0;
+    int nkv = 0;  // items whose K/V load was issued
     bool ok = true;
     // Items are taken one at a time from the global counter (counters[2]) once the K/V buffer
     // they will use is free, and published to the other roles through the item ring; the
@@ -750,6 +760,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       x = __shfl_sync(0xffffffffu, x, 0);
       if (x >= nitems) break;
       const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+      nkv = I + 1;
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar->kv_full[kb], 2 * C::TILE);
         const int krow = it.unit * 128;
@@ -789,8 +800,11 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       }
     }
     if (lane == 0 && !ok) {
+      // drain: the Q/dO loads of the last NST pairs and the K/V loads of the last KVB items
       for (int pp = max(0, P - NST); pp < P; ++pp)
         mbar_wait(&bar->q_full[pp % NST], (pp / NST) & 1, nullptr, nullptr);
+      for (int ii = max(0, nkv - KVB); ii < nkv; ++ii)
+        mbar_wait(&bar->kv_full[ii % KVB], (ii / KVB) & 1, nullptr, nullptr);
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer

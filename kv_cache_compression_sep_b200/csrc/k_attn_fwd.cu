@@ -41,6 +41,7 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   unsigned* err;
+  unsigned long long wait_ns;  // limit of each pipeline wait (drain waits keep kWaitLimitNs)
   int B, L, Hq, Hkv, T, W, a, n;
   float scale_log2;
 };
@@ -66,6 +67,7 @@ struct FwdBar {
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
   uint64_t s_full, s_free, p_ready, pv_done;
   uint64_t drain;
+  uint64_t pair[4];      // exchange barrier of softmax warps w and w + 4 (64 arrivals)
   float xch[2][2][128];  // row-max halves exchanged by the two softmax warpgroups (by tile parity)
   float xl[2][128];      // row-sum halves, exchanged once per item
   uint32_t tmem_base;
@@ -157,6 +159,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     mbar_init(&bar->p_ready, 256);
     mbar_init(&bar->pv_done, 1);
     mbar_init(&bar->drain, 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&bar->pair[s], 64);
     bar->abort_flag = 0;
     fence_barrier_init();
   }
@@ -178,6 +181,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&p.tmKc);
       tma_prefetch_desc(&p.tmVc);
       int g = 0;
+      int kq = 0;  // items whose Q load was issued
       bool ok = true;
       int ge_cur = fwd_item_ge(p, blockIdx.x);
       for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
@@ -185,10 +189,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         if (x + (int)gridDim.x < nitems) ge_cur = fwd_item_ge(p, x + gridDim.x);  // prefetch
         const int kvh = it.h / (p.Hq / p.Hkv);
         const int qb = k & 1;
-        if (k >= 2 && !mbar_wait(&bar->q_empty[qb], ((k - 2) >> 1) & 1, p.err, abort_flag)) {
+        if (k >= 2 &&
+            !mbar_wait(&bar->q_empty[qb], ((k - 2) >> 1) & 1, p.err, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
+        kq = k + 1;
         mbar_arrive_expect_tx(&bar->q_full[qb], C::TILE_BYTES);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_4d(sQ + qb * C::TILE_BYTES + kb * C::BOX_BYTES, &p.tmQ, &bar->q_full[qb],
@@ -199,7 +205,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           const CUtensorMap* mk = win ? &p.tmK : &p.tmKc;
           const CUtensorMap* mv = win ? &p.tmV : &p.tmVc;
           const int row0 = win ? (it.t - j) * C::BN : (j - it.nwin) * C::BN;
-          if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag)) {
+          if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -207,7 +213,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int kb = 0; kb < C::KB; ++kb)
             tma_load_4d(sK + st * C::TILE_BYTES + kb * C::BOX_BYTES, mk, &bar->k_full[st],
                         kb * 64, kvh, row0, it.b);
-          if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag)) {
+          if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag, p.wait_ns)) {
             mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
             ok = false;
             break;
@@ -219,11 +225,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
       }
       if (!ok) {
-        // drain: let every load issued for the last NST tiles and both Q buffers land
+        // drain: let every load issued for the last NST tiles and the last two Q tiles land
+        // (older phases completed already, so their waits return at once)
         for (int gg = max(0, g - NST); gg < g; ++gg) {
           mbar_wait(&bar->k_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
           mbar_wait(&bar->v_full[gg % NST], (gg / NST) & 1, nullptr, nullptr);
         }
+        for (int kk = max(0, kq - 2); kk < kq; ++kk)
+          mbar_wait(&bar->q_full[kk & 1], (kk >> 1) & 1, nullptr, nullptr);
       }
     }
   } else if (warp == 9) {
@@ -238,8 +247,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       int pv_first = 0;    // that tile is the first of its item (overwrite O)
       auto issue_PV = [&](int gg, int first) -> bool {
         const int st = gg % NST;
-        if (!mbar_wait(&bar->p_ready, gg & 1, p.err, abort_flag)) return false;
-        if (!mbar_wait(&bar->v_full[st], (gg / NST) & 1, p.err, abort_flag)) return false;
+        if (!mbar_wait(&bar->p_ready, gg & 1, p.err, abort_flag, p.wait_ns)) return false;
+        if (!mbar_wait(&bar->v_full[st], (gg / NST) & 1, p.err, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
         const uint32_t aP = tmem + C::COL_P;
 #pragma unroll
@@ -257,16 +266,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const FwdItem it = fwd_item_with(p, x, ge_cur);
         if (x + (int)gridDim.x < nitems) ge_cur = fwd_item_ge(p, x + gridDim.x);  // prefetch
         const int qb = k & 1;
-        if (!mbar_wait(&bar->q_full[qb], (k >> 1) & 1, p.err, abort_flag)) {
+        if (!mbar_wait(&bar->q_full[qb], (k >> 1) & 1, p.err, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
         const uint32_t sQb = sQa + qb * C::TILE_BYTES;
         for (int j = 0; j < it.N; ++j, ++g) {
           const int st = g % NST;
-          if (!mbar_wait(&bar->k_full[st], (g / NST) & 1, p.err, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bar->k_full[st], (g / NST) & 1, p.err, abort_flag, p.wait_ns)) {
+            ok = false;
+            break;
+          }
           // S has one buffer: the softmax warps must have loaded S_{g-1}
-          if (g > 0 && !mbar_wait(&bar->s_free, (g - 1) & 1, p.err, abort_flag)) { ok = false; break; }
+          if (g > 0 && !mbar_wait(&bar->s_free, (g - 1) & 1, p.err, abort_flag, p.wait_ns)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -293,7 +308,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       bool ok = true;
       for (int k = 0, x = blockIdx.x; ok && x < nitems; ++k, x += gridDim.x) {
         const FwdItem it = fwd_item_base(p, x);
-        if (!mbar_wait(&bar->o_staged[k & 1], (k >> 1) & 1, p.err, abort_flag)) {
+        if (!mbar_wait(&bar->o_staged[k & 1], (k >> 1) & 1, p.err, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -311,7 +326,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int row = threadIdx.x & 127;  // query row = TMEM lane
     const int wg = threadIdx.x >> 7;    // column half
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t pair_bar = 1 + (warp & 3);  // named barrier of warps w and w + 4 (64 threads)
+    // Warps w and w + 4 (the two halves of the same rows) exchange row statistics through an
+    // mbarrier with a bounded wait, so that when one of them gives up the other cannot block
+    // on the exchange.
+    int xph = 0;  // exchanges done
+    auto pair_sync = [&]() -> bool {
+      mbar_arrive(&bar->pair[warp & 3]);
+      const bool r = mbar_wait(&bar->pair[warp & 3], xph & 1, p.err, abort_flag, p.wait_ns);
+      ++xph;
+      return __all_sync(0xffffffffu, r);
+    };
     const float sl2 = p.scale_log2;
     bool ok = true;
     int g = 0;
@@ -338,7 +362,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           const FwdItem fn = fwd_item_base(p, xn);
           cur = load_tile_raw(p, fn.b, fn.t, fn.t);
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, g & 1, p.err, abort_flag))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full, g & 1, p.err, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -394,7 +418,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const float mh = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         bar->xch[g & 1][wg][row] = mh;
-        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        if (!pair_sync()) {
+          ok = false;
+          break;
+        }
         const float mx = fmaxf(mh, bar->xch[g & 1][wg ^ 1][row]);
         // ---- online max with lazy rescale (only when the max grows by more than 2^8); both
         // halves of a row take the same decision from the same values
@@ -432,7 +459,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                  ((sum4[2].x + sum4[2].y) + (sum4[3].x + sum4[3].y));
         // P and O: the previous tile's P V must be complete (it read P and accumulated O)
         if (g > 0 &&
-            !__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {
+            !__all_sync(0xffffffffu,
+                        mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -460,9 +488,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       // (its own slot: the next item's first row-max exchange may start before the other half
       // has read this value; the next write here is an item later, after further pair barriers)
       bar->xl[wg][row] = l_run;
-      asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+      if (!pair_sync()) {
+        ok = false;
+        break;
+      }
       const float l_tot = l_run + bar->xl[wg ^ 1][row];
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag))) {
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag, p.wait_ns))) {
         ok = false;
         break;
       }
@@ -585,6 +617,7 @@ cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.o = static_cast<__nv_bfloat16*>(o);
   prm.lse = lse;
   prm.err = device_error_word();
+  prm.wait_ns = pipeline_wait_limit_ns();
   prm.B = s.B;
   prm.L = s.L;
   prm.Hq = s.Hq;

@@ -1,5 +1,5 @@
-// SepCache streaming decode on sm_100a: cache update (append / compress) and single-query
-// attention with positional-encoding shifting.
+// SepCache streaming decode on sm_100a: cache update (append / compress), prefill from a prompt
+// and single-query attention with positional-encoding shifting.
 //
 // Cache blocks ("How SepLLM reorchestrates the language model...", beiduofen.top, section
 // "SepLLM's Architecture: Composing Efficiency"): a initial slots, a separator FIFO of s slots,
@@ -9,19 +9,30 @@
 // the Past Window, which is compressed (its separators to the FIFO, the rest dropped) by the
 // step that makes the total usage reach c. The separator FIFO drops its oldest entries when
 // full. Positions are ranks inside the cache (SepLLM project card, "Limitations & Caveats":
-// streaming needs positional-encoding shifting), so a key is rotated by RoPE(rank) at every
-// step and the query by RoPE(occupied - 1).
+// streaming needs positional-encoding shifting): the key of rank p is seen at RoPE(p) and the
+// query at RoPE(occupied - 1).
 //
 // Slot storage per (sequence, KV head) is [n][d], n = a + s + P + w: initial slots, the
 // separator ring, the past window (a plain array, emptied by each compression), the window
-// ring. Keys are stored without rotation.
+// ring.
 //
-// Decode: one CTA per (sequence, KV head), all of them resident at once (4 per SM), so the
-// whole cache streams in a single wave. Each CTA streams its ranks through a shared-memory ring
-// filled by bulk copies, with 8 half-warps (one key per half-warp per step, the row spread over
-// 16 lanes), rotates keys in registers (cos/sin advanced by a complex recurrence from the table
-// row of the first rank), keeps an online softmax per query head, and combines its half-warps
-// through shared memory. No global scratch is used.
+// Rotation storage. Inside each block the rank of a key is its own counter plus one offset that
+// the whole block shares: initial, past-window and window keys hold consecutive original
+// positions t, and the separators in the FIFO hold consecutive admission indices A (the A-th
+// separator ever admitted; the FIFO keeps the newest, oldest first). So every key is stored
+// rotated once by RoPE(counter), counter = t or A, and since RoPE(m)q . RoPE(p)k =
+// RoPE(m - p + u)q . RoPE(u)k, the query is rotated once per block by RoPE(m - offset) instead of
+// rotating every key at every step. A key is rotated by RoPE(t) when it is appended and, when it
+// enters the separator FIFO, re-rotated by RoPE(A - t). Without positional shifting
+// (original_positions) keys stay at RoPE(t) and every block's query angle is its own position.
+// Angles are formed in fp64 (position x inverse frequency), rotations are rounded once to bf16.
+//
+// Decode: one CTA per (sequence, KV head), all resident in one wave. Bulk copies stream the
+// retained K/V rows in rank order through a shared-memory ring; a group of D/8 lanes takes one
+// key row (8 contiguous elements per lane, one 16-byte load of K and one of V), forms the
+// partial dot products with the block's rotated queries, reduces them across the group so that
+// each lane is left the score of one query, keeps that query's online softmax, and accumulates
+// the V rows of every query. Groups are combined through shared memory. No global scratch.
 #include <cuda_runtime.h>
 
 #include "sep_common.cuh"
@@ -29,50 +40,28 @@
 
 namespace sep {
 
-constexpr int kDecThreads = 128;   // 8 half-warps per CTA; one CTA per (sequence, KV head)
-constexpr int kHalfWarps = kDecThreads / 16;
-
-// ------------------------------------------------------------------ init
-__global__ void sepcache_init_kernel(int S, int c, int d, double theta, int32_t* meta,
-                                     int32_t* slot_pos, uint8_t* slot_sep, float* rope_cs) {
-  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
-  const int nthr = gridDim.x * blockDim.x;
-  for (int e = tid; e < S * SEPCACHE_META; e += nthr) meta[e] = 0;
-  for (int e = tid; e < S * c; e += nthr) {
-    slot_pos[e] = -1;
-    slot_sep[e] = 0;
-  }
-  const int h = d / 2;
-  for (int e = tid; e < c * h; e += nthr) {
-    const int p = e / h, k = e % h;
-    const double ang = (double)p * pow(theta, -2.0 * (double)k / (double)d);
-    double sn, cs;
-    sincos(ang, &sn, &cs);
-    rope_cs[2 * e] = (float)cs;
-    rope_cs[2 * e + 1] = (float)sn;
-  }
-}
-
-// Key rotation for a cache without positional shifting: the 16-byte chunks x (dims k0..k0+7)
-// and y (dims k0+d/2..k0+d/2+7) of one key row rotated at original position pos, the angle of
-// pair k being pos * theta^(-2k/d) as in the cos/sin table; fp64 arithmetic, rounded to bf16.
-__device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, int pos, int d,
-                                                   double theta) {
+// ------------------------------------------------------------------ RoPE of stored keys
+// Rotate-half pairs (k, k + d/2), angle pos * freq[k], freq[k] = theta^(-2k/d) (fp64 table).
+// x holds dims k0..k0+7, y dims k0+d/2..k0+d/2+7 of one key row; fp64 arithmetic with the
+// operations spelled out (no contraction choices left to the compiler), rounded to bf16, so that
+// every kernel that rotates the same row by the same angle produces the same bits.
+__device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, long long pos,
+                                                   const double* __restrict__ freq) {
+  if (pos == 0) return;
   uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&xs[q]);
     const __nv_bfloat162 ya = *reinterpret_cast<const __nv_bfloat162*>(&ys[q]);
-    double xv[2] = {(double)__low2float(xa), (double)__high2float(xa)};
-    double yv[2] = {(double)__low2float(ya), (double)__high2float(ya)};
+    const double xv[2] = {(double)__low2float(xa), (double)__high2float(xa)};
+    const double yv[2] = {(double)__low2float(ya), (double)__high2float(ya)};
     __nv_bfloat16 xo[2], yo[2];
 #pragma unroll
     for (int z = 0; z < 2; ++z) {
-      const int k = k0 + 2 * q + z;
       double sn, cs;
-      sincos((double)pos * pow(theta, -2.0 * (double)k / (double)d), &sn, &cs);
-      xo[z] = __double2bfloat16(xv[z] * cs - yv[z] * sn);
-      yo[z] = __double2bfloat16(yv[z] * cs + xv[z] * sn);
+      sincos(__dmul_rn((double)pos, __ldg(freq + k0 + 2 * q + z)), &sn, &cs);
+      xo[z] = __double2bfloat16(__fma_rn(xv[z], cs, -__dmul_rn(yv[z], sn)));
+      yo[z] = __double2bfloat16(__fma_rn(yv[z], cs, __dmul_rn(xv[z], sn)));
     }
     const __nv_bfloat162 xp = __halves2bfloat162(xo[0], xo[1]);
     const __nv_bfloat162 yp = __halves2bfloat162(yo[0], yo[1]);
@@ -83,45 +72,65 @@ __device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, i
   y = make_uint4(ys[0], ys[1], ys[2], ys[3]);
 }
 
+// ------------------------------------------------------------------ init
+__global__ void sepcache_init_kernel(int S, int c, int d, double theta, int32_t* meta,
+                                     int32_t* slot_pos, uint8_t* slot_sep, double* freq) {
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int nthr = gridDim.x * blockDim.x;
+  for (int e = tid; e < S * SEPCACHE_META; e += nthr) meta[e] = 0;
+  for (int e = tid; e < S * c; e += nthr) {
+    slot_pos[e] = -1;
+    slot_sep[e] = 0;
+  }
+  for (int k = tid; k < d / 2; k += nthr) freq[k] = pow(theta, -2.0 * (double)k / (double)d);
+}
+
 // ------------------------------------------------------------------ update
 // One CTA per sequence. Thread 0 plans the step, all threads copy rows (16-byte vectors). With a
 // Past Window (P > 0) the step that makes the usage reach c then compresses it: a block-wide
 // scan numbers the past window's separators k = 0, 1, ... (oldest first); the FIFO keeps the
 // last s of its current entries followed by them, so separator k lands at ring index
-// (sep_head + sep_cnt + k) mod s and is kept when it is among the last s (k >= nnew - s).
+// (sep_head + sep_cnt + k) mod s, gets admission index admit + k, and is kept when it is among
+// the last s (k >= nnew - s).
 constexpr int kUpdateThreads = 128;
 
+struct CacheDims {
+  int Hkv, d, a, s, w, P, c, orig;
+};
+
 __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
-    int Hkv, int d, int a, int s, int w, int P, int c, int orig, double theta,
-    uint4* __restrict__ k_slots,
+    CacheDims cd, const double* __restrict__ freq, uint4* __restrict__ k_slots,
     uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
     int32_t* __restrict__ meta, const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
     const uint8_t* __restrict__ sep_new) {
   extern __shared__ int2 s_moves[];  // compression: (past slot, separator slot), min(s, P) at most
+  const int Hkv = cd.Hkv, d = cd.d, a = cd.a, s = cd.s, w = cd.w, P = cd.P;
   const int seq = blockIdx.x;
-  const int ns = a + s + P + w;       // slots per sequence
+  const int ns = a + s + P + w;  // slots per sequence
   const int win_base = a + s + P;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* m = meta + (size_t)seq * SEPCACHE_META;
-  // slot_new, move_from, move_to, t, compress, past_cnt, sep_head, sep_cnt
-  __shared__ int plan[8];
+  // slot_new, move_from, move_to, t, compress, past_cnt, sep_head, sep_cnt, move_angle, admit
+  __shared__ int plan[10];
   __shared__ int s_warp[kUpdateThreads / 32];
-  // the metadata and the flag of the window's oldest slot, loaded in parallel
+  // the metadata and the window's oldest slot (flag, position), loaded in parallel
   __shared__ int s_meta[SEPCACHE_META];
-  __shared__ int s_oldsep;
+  __shared__ int s_oldsep, s_oldpos;
   if (tid < SEPCACHE_META) s_meta[tid] = m[tid];
   if (tid == 32) {
     const int wh = m[SEPCACHE_META_WIN_HEAD];
     s_oldsep = slot_sep[(size_t)seq * ns + win_base + wh];
+    s_oldpos = slot_pos[(size_t)seq * ns + win_base + wh];
   }
   __syncthreads();
   if (tid == 0) {
     const int t = s_meta[SEPCACHE_META_T];
-    int slot_new, move_from = -1, move_to = -1;
+    int slot_new, move_from = -1, move_to = -1, move_angle = 0;
     int ninit = s_meta[SEPCACHE_META_NINIT];
     int sep_head = s_meta[SEPCACHE_META_SEP_HEAD], sep_cnt = s_meta[SEPCACHE_META_SEP_CNT];
     int win_head = s_meta[SEPCACHE_META_WIN_HEAD], win_cnt = s_meta[SEPCACHE_META_WIN_CNT];
     int past_cnt = (P > 0) ? s_meta[SEPCACHE_META_PAST_CNT] : 0;
+    int admit = s_meta[SEPCACHE_META_SEP_ADMIT];
     if (t < a) {
       slot_new = t;
       ninit = t + 1;
@@ -144,11 +153,14 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
           sep_head = (sep_head + 1) % s;
         }
         move_from = old_slot;
+        // stored at RoPE(t_old); in the FIFO it is seen at RoPE(admission index)
+        move_angle = cd.orig ? 0 : admit - s_oldpos;
+        ++admit;
       }
       slot_new = old_slot;
       win_head = (win_head + 1) % w;
     }
-    const bool compress = P > 0 && ninit + sep_cnt + past_cnt + win_cnt >= c;
+    const bool compress = P > 0 && ninit + sep_cnt + past_cnt + win_cnt >= cd.c;
     m[SEPCACHE_META_T] = t + 1;
     m[SEPCACHE_META_NINIT] = ninit;
     m[SEPCACHE_META_SEP_HEAD] = sep_head;
@@ -156,6 +168,7 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
     m[SEPCACHE_META_WIN_HEAD] = win_head;
     m[SEPCACHE_META_WIN_CNT] = win_cnt;
     if (P > 0) m[SEPCACHE_META_PAST_CNT] = past_cnt;
+    m[SEPCACHE_META_SEP_ADMIT] = admit;
     plan[0] = slot_new;
     plan[1] = move_from;
     plan[2] = move_to;
@@ -164,35 +177,46 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
     plan[5] = past_cnt;
     plan[6] = sep_head;
     plan[7] = sep_cnt;
+    plan[8] = move_angle;
+    plan[9] = admit;
   }
   __syncthreads();
   const int slot_new = plan[0], move_from = plan[1], move_to = plan[2], t = plan[3];
   const int vec = d / 8;  // 16-byte vectors per row
+  const int hv = vec / 2; // vectors per RoPE half
   const size_t seq_rows = (size_t)seq * Hkv * ns;
-  auto copy_row = [&](int from, int to) {  // all heads, all threads
-    for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
-      const int hh = e / vec, q = e % vec;
+  // move a row (all heads, all threads): V copied, K re-rotated by `angle` on the way
+  auto move_row = [&](int from, int to, int angle) {
+    for (int e = tid; e < Hkv * hv; e += kUpdateThreads) {
+      const int hh = e / hv, q = e % hv;
       const size_t src = (seq_rows + (size_t)hh * ns + from) * vec + q;
       const size_t dst = (seq_rows + (size_t)hh * ns + to) * vec + q;
-      k_slots[dst] = k_slots[src];
-      v_slots[dst] = v_slots[src];
+      uint4 x = k_slots[src], y = k_slots[src + hv];
+      rope_rotate_chunks(x, y, 8 * q, angle, freq);
+      k_slots[dst] = x;
+      k_slots[dst + hv] = y;
+    }
+    for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
+      const int hh = e / vec, q = e % vec;
+      v_slots[(seq_rows + (size_t)hh * ns + to) * vec + q] =
+          v_slots[(seq_rows + (size_t)hh * ns + from) * vec + q];
     }
   };
   if (move_from >= 0) {
-    copy_row(move_from, move_to);
+    move_row(move_from, move_to, plan[8]);
     if (tid == 0) {
       slot_pos[(size_t)seq * ns + move_to] = slot_pos[(size_t)seq * ns + move_from];
       slot_sep[(size_t)seq * ns + move_to] = slot_sep[(size_t)seq * ns + move_from];
     }
     __syncthreads();
   }
-  const int hv = vec / 2;  // chunks per RoPE half
-  for (int e = tid; e < Hkv * hv; e += kUpdateThreads) {  // K: chunk q and its partner q + hv
+  // the new token: K rotated at its original position t
+  for (int e = tid; e < Hkv * hv; e += kUpdateThreads) {
     const int hh = e / hv, q = e % hv;
     const size_t dst = (seq_rows + (size_t)hh * ns + slot_new) * vec + q;
     const size_t src = ((size_t)seq * Hkv + hh) * vec + q;
     uint4 x = k_new[src], y = k_new[src + hv];
-    if (orig) rope_rotate_chunks(x, y, 8 * q, t, d, theta);
+    rope_rotate_chunks(x, y, 8 * q, t, freq);
     k_slots[dst] = x;
     k_slots[dst + hv] = y;
   }
@@ -208,7 +232,7 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
 
   // ---- compression of the past window [a + s, a + s + past_cnt)
   __syncthreads();
-  const int past_cnt = plan[5], sep_head = plan[6], sep_cnt = plan[7];
+  const int past_cnt = plan[5], sep_head = plan[6], sep_cnt = plan[7], admit = plan[9];
   const uint8_t* pflag = slot_sep + (size_t)seq * ns + a + s;
   int cnt = 0;
   for (int i = tid; i < past_cnt; i += kUpdateThreads) cnt += pflag[i] != 0;
@@ -242,9 +266,11 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
   const int nkept = nnew - kfirst;
   for (int j = 0; j < nkept; ++j) {
     const int2 mv = s_moves[j];
-    copy_row(mv.x, mv.y);
+    const int tp = slot_pos[(size_t)seq * ns + mv.x];
+    // admission index of new separator k = kfirst + j is admit + k
+    move_row(mv.x, mv.y, cd.orig ? 0 : admit + kfirst + j - tp);
     if (tid == 0) {
-      slot_pos[(size_t)seq * ns + mv.y] = slot_pos[(size_t)seq * ns + mv.x];
+      slot_pos[(size_t)seq * ns + mv.y] = tp;
       slot_sep[(size_t)seq * ns + mv.y] = 1;
     }
   }
@@ -260,67 +286,95 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
       m[SEPCACHE_META_SEP_CNT] = min(total, s);
     }
     m[SEPCACHE_META_PAST_CNT] = 0;
+    m[SEPCACHE_META_SEP_ADMIT] = admit + nnew;
   }
 }
 
 // ------------------------------------------------------------------ prefill
 // State after appending the L prompt tokens of every sequence one at a time to an empty cache,
-// in one pass (the same rule as sepcache_update, solved in closed form):
+// in one pass (the rule of sepcache_update solved in closed form):
 //   initial slots 0..min(a, L)-1 hold tokens 0..min(a, L)-1;
-//   the window ring holds the last min(w, L - a) tokens, token u at ring index (u - a) mod w,
-//   its head at (L - a) mod w once the ring has wrapped;
-//   the tokens u in [a, L - w) have left the window; the k-th separator among them (k = 0,
-//   1, ...) went to separator ring index k mod s, so the ring keeps the last min(s, count) of
-//   them, its head at count mod s once full (nothing is kept when s = 0).
-// One CTA per (sequence, KV head): each scans the flags (block-wide exclusive scan) to place the
-// kept separators, copies its head's K/V rows, and the head-0 CTA writes the metadata and the
-// slot maps. K/V rows of unused slots are left as they are.
+//   the window ring holds the last nwin = min(w, L - a) tokens, token u at ring index
+//   (u - a) mod w, its head at (L - a) mod w once the ring has wrapped;
+//   tokens u in [a, e_end) were compressed: the A-th separator among them (A = 0, 1, ...) was
+//   admitted to the FIFO at ring index A mod s, so the ring keeps the last min(s, count) of
+//   them, its head at (count - kept) mod s;
+//   with c = 0, e_end = L - nwin (every token that left the window was compressed at once) and
+//   the past window is empty; with c > 0 the past window is compressed in runs: after the
+//   window is full every step moves one token into it, and a run of need = c - a - w - sep_cnt
+//   tokens triggers a compression, so run boundaries follow the recurrence
+//   e <- e + need(sep_cnt), sep_cnt <- min(s, sep_cnt + separators in the run), as long as a
+//   run has left the window entirely; tokens [e_end, L - nwin) are the past window.
+// One CTA per (sequence, KV head): each finds e_end and the separator count (block-wide counts),
+// scans the flags to place the kept separators, copies and rotates its head's K/V rows; the
+// head-0 CTA writes the metadata and the slot maps. K/V rows of unused slots are left as they
+// are. Keys get exactly the rotations the single-token updates give them: RoPE(t) on entry
+// and, for separators with shifting, RoPE(A - t) on admission.
 constexpr int kPrefillThreads = 256;
 constexpr int kPrefillItems = 16;
 
+__device__ __forceinline__ int block_count_flags(const uint8_t* flags, int lo, int hi,
+                                                 int* s_warp) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int cnt = 0;
+  for (int u = lo + tid; u < hi; u += kPrefillThreads) cnt += flags[u] != 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o);
+  __syncthreads();  // s_warp free (an earlier call may still be reading it)
+  if (lane == 0) s_warp[warp] = cnt;
+  __syncthreads();
+  int tot = 0;
+  for (int x = 0; x < kPrefillThreads / 32; ++x) tot += s_warp[x];
+  return tot;
+}
+
 __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
-    int L, int Hkv, int d, int a, int s, int w, int orig, double theta,
-    const uint4* __restrict__ k_in,
+    int L, CacheDims cd, const double* __restrict__ freq, const uint4* __restrict__ k_in,
     const uint4* __restrict__ v_in, const uint8_t* __restrict__ sep_in, uint4* __restrict__ k_slots,
     uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
     int32_t* __restrict__ meta) {
   extern __shared__ int s_seppos[];  // [s]: position of the separator at each ring index
   __shared__ int s_warp[kPrefillThreads / 32];
-  __shared__ int s_total;
+  const int Hkv = cd.Hkv, d = cd.d, a = cd.a, s = cd.s, w = cd.w, P = cd.P;
   const int seq = blockIdx.x, head = blockIdx.y;
-  const int c = a + s + w;
+  const int ns = a + s + P + w;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint8_t* flags = sep_in + (size_t)seq * L;
   const int ninit = min(a, L);
   const int nwin = max(0, min(w, L - a));
-  const int left_end = max(a, L - w);  // tokens in [a, left_end) have left the window
+  const int win_first = L - nwin;  // oldest token in the window (>= a)
 
-  // ---- pass 1: how many separators left the window
-  int cnt = 0;
-  for (int u = a + tid; u < left_end; u += kPrefillThreads) cnt += flags[u] != 0;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_down_sync(0xffffffffu, cnt, o);
-  if (lane == 0) s_warp[warp] = cnt;
-  __syncthreads();
-  if (tid == 0) {
-    int tot = 0;
-    for (int x = 0; x < kPrefillThreads / 32; ++x) tot += s_warp[x];
-    s_total = tot;
+  // ---- compressed range [a, e_end) and the number of separators admitted from it
+  int e_end, count;
+  if (P == 0) {
+    e_end = max(a, win_first);
+    count = (s > 0) ? block_count_flags(flags, a, e_end, s_warp) : 0;
+  } else {
+    e_end = a;
+    count = 0;
+    int kept = 0;
+    for (;;) {
+      const int need = cd.c - a - w - kept;  // >= 1 since c > a + s + w
+      if (nwin < w || e_end + need > win_first) break;  // the run has not left the window
+      const int nsep = block_count_flags(flags, e_end, e_end + need, s_warp);
+      count += nsep;
+      kept = min(s, kept + nsep);
+      e_end += need;
+    }
   }
-  __syncthreads();
-  const int count = (s > 0) ? s_total : 0;
   const int sep_cnt = min(s, count);
   const int first_kept = count - sep_cnt;
+  const int past_cnt = (P > 0) ? max(0, win_first - e_end) : 0;
 
-  // ---- pass 2: exclusive scan; the kept separators record their positions by ring index
+  // ---- exclusive scan over [a, e_end); the kept separators record their positions by ring index
   if (sep_cnt > 0) {
     int carry = 0;
-    for (int base = a; base < left_end; base += kPrefillThreads * kPrefillItems) {
+    for (int base = a; base < e_end; base += kPrefillThreads * kPrefillItems) {
       const int u0 = base + tid * kPrefillItems;
       uint32_t bits = 0;
 #pragma unroll
       for (int q = 0; q < kPrefillItems; ++q)
-        if (u0 + q < left_end && flags[u0 + q] != 0) bits |= 1u << q;
+        if (u0 + q < e_end && flags[u0 + q] != 0) bits |= 1u << q;
       const int n = __popc(bits);
       int incl = n;
 #pragma unroll
@@ -348,50 +402,62 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
   }
   __syncthreads();
 
-  // slot -> original position (-1: unused)
-  auto pos_of = [&](int slot) -> int {
+  // slot -> original position (-1: unused); for separator slots also the admission index
+  auto pos_of = [&](int slot, int* admit_idx) -> int {
     if (slot < a) return slot < ninit ? slot : -1;
     if (slot < a + s) {
       const int r = slot - a;
-      return (count >= s || r < count) ? s_seppos[r] : -1;
+      if (!(count >= s || r < count)) return -1;
+      // kept admission indices are first_kept..count-1, one per residue mod s
+      *admit_idx = first_kept + (((r - first_kept) % s) + s) % s;
+      return s_seppos[r];
     }
-    const int r = slot - a - s;
+    if (slot < a + s + P) {
+      const int r = slot - a - s;
+      return r < past_cnt ? e_end + r : -1;
+    }
+    const int r = slot - a - s - P;
     if (nwin == w || r < nwin) {
-      const int first = L - nwin;  // oldest token in the window
-      const int r0 = (first - a) % w;
-      return first + (r - r0 + w) % w;
+      const int r0 = (win_first - a) % w;
+      return win_first + (r - r0 + w) % w;
     }
     return -1;
   };
 
   // ---- metadata and slot maps (once per sequence)
   if (head == 0) {
-    for (int slot = tid; slot < c; slot += kPrefillThreads) {
-      const int pos = pos_of(slot);
-      slot_pos[(size_t)seq * c + slot] = pos;
-      slot_sep[(size_t)seq * c + slot] = (pos >= 0 && flags[pos] != 0) ? 1 : 0;
+    for (int slot = tid; slot < ns; slot += kPrefillThreads) {
+      int A = 0;
+      const int pos = pos_of(slot, &A);
+      slot_pos[(size_t)seq * ns + slot] = pos;
+      slot_sep[(size_t)seq * ns + slot] = (pos >= 0 && flags[pos] != 0) ? 1 : 0;
     }
     if (tid == 0) {
       int32_t* m = meta + (size_t)seq * SEPCACHE_META;
       m[SEPCACHE_META_T] = L;
       m[SEPCACHE_META_NINIT] = ninit;
-      m[SEPCACHE_META_SEP_HEAD] = (count >= s && s > 0) ? count % s : 0;
+      m[SEPCACHE_META_SEP_HEAD] = (s > 0) ? first_kept % s : 0;
       m[SEPCACHE_META_SEP_CNT] = sep_cnt;
       m[SEPCACHE_META_WIN_HEAD] = (L - a >= w) ? (L - a) % w : 0;
       m[SEPCACHE_META_WIN_CNT] = nwin;
+      m[SEPCACHE_META_PAST_CNT] = past_cnt;
+      m[SEPCACHE_META_SEP_ADMIT] = count;
     }
   }
   // ---- this head's K/V rows of the occupied slots (one warp per row, 16-byte vectors)
   const int vec = d / 8;
-  const size_t dst_base = ((size_t)seq * Hkv + head) * c;
-  for (int slot = warp; slot < c; slot += kPrefillThreads / 32) {
-    const int pos = pos_of(slot);
+  const size_t dst_base = ((size_t)seq * Hkv + head) * ns;
+  for (int slot = warp; slot < ns; slot += kPrefillThreads / 32) {
+    int A = 0;
+    const int pos = pos_of(slot, &A);
     if (pos < 0) continue;
+    const bool is_sep_slot = slot >= a && slot < a + s;
     const size_t src = (((size_t)seq * L + pos) * Hkv + head) * vec;
     const size_t dst = (dst_base + slot) * vec;
     for (int e = lane; e < vec / 2; e += 32) {  // K: chunk e and its RoPE partner
       uint4 x = __ldg(k_in + src + e), y = __ldg(k_in + src + e + vec / 2);
-      if (orig) rope_rotate_chunks(x, y, 8 * e, pos, d, theta);
+      rope_rotate_chunks(x, y, 8 * e, pos, freq);
+      if (is_sep_slot && !cd.orig) rope_rotate_chunks(x, y, 8 * e, (long long)A - pos, freq);
       k_slots[dst + e] = x;
       k_slots[dst + e + vec / 2] = y;
     }
@@ -399,22 +465,372 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
   }
 }
 
-cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, const void* v,
-                                    const uint8_t* sep, int L, cudaStream_t stream) {
-  const size_t smem = (size_t)max(st.s, 1) * sizeof(int);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(sepcache_prefill_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  sepcache_prefill_kernel<<<dim3(st.S, st.Hkv), kPrefillThreads, smem, stream>>>(
-      L, st.Hkv, st.d, st.a, st.s, st.w, st.original_positions, (double)st.rope_theta,
-      static_cast<const uint4*>(k),
-      static_cast<const uint4*>(v), sep, reinterpret_cast<uint4*>(st.k_slots),
-      reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta);
-  return cudaGetLastError();
+// ------------------------------------------------------------------ decode
+// Lane groups: LPK = D / 8 lanes per key row, 8 contiguous elements per lane; NG = 128 / LPK
+// groups per CTA, each taking two rows of every KC = 2 NG row chunk.
+constexpr int kDecThreads = 128;
+constexpr int kDecStages = 4;
+constexpr int kDecWarps = kDecThreads / 32;
+
+template <int N>
+__host__ __device__ constexpr int ilog2() {
+  return N >= 32 ? 5 : N >= 16 ? 4 : N >= 8 ? 3 : N >= 4 ? 2 : N >= 2 ? 1 : 0;
 }
 
+// Reduction over the LPK lanes of a group of GP per-query partial sums: the first log2(GP)
+// butterfly levels halve what a lane holds (it keeps one half, adding its partner's copy of it,
+// and sends the other half); the remaining levels sum one value. Afterwards lane l of the group
+// holds the full score of query own_query(l).
+template <int GP, int LPK>
+__device__ __forceinline__ float group_reduce_own(float (&v)[GP], int l) {
+  constexpr int LG = ilog2<GP>(), LL = ilog2<LPK>();
+  static_assert((1 << LG) == GP && (1 << LL) == LPK && GP <= LPK, "group shape");
+#pragma unroll
+  for (int lv = 0; lv < LG; ++lv) {
+    const int off = LPK >> (lv + 1), h = (GP >> lv) >> 1;
+    const bool upper = (l & off) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h];
+      const float keep = upper ? v[i + h] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float r = v[0];
+#pragma unroll
+  for (int lv = LG; lv < LL; ++lv) r += __shfl_xor_sync(0xffffffffu, r, LPK >> (lv + 1));
+  return r;
+}
+template <int GP, int LPK>
+__device__ __forceinline__ int own_query(int l) {
+  int g = 0;
+#pragma unroll
+  for (int lv = 0; lv < ilog2<GP>(); ++lv)
+    if (l & (LPK >> (lv + 1))) g += GP >> (lv + 1);
+  return g;
+}
+template <int GP, int LPK>
+__device__ __forceinline__ int lane_of_query(int g) {
+  int src = 0;
+#pragma unroll
+  for (int lv = 0; lv < ilog2<GP>(); ++lv)
+    if (g & (GP >> (lv + 1))) src |= LPK >> (lv + 1);
+  return src;
+}
+
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+template <int D, int GP>
+struct DecCfg {
+  static constexpr int LPK = D / 8;
+  static constexpr int NG = kDecThreads / LPK;
+  static constexpr int KC = 2 * NG;  // rows per ring stage
+  static constexpr int RING_BYTES = kDecStages * KC * D * 2 * 2;
+  static constexpr int COMB_BYTES = kDecWarps * GP * D * 4;  // per-warp V sums at the end
+  static constexpr int BUF_BYTES = RING_BYTES > COMB_BYTES ? RING_BYTES : COMB_BYTES;
+};
+
+template <int D, int GP>
+struct DecSmem {
+  alignas(128) uint8_t buf[DecCfg<D, GP>::BUF_BYTES];  // K/V ring, later the combine buffer
+  alignas(16) float qrot[3][GP][D];  // the queries rotated for each block, x scale*log2(e)
+  uint64_t full[kDecStages];
+  int done[kDecStages];  // warps finished with the stage's current chunk
+  int issued;            // chunks whose copies were issued (0..issued-1)
+  float wm[kDecWarps][GP], wl[kDecWarps][GP];
+  int abort_flag;
+};
+
+struct DecodeArgs {
+  int Hq, Hkv, G, a, s, P, w;
+  const __nv_bfloat16* k_slots;
+  const __nv_bfloat16* v_slots;
+  const int32_t* meta;
+  const double* freq;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* o;
+  float* lse;
+  float scale_log2;
+  unsigned* err;
+};
+
+template <int D, int GP, bool ORIG>
+__global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
+    sepcache_decode_kernel(const __grid_constant__ DecodeArgs p) {
+  using C = DecCfg<D, GP>;
+  constexpr int LPK = C::LPK, NG = C::NG, KC = C::KC;
+  constexpr int HALF = D / 2;
+  const int kvh = blockIdx.x, seq = blockIdx.y;
+  const int ns = p.a + p.s + p.P + p.w;
+  const int tid = threadIdx.x, warp = tid >> 5, grp = tid / LPK, l = tid % LPK;
+  extern __shared__ __align__(128) uint8_t dsm_raw[];
+  DecSmem<D, GP>& sm = *reinterpret_cast<DecSmem<D, GP>*>(dsm_raw);
+  __nv_bfloat16* ring = reinterpret_cast<__nv_bfloat16*>(sm.buf);
+  auto ring_k = [&](int st, int row) { return ring + ((size_t)(st * 2 + 0) * KC + row) * D; };
+  auto ring_v = [&](int st, int row) { return ring + ((size_t)(st * 2 + 1) * KC + row) * D; };
+
+  const int32_t* m = p.meta + (size_t)seq * SEPCACHE_META;
+  const int T = m[SEPCACHE_META_T];
+  const int ninit = m[SEPCACHE_META_NINIT];
+  const int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
+  const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
+  const int past_cnt = (p.P > 0) ? m[SEPCACHE_META_PAST_CNT] : 0;
+  const int admit = m[SEPCACHE_META_SEP_ADMIT];
+  const int occ = ninit + sep_cnt + past_cnt + win_cnt;
+  const int mq = occ - 1;  // the query's own rank
+  const int nchunks = (occ + KC - 1) / KC;
+  const size_t row_base = ((size_t)seq * p.Hkv + kvh) * ns;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  auto issue_chunk = [&](int ch) {  // one thread: bulk copies of chunk ch into its stage
+    const int st = ch % kDecStages;
+    const int c0 = ch * KC;
+    const int rows = min(KC, occ - c0);
+    mbar_arrive_expect_tx(&sm.full[st], (uint32_t)(rows * D * 2 * 2));
+    // ranks map to slots piecewise contiguously: initial block, the separator ring, the past
+    // window, the window ring; a run ends at a block boundary or a ring wrap
+    int r = c0;
+    const int end = c0 + rows;
+    while (r < end) {
+      int slot, len;
+      if (r < ninit) {
+        slot = r;
+        len = min(end, ninit) - r;
+      } else if (r < ninit + sep_cnt) {
+        const int x = (sep_head + (r - ninit)) % p.s;
+        slot = p.a + x;
+        len = min(min(end, ninit + sep_cnt) - r, p.s - x);
+      } else if (r < ninit + sep_cnt + past_cnt) {
+        slot = p.a + p.s + (r - ninit - sep_cnt);
+        len = min(end, ninit + sep_cnt + past_cnt) - r;
+      } else {
+        const int x = (win_head + (r - ninit - sep_cnt - past_cnt)) % p.w;
+        slot = p.a + p.s + p.P + x;
+        len = min(end - r, p.w - x);
+      }
+      const size_t src = (row_base + slot) * D;
+      bulk_load(ring_k(st, r - c0), p.k_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
+      bulk_load(ring_v(st, r - c0), p.v_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
+      r += len;
+    }
+    atomicMax(&sm.issued, ch + 1);  // warps may refill different stages at the same time
+  };
+  if (tid == 0) {
+    for (int st = 0; st < kDecStages; ++st) {
+      mbar_init(&sm.full[st], 1);
+      sm.done[st] = 0;
+    }
+    sm.abort_flag = 0;
+    sm.issued = 0;
+    fence_barrier_init();
+    for (int ch = 0; ch < min(kDecStages, nchunks); ++ch) issue_chunk(ch);
+  }
+
+  // ---- the G queries of this KV head rotated once per block (while the first chunks load):
+  // block 0 = initial keys (stored at RoPE(rank)), 1 = separators (stored at RoPE(admission
+  // index), rank = ninit + index - oldest index), 2 = past window and window (stored at
+  // RoPE(original position), query at T - 1). Without shifting every block uses T - 1.
+  {
+    long long qpos[3];
+    qpos[0] = ORIG ? (long long)T - 1 : (long long)mq;
+    qpos[1] = ORIG ? (long long)T - 1 : (long long)mq - ninit + (admit - sep_cnt);
+    qpos[2] = (long long)T - 1;
+    for (int e = tid; e < 3 * HALF; e += kDecThreads) {
+      const int blk = e / HALF, k = e % HALF;
+      double sn, cs;
+      sincos(__dmul_rn((double)qpos[blk], __ldg(p.freq + k)), &sn, &cs);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float r1 = 0.f, r2 = 0.f;
+        if (g < p.G) {
+          const __nv_bfloat16* qh = p.q + ((size_t)seq * p.Hq + kvh * p.G + g) * D;
+          const double x1 = (double)__bfloat162float(qh[k]);
+          const double x2 = (double)__bfloat162float(qh[k + HALF]);
+          r1 = (float)(x1 * cs - x2 * sn) * p.scale_log2;
+          r2 = (float)(x2 * cs + x1 * sn) * p.scale_log2;
+        }
+        sm.qrot[blk][g][k] = r1;
+        sm.qrot[blk][g][k + HALF] = r2;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- consumers: group grp takes rows grp and grp + NG of every chunk
+  float2 qr[GP][4];   // this lane's 8 query elements (as pairs) of the current block
+  float2 acc[GP][4];  // V sums of every query over this lane's 8 elements
+  float m_own = -INFINITY, l_own = 0.f;  // softmax state of this lane's own query
+  int cur_blk = -1;
+#pragma unroll
+  for (int g = 0; g < GP; ++g)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[g][i] = make_float2(0.f, 0.f);
+
+  bool ok = true;
+  for (int ch = 0; ch < nchunks && ok; ++ch) {
+    const int st = ch % kDecStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[st], (ch / kDecStages) & 1, p.err, abort_flag))) {
+      ok = false;
+      break;
+    }
+    const int c0 = ch * KC;
+#pragma unroll
+    for (int sub = 0; sub < 2; ++sub) {
+      const int row = sub * NG + grp;
+      const int r = c0 + row;
+      const bool valid = r < occ;
+      const int blk = (r < ninit) ? 0 : (r < ninit + sep_cnt) ? 1 : 2;
+      if (blk != cur_blk) {
+        cur_blk = blk;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float4 a0 = *reinterpret_cast<const float4*>(&sm.qrot[blk][g][l * 8]);
+          const float4 a1 = *reinterpret_cast<const float4*>(&sm.qrot[blk][g][l * 8 + 4]);
+          qr[g][0] = make_float2(a0.x, a0.y);
+          qr[g][1] = make_float2(a0.z, a0.w);
+          qr[g][2] = make_float2(a1.x, a1.y);
+          qr[g][3] = make_float2(a1.z, a1.w);
+        }
+      }
+      uint4 kk = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) {
+        kk = *reinterpret_cast<const uint4*>(ring_k(st, row) + l * 8);
+        vv = *reinterpret_cast<const uint4*>(ring_v(st, row) + l * 8);
+      }
+      const float2 k2[4] = {bf16x2_to_float2(kk.x), bf16x2_to_float2(kk.y),
+                            bf16x2_to_float2(kk.z), bf16x2_to_float2(kk.w)};
+      float part[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float2 s2 = f2_mul(qr[g][0], k2[0]);
+        s2 = f2_fma(qr[g][1], k2[1], s2);
+        s2 = f2_fma(qr[g][2], k2[2], s2);
+        s2 = f2_fma(qr[g][3], k2[3], s2);
+        part[g] = s2.x + s2.y;
+      }
+      const float sc = group_reduce_own<GP, LPK>(part, l);
+      // online softmax of this lane's query, lazy rescale (only when the max grows by > 2^8)
+      const bool need = valid && sc > m_own + 8.0f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2(m_own - sc) : 1.0f;
+        if (need) {
+          l_own *= alpha;
+          m_own = sc;
+        }
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float ag = __shfl_sync(0xffffffffu, alpha, lane_of_query<GP, LPK>(g), LPK);
+          const float2 ag2 = make_float2(ag, ag);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[g][i] = f2_mul(acc[g][i], ag2);
+        }
+      }
+      const float p_own = valid ? ex2(sc - m_own) : 0.f;
+      l_own += p_own;
+      const float2 v2[4] = {bf16x2_to_float2(vv.x), bf16x2_to_float2(vv.y),
+                            bf16x2_to_float2(vv.z), bf16x2_to_float2(vv.w)};
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pg = __shfl_sync(0xffffffffu, p_own, lane_of_query<GP, LPK>(g), LPK);
+        const float2 pg2 = make_float2(pg, pg);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[g][i] = f2_fma(pg2, v2[i], acc[g][i]);
+      }
+    }
+    // the last warp done with this stage refills it (its reads all precede the atomic)
+    __syncwarp();
+    if ((tid & 31) == 0) {
+      __threadfence_block();
+      if (atomicAdd(&sm.done[st], 1) == kDecWarps - 1) {
+        sm.done[st] = 0;
+        if (ch + kDecStages < nchunks) {
+          fence_proxy_async_smem();
+          issue_chunk(ch + kDecStages);
+        }
+      }
+    }
+  }
+  if (__syncthreads_or(!ok)) {
+    // a wait ran out: let the copies of the last issued chunks land before the CTA leaves
+    // (no chunk is issued any more: every warp has left the loop)
+    if (tid == 0) {
+      const int n_is = *reinterpret_cast<volatile int*>(&sm.issued);
+      for (int ch = max(0, n_is - kDecStages); ch < n_is; ++ch)
+        mbar_wait(&sm.full[ch % kDecStages], (ch / kDecStages) & 1, nullptr, nullptr);
+    }
+  }
+
+  // ---- every query's softmax state from the lanes that own it
+  float mrun[GP], lrun[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    mrun[g] = __shfl_sync(0xffffffffu, m_own, lane_of_query<GP, LPK>(g), LPK);
+    lrun[g] = __shfl_sync(0xffffffffu, l_own, lane_of_query<GP, LPK>(g), LPK);
+  }
+  // ---- combine the groups of each warp (lanes l and l ^ LPK, l ^ 2 LPK, ... hold the same
+  // elements)
+#pragma unroll
+  for (int off = LPK; off < 32; off <<= 1) {
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float mo = __shfl_xor_sync(0xffffffffu, mrun[g], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, lrun[g], off);
+      const float M = fmaxf(mrun[g], mo);
+      const float Mu = (M == -INFINITY) ? 0.f : M;
+      const float fs = ex2(mrun[g] - Mu), fo = ex2(mo - Mu);
+      const float2 fs2 = make_float2(fs, fs), fo2 = make_float2(fo, fo);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float2 ao;
+        ao.x = __shfl_xor_sync(0xffffffffu, acc[g][i].x, off);
+        ao.y = __shfl_xor_sync(0xffffffffu, acc[g][i].y, off);
+        acc[g][i] = f2_fma(acc[g][i], fs2, f2_mul(ao, fo2));
+      }
+      lrun[g] = lrun[g] * fs + lo * fo;
+      mrun[g] = M;
+    }
+  }
+  // ---- combine the warps of this CTA through shared memory (the ring is no longer used)
+  __syncthreads();
+  float* s_acc = reinterpret_cast<float*>(sm.buf);  // [kDecWarps][GP][D]
+  if ((tid & 31) < LPK) {
+    if (l == 0) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        sm.wm[warp][g] = mrun[g];
+        sm.wl[warp][g] = lrun[g];
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float4* dst = reinterpret_cast<float4*>(s_acc + ((size_t)warp * GP + g) * D + l * 8);
+      dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+      dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < p.G * D; e += kDecThreads) {
+    const int g = e / D, col = e % D;
+    float M = -INFINITY;
+    for (int x = 0; x < kDecWarps; ++x) M = fmaxf(M, sm.wm[x][g]);
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float sum = 0.f, lsum = 0.f;
+    for (int x = 0; x < kDecWarps; ++x) {
+      const float f = ex2(sm.wm[x][g] - Mu);
+      sum += s_acc[((size_t)x * GP + g) * D + col] * f;
+      lsum += sm.wl[x][g] * f;
+    }
+    const int hq = kvh * p.G + g;
+    p.o[((size_t)seq * p.Hq + hq) * D + col] = __float2bfloat16(lsum > 0.f ? sum / lsum : 0.f);
+    if (col == 0 && p.lse)
+      p.lse[(size_t)seq * p.Hq + hq] =
+          lsum > 0.f ? (M + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+// ------------------------------------------------------------------ export order
 // Slot holding logical rank r (r < occupied).
 __device__ __forceinline__ int rank_to_slot(int r, int ninit, int sep_head, int sep_cnt,
                                             int past_cnt, int win_head, int a, int s, int P,
@@ -428,424 +844,6 @@ __device__ __forceinline__ int rank_to_slot(int r, int ninit, int sep_head, int 
   return a + s + P + (win_head + r) % w;
 }
 
-// N consecutive bf16 from shared memory (4- or 8-byte aligned) to fp32.
-template <int N>
-__device__ __forceinline__ void load_bf16_vec_smem(const __nv_bfloat16* p, float (&out)[N]) {
-  if constexpr (N == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(p);
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-    const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-    out[0] = __low2float(x); out[1] = __high2float(x);
-    out[2] = __low2float(y); out[3] = __high2float(y);
-  } else {
-    static_assert(N == 2, "two or four elements per lane");
-    const uint32_t u = *reinterpret_cast<const unsigned int*>(p);
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u);
-    out[0] = __low2float(x); out[1] = __high2float(x);
-  }
-}
-
-// ------------------------------------------------------------------ decode
-// Streaming: bulk copies bring the K and V rows of kChunk consecutive ranks (as few contiguous
-// slot segments as the rings allow) into a kStages-deep shared-memory ring. Thread 0 fills the
-// first stages; afterwards the last warp to finish reading a stage refills it with the chunk
-// kStages further on, so no thread waits to issue. Half-warp hw handles ranks r0 + hw + 16k;
-// lane16 owns HP rotation pairs (k, k + d/2), k = lane16 * HP + e, of every row it reads.
-// Half-warp reduction of the G per-query partial dot products of one key row: the first
-// log2(G) butterfly levels halve what a lane holds (it keeps one half, adding its partner's copy
-// of it, and sends the other half), the remaining levels sum a single value. Afterwards lane
-// l16 holds the full score of query own_query<G>(l16): 2G + 3 - log2(G) shuffles and adds
-// instead of 4G for one reduction per query.
-template <int G>
-__host__ __device__ constexpr int log2_of() {
-  return G >= 16 ? 4 : G >= 8 ? 3 : G >= 4 ? 2 : G >= 2 ? 1 : 0;
-}
-template <int G>
-__device__ __forceinline__ float halfwarp_reduce_own(float (&v)[G], int lane16) {
-  constexpr int LG = log2_of<G>();
-  static_assert((1 << LG) == G && G <= 16, "G must be a power of two <= 16");
-#pragma unroll
-  for (int l = 0; l < LG; ++l) {
-    const int off = 8 >> l, h = (G >> l) >> 1;
-    const bool upper = (lane16 & off) != 0;
-#pragma unroll
-    for (int i = 0; i < h; ++i) {
-      const float send = upper ? v[i] : v[i + h];
-      const float keep = upper ? v[i + h] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
-  }
-  float r = v[0];
-#pragma unroll
-  for (int l = LG; l < 4; ++l) r += __shfl_xor_sync(0xffffffffu, r, 8 >> l);
-  return r;
-}
-// The query whose score lane l16 holds after halfwarp_reduce_own, and a lane holding query g.
-template <int G>
-__device__ __forceinline__ int own_query(int lane16) {
-  int g = 0;
-#pragma unroll
-  for (int l = 0; l < log2_of<G>(); ++l)
-    if (lane16 & (8 >> l)) g += G >> (l + 1);
-  return g;
-}
-template <int G>
-__device__ __forceinline__ int lane_of_query(int g) {
-  int src = 0;
-#pragma unroll
-  for (int l = 0; l < log2_of<G>(); ++l)
-    if (g & (G >> (l + 1))) src |= 8 >> l;
-  return src;
-}
-
-constexpr int kChunk = 16;
-constexpr int kStages = 4;
-constexpr int kConsumerWarps = kDecThreads / 32;
-
-template <int D>
-struct DecSmem {
-  alignas(128) __nv_bfloat16 k[kStages][kChunk][D];
-  alignas(128) __nv_bfloat16 v[kStages][kChunk][D];
-  uint64_t full[kStages];
-  int done[kStages];  // warps finished with the stage's current chunk
-  int abort_flag;
-};
-
-// ORIG: keys were stored rotated at their original positions (no positional shifting): no
-// rotation of keys here, and the query is rotated at its own original position T - 1.
-template <int D, int G, bool ORIG>
-__global__ void __launch_bounds__(kDecThreads, (G >= 8) ? 2 : 4)
-    sepcache_decode_kernel(int Hq, int Hkv, int a, int s, int P, int w,
-                           const __nv_bfloat16* __restrict__ k_slots,
-                           const __nv_bfloat16* __restrict__ v_slots,
-                           const int32_t* __restrict__ meta, const float2* __restrict__ rope_cs,
-                           const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ o,
-                           float* __restrict__ lse, float scale_log2, double theta,
-                           unsigned* err) {
-  constexpr int HP = D / 32;       // rotation pairs per lane
-  constexpr int HALF = D / 2;
-  const int kvh = blockIdx.x, seq = blockIdx.y;
-  const int c = a + s + P + w;  // slots per sequence (and rows of the cos/sin table)
-  const int tid = threadIdx.x, lane16 = tid & 15, hw = tid >> 4, warp = tid >> 5;
-  extern __shared__ __align__(128) uint8_t dsm_raw[];
-  DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
-
-  const int32_t* m = meta + (size_t)seq * SEPCACHE_META;
-  const int ninit = m[SEPCACHE_META_NINIT];
-  const int sep_head = m[SEPCACHE_META_SEP_HEAD], sep_cnt = m[SEPCACHE_META_SEP_CNT];
-  const int win_head = m[SEPCACHE_META_WIN_HEAD], win_cnt = m[SEPCACHE_META_WIN_CNT];
-  const int past_cnt = (P > 0) ? m[SEPCACHE_META_PAST_CNT] : 0;
-  const int occ = ninit + sep_cnt + past_cnt + win_cnt;
-  const int mq = occ - 1;  // the query's own rank
-  const int r0 = 0, r1 = occ;
-  const int nchunks = r1 > r0 ? (r1 - r0 + kChunk - 1) / kChunk : 0;
-  const size_t row_base = ((size_t)seq * Hkv + kvh) * c;
-  volatile int* abort_flag = &sm.abort_flag;
-
-  auto issue_chunk = [&](int ch) {  // one thread: bulk copies of chunk ch into its stage
-    const int st = ch % kStages;
-    const int c0 = r0 + ch * kChunk;
-    const int rows = min(kChunk, r1 - c0);
-    mbar_arrive_expect_tx(&sm.full[st], (uint32_t)(rows * D * 2 * 2));
-    // ranks map to slots piecewise contiguously: initial block, then the separator ring, then
-    // the past window, then the window ring; a run ends at a block boundary or a ring wrap
-    int r = c0;
-    const int end = c0 + rows;
-    while (r < end) {
-      int slot, len;
-      if (r < ninit) {
-        slot = r;
-        len = min(end, ninit) - r;
-      } else if (r < ninit + sep_cnt) {
-        const int x = (sep_head + (r - ninit)) % s;
-        slot = a + x;
-        len = min(min(end, ninit + sep_cnt) - r, s - x);
-      } else if (r < ninit + sep_cnt + past_cnt) {
-        slot = a + s + (r - ninit - sep_cnt);
-        len = min(end, ninit + sep_cnt + past_cnt) - r;
-      } else {
-        const int x = (win_head + (r - ninit - sep_cnt - past_cnt)) % w;
-        slot = a + s + P + x;
-        len = min(end - r, w - x);
-      }
-      const size_t src = (row_base + slot) * D;
-      bulk_load(&sm.k[st][r - c0][0], k_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
-      bulk_load(&sm.v[st][r - c0][0], v_slots + src, (uint32_t)(len * D * 2), &sm.full[st]);
-      r += len;
-    }
-  };
-  if (tid == 0) {
-    for (int st = 0; st < kStages; ++st) {
-      mbar_init(&sm.full[st], 1);
-      sm.done[st] = 0;
-    }
-    sm.abort_flag = 0;
-    fence_barrier_init();
-    for (int ch = 0; ch < min(kStages, nchunks); ++ch) issue_chunk(ch);
-  }
-  __syncthreads();
-
-  // per-head softmax state (consumers)
-  // softmax state of this lane's own query (see halfwarp_reduce_own); V sums of every query,
-  // as pairs of consecutive elements for the packed fp32x2 arithmetic (lo: elements
-  // lane16 * HP + 2i, +1; hi: the same plus d/2)
-  static_assert(HP % 2 == 0, "rotation pairs per lane come in twos");
-  constexpr int HP2 = HP / 2;
-  float m_own = -INFINITY, l_own = 0.f;
-  float2 acc_lo[G][HP2], acc_hi[G][HP2];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int i = 0; i < HP2; ++i) acc_lo[g][i] = acc_hi[g][i] = make_float2(0.f, 0.f);
-  }
-
-  {
-    // ---------------------------------------------------------------- consumers
-    // query heads of this KV head, rotated by RoPE(mq) (by RoPE(T - 1) without shifting) and
-    // scaled by scale*log2(e)
-    float2 q_lo[G][HP2], q_hi[G][HP2];
-    {
-      float2 qcs[HP];
-#pragma unroll
-      for (int e = 0; e < HP; ++e) {
-        const int k = lane16 * HP + e;
-        if constexpr (ORIG) {
-          double sn, cs;
-          sincos((double)(m[SEPCACHE_META_T] - 1) * pow(theta, -2.0 * (double)k / (double)D), &sn,
-                 &cs);
-          qcs[e] = make_float2((float)cs, (float)sn);
-        } else {
-          qcs[e] = rope_cs[(size_t)max(mq, 0) * HALF + k];
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const __nv_bfloat16* qh = q + ((size_t)seq * Hq + kvh * G + g) * D;
-        float qa[HP], qb[HP];
-#pragma unroll
-        for (int e = 0; e < HP; ++e) {
-          const int k = lane16 * HP + e;
-          const float x1 = __bfloat162float(qh[k]), x2 = __bfloat162float(qh[k + HALF]);
-          const float2 rr = qcs[e];
-          qa[e] = (x1 * rr.x - x2 * rr.y) * scale_log2;
-          qb[e] = (x2 * rr.x + x1 * rr.y) * scale_log2;
-        }
-#pragma unroll
-        for (int i = 0; i < HP2; ++i) {
-          q_lo[g][i] = make_float2(qa[2 * i], qa[2 * i + 1]);
-          q_hi[g][i] = make_float2(qb[2 * i], qb[2 * i + 1]);
-        }
-      }
-    }
-    // cos/sin of this half-warp's current rank, advanced by kHalfWarps per step (pairs of
-    // consecutive frequencies; nsd = -sin of the step)
-    float2 cr[HP2], sr[HP2], cd[HP2], sd[HP2], nsd[HP2];
-    {
-      const int rf = r0 + hw;
-#pragma unroll
-      for (int i = 0; i < HP2; ++i) {
-        const int k = lane16 * HP + 2 * i;
-        const float2 v0 = (rf < r1) ? rope_cs[(size_t)rf * HALF + k] : make_float2(1.f, 0.f);
-        const float2 v1 = (rf < r1) ? rope_cs[(size_t)rf * HALF + k + 1] : make_float2(1.f, 0.f);
-        cr[i] = make_float2(v0.x, v1.x);
-        sr[i] = make_float2(v0.y, v1.y);
-        const float2 t0 = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k];
-        const float2 t1 = rope_cs[(size_t)min(kHalfWarps, c - 1) * HALF + k + 1];
-        cd[i] = make_float2(t0.x, t1.x);
-        sd[i] = make_float2(t0.y, t1.y);
-        nsd[i] = make_float2(-t0.y, -t1.y);
-      }
-    }
-    bool ok = true;
-    for (int ch = 0; ch < nchunks && ok; ++ch) {
-      const int st = ch % kStages;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[st], (ch / kStages) & 1, err, abort_flag))) {
-        ok = false;
-        break;
-      }
-      const int c0 = r0 + ch * kChunk;
-#pragma unroll
-      for (int sub = 0; sub < kChunk / kHalfWarps; ++sub) {
-        const int row = sub * kHalfWarps + hw;
-        const bool valid = c0 + row < r1;
-        float k1[HP], k2[HP], v1[HP], v2[HP];
-        const __nv_bfloat16* kr = &sm.k[st][row][lane16 * HP];
-        const __nv_bfloat16* vr = &sm.v[st][row][lane16 * HP];
-        if (valid) {
-          load_bf16_vec_smem<HP>(kr, k1);
-          load_bf16_vec_smem<HP>(kr + HALF, k2);
-          load_bf16_vec_smem<HP>(vr, v1);
-          load_bf16_vec_smem<HP>(vr + HALF, v2);
-        } else {
-#pragma unroll
-          for (int e = 0; e < HP; ++e) k1[e] = k2[e] = v1[e] = v2[e] = 0.f;
-        }
-        // rotate (y1, y2) = RoPE(rank) (k1, k2) and form the G partial dot products, two
-        // frequencies per packed instruction
-        float2 part2[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) part2[g] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < HP2; ++i) {
-          const float2 x1 = make_float2(k1[2 * i], k1[2 * i + 1]);
-          const float2 x2 = make_float2(k2[2 * i], k2[2 * i + 1]);
-          float2 y1 = x1, y2 = x2;
-          if constexpr (!ORIG) {
-            y1 = f2_sub(f2_mul(x1, cr[i]), f2_mul(x2, sr[i]));
-            y2 = f2_fma(x2, cr[i], f2_mul(x1, sr[i]));
-          }
-#pragma unroll
-          for (int g = 0; g < G; ++g) part2[g] = f2_fma(q_lo[g][i], y1, f2_fma(q_hi[g][i], y2, part2[g]));
-        }
-        float part[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) part[g] = part2[g].x + part2[g].y;
-        if constexpr (!ORIG) {
-#pragma unroll
-          for (int i = 0; i < HP2; ++i) {
-            const float2 cn = f2_fma(cr[i], cd[i], f2_mul(sr[i], nsd[i]));
-            sr[i] = f2_fma(sr[i], cd[i], f2_mul(cr[i], sd[i]));
-            cr[i] = cn;
-          }
-        }
-        // this lane's query score; the online softmax of that query only, its probability
-        // then broadcast to the lanes of the half-warp for the V accumulation of every query
-        const float sc = halfwarp_reduce_own<G>(part, lane16);
-        const bool need = valid && sc > m_own + 8.0f;  // lazy rescale (max grew by > 2^8)
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2(m_own - sc) : 1.0f;
-          if (need) {
-            l_own *= alpha;
-            m_own = sc;
-          }
-#pragma unroll
-          for (int g = 0; g < G; ++g) {
-            const float ag = __shfl_sync(0xffffffffu, alpha, lane_of_query<G>(g), 16);
-            const float2 ag2 = make_float2(ag, ag);
-#pragma unroll
-            for (int i = 0; i < HP2; ++i) {
-              acc_lo[g][i] = f2_mul(acc_lo[g][i], ag2);
-              acc_hi[g][i] = f2_mul(acc_hi[g][i], ag2);
-            }
-          }
-        }
-        const float p_own = valid ? ex2(sc - m_own) : 0.f;
-        l_own += p_own;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pg = __shfl_sync(0xffffffffu, p_own, lane_of_query<G>(g), 16);
-          const float2 pg2 = make_float2(pg, pg);
-#pragma unroll
-          for (int i = 0; i < HP2; ++i) {
-            acc_lo[g][i] = f2_fma(pg2, make_float2(v1[2 * i], v1[2 * i + 1]), acc_lo[g][i]);
-            acc_hi[g][i] = f2_fma(pg2, make_float2(v2[2 * i], v2[2 * i + 1]), acc_hi[g][i]);
-          }
-        }
-      }
-      // the last warp done with this stage refills it (its reads all precede the atomic)
-      __syncwarp();
-      if ((tid & 31) == 0) {
-        if (atomicAdd(&sm.done[st], 1) == kConsumerWarps - 1) {
-          sm.done[st] = 0;
-          if (ch + kStages < nchunks) {
-            fence_proxy_async_smem();
-            issue_chunk(ch + kStages);
-          }
-        }
-      }
-    }
-    if (!ok) {
-      // a wait ran out: let every copy still in flight land before the CTA leaves
-      if (tid == 0)
-        for (int ch = 0; ch < nchunks; ++ch)
-          mbar_wait(&sm.full[ch % kStages], (ch / kStages) & 1, nullptr, nullptr);
-    }
-  }
-
-  float acc[G][2 * HP];  // V sums, elements lane16 * HP + e (e < HP) and the same plus d/2
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-#pragma unroll
-    for (int i = 0; i < HP2; ++i) {
-      acc[g][2 * i] = acc_lo[g][i].x;
-      acc[g][2 * i + 1] = acc_lo[g][i].y;
-      acc[g][HP + 2 * i] = acc_hi[g][i].x;
-      acc[g][HP + 2 * i + 1] = acc_hi[g][i].y;
-    }
-  }
-  // every query's softmax state from the lanes that own it
-  float mrun[G], lrun[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    mrun[g] = __shfl_sync(0xffffffffu, m_own, lane_of_query<G>(g), 16);
-    lrun[g] = __shfl_sync(0xffffffffu, l_own, lane_of_query<G>(g), 16);
-  }
-  // ---- combine the two half-warps of each warp (lanes l and l^16 hold the same columns)
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float mo = __shfl_xor_sync(0xffffffffu, mrun[g], 16);
-    const float lo = __shfl_xor_sync(0xffffffffu, lrun[g], 16);
-    const float M = fmaxf(mrun[g], mo);
-    const float Mu = (M == -INFINITY) ? 0.f : M;
-    const float fs = ex2(mrun[g] - Mu), fo = ex2(mo - Mu);
-#pragma unroll
-    for (int e = 0; e < 2 * HP; ++e) {
-      const float ao = __shfl_xor_sync(0xffffffffu, acc[g][e], 16);
-      acc[g][e] = acc[g][e] * fs + ao * fo;
-    }
-    lrun[g] = lrun[g] * fs + lo * fo;
-    mrun[g] = M;
-  }
-  // ---- combine the consumer warps of this CTA through shared memory
-  __shared__ float s_m[kConsumerWarps][G], s_l[kConsumerWarps][G];
-  __shared__ float s_acc[kConsumerWarps][G][D];
-  __shared__ float s_res[G][D + 2];  // this CTA's combined (acc..., m, l) per head
-  if ((tid & 31) < 16) {
-    if (lane16 == 0) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        s_m[warp][g] = mrun[g];
-        s_l[warp][g] = lrun[g];
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-      for (int e = 0; e < HP; ++e) {
-        s_acc[warp][g][lane16 * HP + e] = acc[g][e];
-        s_acc[warp][g][HALF + lane16 * HP + e] = acc[g][HP + e];
-      }
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < G * D; e += blockDim.x) {
-    const int g = e / D, col = e % D;
-    float M = -INFINITY;
-    for (int x = 0; x < kConsumerWarps; ++x) M = fmaxf(M, s_m[x][g]);
-    const float Mu = (M == -INFINITY) ? 0.f : M;
-    float sum = 0.f, lsum = 0.f;
-    for (int x = 0; x < kConsumerWarps; ++x) {
-      const float f = ex2(s_m[x][g] - Mu);
-      sum += s_acc[x][g][col] * f;
-      lsum += s_l[x][g] * f;
-    }
-    s_res[g][col] = sum;
-    if (col == 0) {
-      s_res[g][D] = M;
-      s_res[g][D + 1] = lsum;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < G * D; e += blockDim.x) {
-    const int g = e / D, col = e % D;
-    const int hq = kvh * G + g;
-    o[((size_t)seq * Hq + hq) * D + col] = __float2bfloat16(s_res[g][col] / s_res[g][D + 1]);
-    if (col == 0 && lse)
-      lse[(size_t)seq * Hq + hq] = (s_res[g][D] + __log2f(s_res[g][D + 1])) * 0.69314718055994531f;
-  }
-}
-
-// ------------------------------------------------------------------ export order
 __global__ void sepcache_export_kernel(int a, int s, int P, int w,
                                        const int32_t* __restrict__ meta,
                                        const int32_t* __restrict__ slot_pos,
@@ -867,14 +865,18 @@ __global__ void sepcache_export_kernel(int a, int s, int P, int w,
   if (threadIdx.x == 0) count[seq] = occ;
 }
 
+// ------------------------------------------------------------------ launchers
 // Past Window slots and slots per sequence of a cache state.
 static int past_slots(const SepCacheState& st) { return st.c > 0 ? st.c - st.a - st.w : 0; }
 static int cache_slots(const SepCacheState& st) { return st.a + st.s + past_slots(st) + st.w; }
+static CacheDims cache_dims(const SepCacheState& st) {
+  return CacheDims{st.Hkv, st.d, st.a, st.s, st.w, past_slots(st), st.c, st.original_positions};
+}
 
 cudaError_t launch_sepcache_init(const SepCacheState& st, cudaStream_t stream) {
   const int c = cache_slots(st);
   sepcache_init_kernel<<<64, 256, 0, stream>>>(st.S, c, st.d, (double)st.rope_theta, st.meta,
-                                               st.slot_pos, st.slot_sep, st.rope_cs);
+                                               st.slot_pos, st.slot_sep, st.rope_freq);
   return cudaGetLastError();
 }
 
@@ -883,54 +885,91 @@ cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new, c
   const int P = past_slots(st);
   const size_t smem = (size_t)max(1, min(st.s, P)) * sizeof(int2);  // compression moves
   sepcache_update_kernel<<<st.S, kUpdateThreads, smem, stream>>>(
-      st.Hkv, st.d, st.a, st.s, st.w, P, st.c, st.original_positions, (double)st.rope_theta,
-      reinterpret_cast<uint4*>(st.k_slots),
+      cache_dims(st), st.rope_freq, reinterpret_cast<uint4*>(st.k_slots),
       reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta,
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), sep_new);
   return cudaGetLastError();
 }
 
-template <int D, int G, bool ORIG>
+cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, const void* v,
+                                    const uint8_t* sep, int L, cudaStream_t stream) {
+  const size_t smem = (size_t)max(st.s, 1) * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(sepcache_prefill_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  sepcache_prefill_kernel<<<dim3(st.S, st.Hkv), kPrefillThreads, smem, stream>>>(
+      L, cache_dims(st), st.rope_freq, static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), sep, reinterpret_cast<uint4*>(st.k_slots),
+      reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta);
+  return cudaGetLastError();
+}
+
+template <int D, int GP, bool ORIG>
 static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void* o, float* lse,
                                    float scale, cudaStream_t stream) {
-  constexpr size_t smem = sizeof(DecSmem<D>);
+  constexpr size_t smem = sizeof(DecSmem<D, GP>);
   static bool attr_set[64] = {false};  // per device: set once, outside any stream capture
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(sepcache_decode_kernel<D, G, ORIG>,
+    e = cudaFuncSetAttribute(sepcache_decode_kernel<D, GP, ORIG>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
+  DecodeArgs a;
+  a.Hq = st.Hq;
+  a.Hkv = st.Hkv;
+  a.G = st.Hq / st.Hkv;
+  a.a = st.a;
+  a.s = st.s;
+  a.P = past_slots(st);
+  a.w = st.w;
+  a.k_slots = reinterpret_cast<const __nv_bfloat16*>(st.k_slots);
+  a.v_slots = reinterpret_cast<const __nv_bfloat16*>(st.v_slots);
+  a.meta = st.meta;
+  a.freq = st.rope_freq;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.err = device_error_word();
   dim3 grid(st.Hkv, st.S);
-  sepcache_decode_kernel<D, G, ORIG><<<grid, kDecThreads, smem, stream>>>(
-      st.Hq, st.Hkv, st.a, st.s, past_slots(st), st.w,
-      reinterpret_cast<const __nv_bfloat16*>(st.k_slots),
-      reinterpret_cast<const __nv_bfloat16*>(st.v_slots), st.meta,
-      reinterpret_cast<const float2*>(st.rope_cs), static_cast<const __nv_bfloat16*>(q),
-      static_cast<__nv_bfloat16*>(o), lse, scale * 1.4426950408889634f, (double)st.rope_theta,
-      device_error_word());
+  sepcache_decode_kernel<D, GP, ORIG><<<grid, kDecThreads, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int GP>
+static cudaError_t launch_decode_d(const SepCacheState& st, const void* q, void* o, float* lse,
+                                   float scale, cudaStream_t stream) {
+  return st.original_positions ? launch_decode_t<D, GP, true>(st, q, o, lse, scale, stream)
+                               : launch_decode_t<D, GP, false>(st, q, o, lse, scale, stream);
 }
 
 cudaError_t launch_sepcache_decode(const SepCacheState& st, const void* q, void* o, float* lse,
                                    float scale, cudaStream_t stream) {
-  const int G = st.Hq / st.Hkv;
-#define SEP_DEC_CASE(DD, GG) \
-  if (st.d == DD && G == GG)                                                             \
-    return st.original_positions ? launch_decode_t<DD, GG, true>(st, q, o, lse, scale, stream) \
-                                 : launch_decode_t<DD, GG, false>(st, q, o, lse, scale, stream);
-  SEP_DEC_CASE(128, 1)
-  SEP_DEC_CASE(128, 2)
-  SEP_DEC_CASE(128, 4)
-  SEP_DEC_CASE(128, 8)
-  SEP_DEC_CASE(64, 1)
-  SEP_DEC_CASE(64, 2)
-  SEP_DEC_CASE(64, 4)
-  SEP_DEC_CASE(64, 8)
-#undef SEP_DEC_CASE
+  const int G = st.Hq / st.Hkv;  // padded to the next power of two (zero queries)
+  const int GP = G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : 8;
+  if (G < 1 || G > 8) return cudaErrorInvalidValue;
+  if (st.d == 128) {
+    switch (GP) {
+      case 1: return launch_decode_d<128, 1>(st, q, o, lse, scale, stream);
+      case 2: return launch_decode_d<128, 2>(st, q, o, lse, scale, stream);
+      case 4: return launch_decode_d<128, 4>(st, q, o, lse, scale, stream);
+      default: return launch_decode_d<128, 8>(st, q, o, lse, scale, stream);
+    }
+  }
+  if (st.d == 64) {
+    switch (GP) {
+      case 1: return launch_decode_d<64, 1>(st, q, o, lse, scale, stream);
+      case 2: return launch_decode_d<64, 2>(st, q, o, lse, scale, stream);
+      case 4: return launch_decode_d<64, 4>(st, q, o, lse, scale, stream);
+      default: return launch_decode_d<64, 8>(st, q, o, lse, scale, stream);
+    }
+  }
   return cudaErrorInvalidValue;
 }
 

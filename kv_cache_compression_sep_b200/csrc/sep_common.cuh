@@ -12,11 +12,12 @@
 #include <stdint.h>
 
 #include "../../include/sepattn.h"
+#include "sep_launch.h"
 
 namespace sep {
 
 // Wall-clock limit of one bounded wait: 1.5 s.
-constexpr unsigned long long kWaitLimitNs = 1500ull * 1000ull * 1000ull;
+constexpr unsigned long long kWaitLimitNs = kDefaultPipelineWaitNs;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -66,17 +67,19 @@ __device__ __forceinline__ void record_failure(unsigned* err, volatile int* abor
   if (abort_flag) *abort_flag = 1;
 }
 
-// Bounded wait for the phase of `parity` to complete. Returns false on timeout or when the
-// CTA abort flag is already raised (another role gave up).
+// Bounded wait for the phase of `parity` to complete. Returns false on timeout (after
+// `limit_ns` of %globaltimer) or when the CTA abort flag is already raised (another role gave
+// up).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_failure(err, abort_flag, SEP_ERR_TIMEOUT);
         return false;
       }

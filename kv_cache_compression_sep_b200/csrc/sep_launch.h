@@ -13,6 +13,10 @@ namespace sep {
 
 // Device address of the sticky error word on the current device (nullptr on failure).
 unsigned* device_error_word();
+// Wall-clock limit of each pipeline wait of the attention forward kernel (sep_set_wait_limit_ns);
+// by default the same 1.5 s as every other bounded wait.
+constexpr unsigned long long kDefaultPipelineWaitNs = 1500ull * 1000ull * 1000ull;
+unsigned long long pipeline_wait_limit_ns();
 // Fixed scratch of sep_attn_fwd_noalloc on the current device (first call per device: setup).
 void* noalloc_fwd_scratch(cudaError_t* err);
 

@@ -46,6 +46,7 @@ def _load():
         "sepcache_prefill": (I, [P, P, P, P, I, P]),
         "sepcache_export_order": (I, [P, P, P, P]),
         "sep_last_device_error": (I, []),
+        "sep_set_wait_limit_ns": (I, [ctypes.c_ulonglong]),
         "sep_status_string": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -73,7 +74,7 @@ class _SepCacheState(ctypes.Structure):
                 ("original_positions", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
-                ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]
+                ("meta", ctypes.c_void_p), ("rope_freq", ctypes.c_void_p)]
 
 
 def _check(status: int, what: str):
@@ -105,6 +106,28 @@ def _cuda(t, dtype, name, shape=None):
         raise SepError(f"{name} must be on a CUDA device (there is no CPU path)")
 
 
+def _current_device_index():
+    return torch.cuda.current_device()
+
+
+def _same_device(dev, *named):
+    """Every tensor of a call on one device, and that device the current one: the library
+    launches on the current device and builds its copy descriptors over these pointers, so a
+    tensor of another GPU would be read as if it were local."""
+    for name, t in named:
+        if t is not None and t.device != dev:
+            raise SepError(f"{name} is on {t.device}, the call's other tensors on {dev}")
+    cur = _current_device_index()
+    if dev.index is not None and dev.index != cur:
+        raise SepError(f"the call's tensors are on {dev} but the current CUDA device is "
+                       f"cuda:{cur}; make {dev} current (torch.cuda.device) for this call")
+
+
+def _mask_tensors(mask):
+    return [("mask." + f, getattr(mask, f)) for f in
+            ("sep", "anchor_idx", "anchor_cnt", "anchor_bits", "gather_end", "tile_map")]
+
+
 def _dims(t, ndim, name):
     if not isinstance(t, torch.Tensor) or t.dim() != ndim:
         raise SepError(f"{name} must be a {ndim}-D tensor")
@@ -113,6 +136,11 @@ def _dims(t, ndim, name):
 
 def sep_last_device_error() -> int:
     return int(_lib.sep_last_device_error())
+
+
+def sep_set_wait_limit_ns(ns: int) -> None:
+    """Test hook: limit of each pipeline wait of later forward launches (0 = default 1.5 s)."""
+    _check(_lib.sep_set_wait_limit_ns(int(ns)), "sep_set_wait_limit_ns")
 
 
 @dataclasses.dataclass
@@ -159,6 +187,7 @@ def sep_mask_build(sep: torch.Tensor, a: int, n: int, bm: int = TILE, bn: int = 
                       gather_end=torch.empty(B, T, dtype=torch.int32, device=dev),
                       tile_map=torch.empty(B, T, U, dtype=torch.int8, device=dev),
                       kept=torch.empty(B, dtype=torch.int64, device=dev), a=a, n=n)
+    _same_device(dev, *_mask_tensors(out), ("out.kept", out.kept))
     _check(_lib.sep_mask_build(_ptr(sep), B, L, a, n, bm, bn, _ptr(out.anchor_idx),
                                _ptr(out.anchor_cnt), _ptr(out.anchor_bits), _ptr(out.gather_end),
                                _ptr(out.tile_map), _ptr(out.kept), _stream()), "sep_mask_build")
@@ -211,6 +240,8 @@ def sep_attn_fwd(q, k, v, mask: SepMask, scale=None, out=None, lse=None, workspa
     _cuda(lse, torch.float32, "lse", (B, Hq, L))
     nbytes = sep_attn_fwd_workspace_size(B, L, Hkv, d)
     ws = _workspace(nbytes, q.device, workspace)
+    _same_device(q.device, ("k", k), ("v", v), ("out", o), ("lse", lse), ("workspace", ws),
+                 *_mask_tensors(mask))
     mc = mask._c()
     args = (_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale), mask.a, mask.n,
             ctypes.byref(mc), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(), _stream())
@@ -234,6 +265,7 @@ def sep_attn_fwd_noalloc(q, k, v, mask: SepMask, scale=None, out=None, lse=None)
     lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device) if lse is None else lse
     _cuda(o, torch.bfloat16, "out", (B, L, Hq, d))
     _cuda(lse, torch.float32, "lse", (B, Hq, L))
+    _same_device(q.device, ("k", k), ("v", v), ("out", o), ("lse", lse), *_mask_tensors(mask))
     mc = mask._c()
     _check(_lib.sep_attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), B, L, Hq, Hkv, d, float(scale),
                                      mask.a, mask.n, ctypes.byref(mc), _ptr(o), _ptr(lse),
@@ -261,6 +293,8 @@ def sep_attn_bwd(q, k, v, o, lse, dout, mask: SepMask, scale=None, workspace=Non
     _cuda(dv, torch.bfloat16, "dv", (B, L, Hkv, d))
     nbytes = sep_attn_bwd_workspace_size(B, L, Hq, Hkv, d)
     ws = _workspace(nbytes, q.device, workspace)
+    _same_device(q.device, ("k", k), ("v", v), ("o", o), ("lse", lse), ("dout", dout),
+                 ("dq", dq), ("dk", dk), ("dv", dv), ("workspace", ws), *_mask_tensors(mask))
     mc = mask._c()
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), B, L, Hq, Hkv, d,
             float(scale), mask.a, mask.n, ctypes.byref(mc), _ptr(dq), _ptr(dk), _ptr(dv),
@@ -299,14 +333,20 @@ class SepCache:
         self.slot_pos = torch.empty(S, self.n, dtype=torch.int32, device=dev)
         self.slot_sep = torch.empty(S, self.n, dtype=torch.uint8, device=dev)
         self.meta = torch.empty(S, META, dtype=torch.int32, device=dev)
-        self.rope_cs = torch.empty(self.n, d, dtype=torch.float32, device=dev)
+        self.rope_freq = torch.empty(d // 2, dtype=torch.float64, device=dev)
         self.original_positions = bool(original_positions)
         self._st = _SepCacheState(S, Hq, Hkv, d, a, s, w, self.c, int(self.original_positions),
                                   self.rope_theta,
                                   self.k_slots.data_ptr(), self.v_slots.data_ptr(),
                                   self.slot_pos.data_ptr(), self.slot_sep.data_ptr(),
-                                  self.meta.data_ptr(), self.rope_cs.data_ptr())
+                                  self.meta.data_ptr(), self.rope_freq.data_ptr())
+        self._on_device()
         _check(_lib.sepcache_state_init(ctypes.byref(self._st), _stream()), "sepcache_state_init")
+
+    def _on_device(self, *named):
+        _same_device(self.k_slots.device, ("v_slots", self.v_slots), ("slot_pos", self.slot_pos),
+                     ("slot_sep", self.slot_sep), ("meta", self.meta),
+                     ("rope_freq", self.rope_freq), *named)
 
     def sepcache_prefill(self, k, v, sep):
         """Seeds every sequence with a prompt: k, v [S, L, Hkv, d] bf16, sep [S, L] uint8."""
@@ -314,11 +354,12 @@ class SepCache:
         _cuda(k, torch.bfloat16, "k", (self.S, L, self.Hkv, self.d))
         _cuda(v, torch.bfloat16, "v", (self.S, L, self.Hkv, self.d))
         _cuda(sep, torch.uint8, "sep", (self.S, L))
+        self._on_device(("k", k), ("v", v), ("sep", sep))
         _check(_lib.sepcache_prefill(ctypes.byref(self._st), _ptr(k), _ptr(v), _ptr(sep), L,
                                      _stream()), "sepcache_prefill")
 
-    # checkpoint / resume: the whole state lives in these tensors (the cos/sin table is a pure
-    # function of c, d and theta and is rebuilt by the constructor)
+    # checkpoint / resume: the whole state lives in these tensors (the RoPE frequency table is a
+    # pure function of d and theta and is rebuilt by the constructor)
     _STATE = ("k_slots", "v_slots", "slot_pos", "slot_sep", "meta")
 
     def state_dict(self):
@@ -338,6 +379,7 @@ class SepCache:
         _cuda(k_new, torch.bfloat16, "k_new", (self.S, self.Hkv, self.d))
         _cuda(v_new, torch.bfloat16, "v_new", (self.S, self.Hkv, self.d))
         _cuda(sep_new, torch.uint8, "sep_new", (self.S,))
+        self._on_device(("k_new", k_new), ("v_new", v_new), ("sep_new", sep_new))
         _check(_lib.sepcache_update(ctypes.byref(self._st), _ptr(k_new), _ptr(v_new),
                                     _ptr(sep_new), _stream()), "sepcache_update")
 
@@ -348,6 +390,7 @@ class SepCache:
         _cuda(o, torch.bfloat16, "out", (self.S, self.Hq, self.d))
         if lse is not None:
             _cuda(lse, torch.float32, "lse", (self.S, self.Hq))
+        self._on_device(("q", q), ("out", o), ("lse", lse))
         _check(_lib.sepcache_decode(ctypes.byref(self._st), _ptr(q), _ptr(o), _ptr(lse),
                                     float(scale), _stream()), "sepcache_decode")
         return o
@@ -355,6 +398,7 @@ class SepCache:
     def sepcache_export_order(self):
         pos = torch.empty(self.S, self.n, dtype=torch.int32, device=self.k_slots.device)
         cnt = torch.empty(self.S, dtype=torch.int32, device=self.k_slots.device)
+        self._on_device()
         _check(_lib.sepcache_export_order(ctypes.byref(self._st), _ptr(pos), _ptr(cnt),
                                           _stream()), "sepcache_export_order")
         return pos, cnt

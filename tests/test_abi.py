@@ -108,7 +108,7 @@ class _CacheState(ctypes.Structure):
                 ("original_positions", ctypes.c_int32), ("rope_theta", ctypes.c_float),
                 ("k_slots", ctypes.c_void_p), ("v_slots", ctypes.c_void_p),
                 ("slot_pos", ctypes.c_void_p), ("slot_sep", ctypes.c_void_p),
-                ("meta", ctypes.c_void_p), ("rope_cs", ctypes.c_void_p)]
+                ("meta", ctypes.c_void_p), ("rope_freq", ctypes.c_void_p)]
 
 
 def test_cache_rejects_bad_state(lib):
@@ -118,7 +118,7 @@ def test_cache_rejects_bad_state(lib):
 
     def st(**kw):
         base = dict(S=2, Hq=8, Hkv=2, d=128, a=4, s=8, w=16, rope_theta=1e4, k_slots=256,
-                    v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_cs=256)
+                    v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_freq=256)
         base.update(kw)
         return _CacheState(**base)
 
@@ -141,10 +141,10 @@ def test_prefill_rejects_bad_arguments(lib):
     f.restype = ctypes.c_int
     P, I = ctypes.c_void_p, ctypes.c_int
     st = _CacheState(S=2, Hq=8, Hkv=2, d=128, a=4, s=8, w=16, rope_theta=1e4, k_slots=256,
-                     v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_cs=256)
+                     v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_freq=256)
     assert f(ctypes.byref(st), P(256), P(256), P(256), I(0), None) == SEP_ERR_INVALID_ARG
     assert f(ctypes.byref(st), None, P(256), P(256), I(8), None) == SEP_ERR_INVALID_ARG
     assert f(ctypes.byref(st), P(264), P(256), P(256), I(8), None) == SEP_ERR_MISALIGNED
     big = _CacheState(S=2, Hq=8, Hkv=2, d=128, a=4, s=20000, w=16, rope_theta=1e4, k_slots=256,
-                      v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_cs=256)
+                      v_slots=256, slot_pos=256, slot_sep=256, meta=256, rope_freq=256)
     assert f(ctypes.byref(big), P(256), P(256), P(256), I(8), None) == SEP_ERR_UNSUPPORTED

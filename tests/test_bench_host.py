@@ -8,13 +8,54 @@ import pytest
 import bench
 
 
-def test_traffic_table_rows():
-    with open(os.path.join(bench.ROOT, "profiles", "traffic.md")) as fh:
-        rows = [ln for ln in fh if ln.startswith("| bwd_dkdv ")]
-    assert len(rows) == 1
-    want = int(rows[0].split("|")[3])
-    assert bench.load_traffic("bwd_dkdv") == want
+def test_traffic_table_follows_the_kernel_source(tmp_path, monkeypatch):
+    """A capture's DRAM bytes are reported only while the kernel source it was taken from is
+    unchanged (the table stores the source file's digest)."""
+    import json
+    good = bench.source_digest("k_attn_bwd.cu")
+    table = {"passes": {"bwd_dkdv": {"source": "k_attn_bwd.cu", "source_sha256": good,
+                                     "bytes_per_launch": 123456},
+                        "fwd_kernel": {"source": "k_attn_fwd.cu", "source_sha256": "0" * 16,
+                                       "bytes_per_launch": 654321}}}
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(table))
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(p))
+    assert bench.load_traffic("bwd_dkdv") == 123456
+    assert bench.load_traffic("fwd_kernel") is None   # source changed since the capture
     assert bench.load_traffic("no_such_pass") is None
+
+
+def test_committed_traffic_table_is_well_formed():
+    import json
+    if not os.path.exists(bench.TRAFFIC_JSON):
+        pytest.skip("no capture table committed")
+    with open(bench.TRAFFIC_JSON) as fh:
+        table = json.load(fh)
+    for name, e in table["passes"].items():
+        assert name in ("fwd_kernel", "bwd_dq", "bwd_dkdv", "decode_attention")
+        assert os.path.exists(os.path.join(bench.CSRC, e["source"]))
+        assert int(e["bytes_per_launch"]) > 0 and len(e["source_sha256"]) == 16
+
+
+def test_algorithmic_bytes_of_the_passes():
+    # Pythia-160m shape: Q, dO, K, V read, dK, dV written, LSE and Delta (fp32) read
+    B, L, H, d = 8, 2048, 12, 64
+    t = B * L * H * d * 2
+    st = B * H * L * 4
+    assert bench.attn_pass_bytes(B, L, H, H, d, "bwd_dkdv") == 6 * t + 2 * st
+    assert bench.attn_pass_bytes(B, L, H, H, d, "fwd_kernel") == 4 * t + st
+    assert bench.attn_pass_bytes(B, L, H, H, d, "bwd_dq") == 5 * t + 2 * st
+
+
+def test_pair_slots_counts_whole_tiles():
+    import numpy as np
+    # L = 512 (4 tiles), n = 64: window tiles t-1..t (t >= 1), tile 0 alone; 200 anchors left
+    # of the window of tile 3 make two anchor chunks there
+    ge = np.array([[0, 0, 5, 200]])
+    slots = bench.pair_slots(ge, 512, 64)
+    assert slots == (1 + 2 + (2 + 1) + (2 + 2)) * 128 * 128
+    # n >= L: every query tile runs tiles 0..t
+    assert bench.pair_slots(np.zeros((1, 4), dtype=int), 512, 512) == (1 + 2 + 3 + 4) * 128 * 128
 
 
 def test_roofline_tensor_pass():
@@ -28,6 +69,19 @@ def test_roofline_tensor_pass():
     assert r["frac"] == pytest.approx(r["achieved"] / 1600.0)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["kernel"] == "sep_attn_bwd_dkv_kernel"
+
+
+def test_combined_roofline_takes_the_slower_bound():
+    import workloads
+    cfg = workloads.PYTHIA160M
+    step = types.SimpleNamespace(flops_fwd=8.15e9, bytes_dec=2.0e8, cfg=cfg)
+    peaks = {"bf16_tflops": 1638.7, "hbm_gbs": 6555.2}
+    r = bench.roofline_for("bwd_dkdv", {"bwd_dkdv": 0.1266}, step, peaks, "measured")
+    byts = bench.attn_pass_bytes(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.d, "bwd_dkdv")
+    assert byts == pytest.approx(152.6e6, rel=2e-3)
+    t_min = max(2 * 8.15e9 / 1638.7e12, byts / 6555.2e9)
+    assert r["combined_frac"] == pytest.approx(t_min / 0.1266e-3)
+    assert r["combined_bound"] == "hbm"
 
 
 def test_roofline_decode_pass():

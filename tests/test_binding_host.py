@@ -77,3 +77,19 @@ def test_attention_refuses_cpu_tensors():
 def test_cache_refuses_a_cpu_device():
     with pytest.raises(S.SepError, match="CUDA"):
         S.SepCache(2, 8, 2, 128, 2, 3, 5, 10000.0, device="cpu")
+
+
+def test_device_checks(monkeypatch):
+    """Every tensor of a call must be on one device, and that device must be the current one
+    (the library launches there); checked before anything reaches the library."""
+    import types
+    d0, d1 = torch.device("cuda", 0), torch.device("cuda", 1)
+    t0, t1 = types.SimpleNamespace(device=d0), types.SimpleNamespace(device=d1)
+    monkeypatch.setattr(S, "_current_device_index", lambda: 0)
+    S._same_device(d0, ("k", t0), ("v", t0), ("lse", None))
+    with pytest.raises(S.SepError, match="v is on cuda:1"):
+        S._same_device(d0, ("k", t0), ("v", t1))
+    with pytest.raises(S.SepError, match="current CUDA device is cuda:0"):
+        S._same_device(d1, ("k", t1))
+    monkeypatch.setattr(S, "_current_device_index", lambda: 1)
+    S._same_device(d1, ("k", t1))

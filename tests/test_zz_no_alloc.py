@@ -2,8 +2,9 @@
 
 Collected last (file name) so that it also runs after every other test in one process. The GPU
 tests compare two calls in a row against the workspace entry point sep_attn_fwd on the same
-inputs, within the forward tolerances; the CPU test checks that an oversized problem is refused
-on the host before any device work.
+inputs: the kernels are the same and deterministic, so the outputs must be bit-identical (the
+forward tolerances are checked as well, for a readable message); the CPU test checks that an
+oversized problem is refused on the host before any device work.
 """
 
 import ctypes
@@ -70,11 +71,14 @@ def S():
 
 
 def _check(o, lse, o_ref, lse_ref, what):
+    import torch
     err = np.abs(f64(o) - f64(o_ref))
     assert np.isfinite(f64(o)).all(), what
     assert err.max() <= O_MAX_ABS and err.mean() <= O_MEAN_ABS, f"{what}: {err.max():.3e}"
     lerr = np.abs(f64(lse) - f64(lse_ref))
     assert lerr.max() <= LSE_ABS, f"{what}: lse {lerr.max():.3e}"
+    assert torch.equal(o, o_ref), f"{what}: O not bit-identical to sep_attn_fwd"
+    assert torch.equal(lse, lse_ref), f"{what}: LSE not bit-identical to sep_attn_fwd"
 
 
 @pytest.mark.gpu

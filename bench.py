@@ -67,7 +67,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.index), "-lms", "100"],
+                 "-i", str(self.index), "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -248,17 +248,19 @@ def native(args, rank, world, dev):
     graph = capture(step.run)
     assert S.sep_last_device_error() == 0
 
-    for i in range(args.warmup):
-        flush_l2(flush)
-        graph.replay()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    with ClockSampler(dev.index) as clk:
+    # clocks sampled from the warm-up on, through the timed steps and the per-pass rows
+    clk = ClockSampler(dev.index).__enter__()
+    try:
+        for i in range(args.warmup):
+            flush_l2(flush)
+            graph.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
         torch.cuda.nvtx.range_push("timed")
         for i in range(args.steps):
             flush_l2(flush)
@@ -267,52 +269,40 @@ def native(args, rank, world, dev):
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         torch.cuda.nvtx.range_pop()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    max_ms = max_over_ranks(sum(step_ms), dev, world)
-    value = job_throughput(step.flops, world, args.steps, max_ms) / 1e12
-    assert S.sep_last_device_error() == 0
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        max_ms = max_over_ranks(sum(step_ms), dev, world)
+        value = job_throughput(step.flops, world, args.steps, max_ms) / 1e12
+        assert S.sep_last_device_error() == 0
 
-    if args.quick:  # timed step only (used under ncu)
-        return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-                "steps": args.steps, "ms_per_step": max_ms / args.steps, "quick": True}
-    # ---- end to end through the public API: host inputs in pinned memory, copies timed
-    e2e = e2e_run(step, args, dev, world)
+        if args.quick:  # timed step only (used under ncu)
+            clk.__exit__(None, None, None)
+            return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                    "steps": args.steps, "ms_per_step": max_ms / args.steps, "quick": True}
+        # ---- end to end through the public API: host inputs in pinned memory, copies timed
+        e2e = e2e_run(step, args, dev, world)
 
-    # ---- per-kernel breakdown (each pass alone, CUDA-graph replays of 20 launches)
-    comps = {}
-    for name, fn in step.components().items():
-        g = capture(fn, reps=20)
-        comps[name] = time_graph(g, 5, flush) / 20.0
-        del g
-    # the decode row needs the cache at full occupancy: update/decode advance it, which is fine
-    fwd_tf = step.flops_fwd / (comps["fwd_kernel"] * 1e-3) / 1e12
-    dq_flops = step.flops_fwd * 1.5 / 1.0  # S, dP, dQ products (3 of the 5 backward GEMMs x 2 / 2)
-    comp_out = {
-        "mask_build_us": comps["mask_build"] * 1e3,
-        "fwd": {"us": (comps["fwd_compact"] + comps["fwd_kernel"]) * 1e3,
-                "kernel_us": comps["fwd_kernel"] * 1e3, "tflops": fwd_tf,
-                "frac_bf16_peak": fwd_tf / peaks["bf16_tflops"]},
-        "bwd": {"us": (comps["bwd_prep"] + comps["bwd_dq"] + comps["bwd_dkdv"]) * 1e3,
-                "prep_us": comps["bwd_prep"] * 1e3, "dq_us": comps["bwd_dq"] * 1e3,
-                "dkdv_us": comps["bwd_dkdv"] * 1e3,
-                "tflops": step.flops_bwd / ((comps["bwd_prep"] + comps["bwd_dq"] + comps["bwd_dkdv"]) * 1e-3) / 1e12},
-        "decode": {"update_us": comps["decode_update"] * 1e3,
-                   "attention_us": comps["decode_attention"] * 1e3,
-                   "gbs": step.bytes_dec / (comps["decode_attention"] * 1e-3) / 1e9,
-                   "frac_hbm": step.bytes_dec / (comps["decode_attention"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-        "kept_pairs": step.kept,
-        "kept_over_dense_causal": step.kept / (step.cfg.B * step.cfg.L * (step.cfg.L + 1) / 2),
-    }
-    comp_out["bwd"]["frac_bf16_peak"] = comp_out["bwd"]["tflops"] / peaks["bf16_tflops"]
-    # dominant kernel of the step by device time
-    shares = {"fwd_kernel": comps["fwd_kernel"], "bwd_dq": comps["bwd_dq"],
-              "bwd_dkdv": comps["bwd_dkdv"], "decode_attention": comps["decode_attention"]}
-    dom = max(shares, key=shares.get)
-    roof = roofline_for(dom, comps, step, peaks, peak_src)
-    del dq_flops
+        # ---- per-kernel breakdown (each pass alone, CUDA-graph replays of 20 launches)
+        comps = {}
+        for name, fn in step.components().items():
+            g = capture(fn, reps=20)
+            comps[name] = time_graph(g, 5, flush) / 20.0
+            del g
+        # the decode row needs the cache at full occupancy: update/decode advance it, which is fine
+        comp_out = train_components(step, comps, peaks, peak_src)
+        # dominant kernel of the step by device time
+        shares = {"fwd_kernel": comps["fwd_kernel"], "bwd_dq": comps["bwd_dq"],
+                  "bwd_dkdv": comps["bwd_dkdv"], "decode_attention": comps["decode_attention"]}
+        dom = max(shares, key=shares.get)
+        roof = roofline_for(dom, comps, step, peaks, peak_src)
+        # ---- the other configurations (same kernels), one row each
+        configs = {}
+        if not args.no_configs and rank == 0:
+            configs = config_rows(S, dev, flush, peaks)
+    finally:
+        clk.__exit__(None, None, None)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -323,14 +313,228 @@ def native(args, rank, world, dev):
                               "one CUDA graph: mask build, fwd, bwd, cache update, decode"),
         "roofline": roof,
         "components": comp_out,
+        "configs": configs,
         "e2e": e2e,
         "gpu_launches": step.launches * args.steps,
-        "clocks": clk.summary(),
+        "clocks": {**clk.summary(), "window": "warm-up, timed steps, e2e and per-pass rows"},
         "peaks": {"source": peak_src, **peaks},
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
+
+
+def train_components(step, comps, peaks, peak_src):
+    """Per-pass rows of the default step: time, kept-pair TFLOP/s, tensor and combined roofline
+    fractions, and the pair slots the kernels compute per kept pair."""
+    cfg = step.cfg
+    slots = pair_slots(step.mask.gather_end.cpu(), cfg.L, cfg.n)
+    computed_over_kept = slots / step.kept
+    rows = {}
+    for name, flops in (("fwd_kernel", step.flops_fwd), ("bwd_dq", 1.5 * step.flops_fwd),
+                        ("bwd_dkdv", 2.0 * step.flops_fwd)):
+        r = roofline_for(name, comps, step, peaks, peak_src)
+        rows[name] = {"us": comps[name] * 1e3, "tflops": r["achieved"], "frac_bf16_peak": r["frac"],
+                      "algorithmic_flops": flops, "algorithmic_bytes": r["algorithmic_bytes_per_launch"],
+                      "combined_frac": r["combined_frac"], "combined_bound": r["combined_bound"],
+                      "computed_pairs_over_kept": computed_over_kept}
+    bwd_ms = comps["bwd_prep"] + comps["bwd_dq"] + comps["bwd_dkdv"]
+    dec = roofline_for("decode_attention", comps, step, peaks, peak_src)
+    return {
+        "mask_build_us": comps["mask_build"] * 1e3,
+        "fwd": {"us": (comps["fwd_compact"] + comps["fwd_kernel"]) * 1e3,
+                "compact_us": comps["fwd_compact"] * 1e3, **rows["fwd_kernel"]},
+        "bwd": {"us": bwd_ms * 1e3, "prep_us": comps["bwd_prep"] * 1e3,
+                "tflops": step.flops_bwd / (bwd_ms * 1e-3) / 1e12,
+                "frac_bf16_peak": step.flops_bwd / (bwd_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "dq": rows["bwd_dq"], "dkdv": rows["bwd_dkdv"]},
+        "decode": {"update_us": comps["decode_update"] * 1e3,
+                   "attention_us": comps["decode_attention"] * 1e3,
+                   "gbs": dec["achieved"], "frac_hbm": dec["frac"],
+                   "algorithmic_bytes": step.bytes_dec},
+        "kept_pairs": step.kept,
+        "kept_over_dense_causal": step.kept / (cfg.B * cfg.L * (cfg.L + 1) / 2),
+        "computed_pairs_over_kept": computed_over_kept,
+    }
+
+
+def device_attn_inputs(cfg, dev, n=None, with_do=True):
+    """A configuration's inputs drawn on the device generator (seeded; the same distributions
+    and flag recipe as workloads.attn_inputs, which draws on the CPU for the parity tests)."""
+    g = torch.Generator(device=dev).manual_seed(cfg.seed)
+    if cfg.flags == "bernoulli":
+        sep = (torch.rand(cfg.B, cfg.L, generator=g, device=dev) < cfg.p).to(torch.uint8)
+    else:
+        sep = workloads.separator_flags(torch.Generator().manual_seed(cfg.seed), cfg.B, cfg.L,
+                                        cfg.flags, cfg.p).to(dev)
+    if cfg.force0:
+        sep[:, 0] = 0
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    q = randn(cfg.B, cfg.L, cfg.Hq, cfg.d)
+    k = randn(cfg.B, cfg.L, cfg.Hkv, cfg.d)
+    v = randn(cfg.B, cfg.L, cfg.Hkv, cfg.d)
+    do = randn(cfg.B, cfg.L, cfg.Hq, cfg.d) if with_do else None
+    return dict(sep=sep, q=q, k=k, v=v, do=do)
+
+
+def attn_row(S, cfg, dev, flush, peaks, n, bwd, iters):
+    """Forward (and backward) of one attention configuration: device time per call, kept-pair
+    TFLOP/s, tensor and combined roofline fractions, computed pair slots per kept pair."""
+    d = device_attn_inputs(cfg, dev, with_do=bwd)
+    mask = S.sep_mask_build(d["sep"], cfg.a, n)
+    o, lse = S.sep_attn_fwd(d["q"], d["k"], d["v"], mask)
+    torch.cuda.synchronize()
+    kept = int(mask.kept.sum())
+    fl = 4.0 * cfg.d * kept * cfg.Hq
+    slots = pair_slots(mask.gather_end.cpu(), cfg.L, n)
+    ws = torch.empty(S.sep_attn_fwd_workspace_size(cfg.B, cfg.L, cfg.Hkv, cfg.d),
+                     dtype=torch.uint8, device=dev)
+    g = capture(lambda: S.sep_attn_fwd(d["q"], d["k"], d["v"], mask, out=o, lse=lse,
+                                       workspace=ws))
+    ms = time_graph(g, iters, flush)
+    del g
+    fb = attn_pass_bytes(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.d, "fwd_kernel")
+    t_f = max(fl / (peaks["bf16_tflops"] * 1e12), fb / (peaks["hbm_gbs"] * 1e9))
+    row = {"B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "L": cfg.L, "d": cfg.d, "a": cfg.a, "n": n,
+           "kept_pairs": kept, "kept_over_dense_causal": kept / (cfg.B * cfg.L * (cfg.L + 1) / 2),
+           "computed_pairs_over_kept": slots / kept,
+           "fwd_ms": ms, "fwd_tflops": fl / (ms * 1e-3) / 1e12,
+           "fwd_frac_bf16_peak": fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "fwd_combined_frac": t_f / (ms * 1e-3)}
+    if bwd:
+        wsb = torch.empty(S.sep_attn_bwd_workspace_size(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.d),
+                          dtype=torch.uint8, device=dev)
+        grads = tuple(torch.empty_like(d[x]) for x in ("q", "k", "v"))
+        g = capture(lambda: S.sep_attn_bwd(d["q"], d["k"], d["v"], o, lse, d["do"], mask,
+                                           workspace=wsb, grads=grads))
+        ms = time_graph(g, iters, flush)
+        del g, wsb, grads
+        row.update({"bwd_ms": ms, "bwd_tflops": 2.5 * fl / (ms * 1e-3) / 1e12,
+                    "bwd_frac_bf16_peak": 2.5 * fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"]})
+    assert S.sep_last_device_error() == 0
+    return row
+
+
+def decode_loop_row(S, dev, peaks, first=2048, steps=63488, chunk=1024):
+    """The SepCache decode configuration as a stream: 64 sequences, steps first..first+steps-1
+    of the 65536-step run (the cache is full from then on), update + decode per step, chunk
+    steps per CUDA-graph replay on the device-drawn input stream; steps run back to back."""
+    dc = workloads.SEPCACHE_DECODE
+    cache = S.SepCache(dc.S, dc.Hq, dc.Hkv, dc.d, dc.a, dc.s, dc.w, dc.theta, device=dev)
+    o = torch.empty(dc.S, dc.Hq, dc.d, dtype=torch.bfloat16, device=dev)
+    # steps 0 .. first - chunk - 1 directly, the chunk before `first` through the capture's own
+    # warm-up call, then the timed chunks replay the graph on their inputs
+    for c0 in range(0, first - chunk, chunk):
+        x = workloads.decode_chunk(dc, c0, chunk, device=dev)
+        for t in range(chunk):
+            cache.sepcache_update(x["k"][t], x["v"][t], x["sep"][t])
+            cache.sepcache_decode(x["q"][t], out=o)
+    buf = workloads.decode_chunk(dc, first - chunk, chunk, device=dev)
+
+    def run():
+        for t in range(chunk):
+            cache.sepcache_update(buf["k"][t], buf["v"][t], buf["sep"][t])
+            cache.sepcache_decode(buf["q"][t], out=o)
+    g = capture(run)
+    m = cache.meta.cpu()
+    occ = (m[:, 1] + m[:, 3] + m[:, 5]).tolist()
+    full = all(v == dc.c for v in occ)
+    total_ms = 0.0
+    st = torch.cuda.current_stream()
+    for c0 in range(first, first + steps, chunk):
+        x = workloads.decode_chunk(dc, c0, chunk, device=dev)
+        for key in buf:
+            buf[key].copy_(x[key])
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        g.replay()
+        e1.record(st)
+        e1.synchronize()
+        total_ms += e0.elapsed_time(e1)
+    assert S.sep_last_device_error() == 0
+    us = total_ms * 1e3 / steps
+    byts = dc.S * (dc.c * dc.Hkv * dc.d * 2 * 2 + 2 * dc.Hq * dc.d * 2 + dc.Hkv * dc.d * 2 * 2)
+    return {"sequences": dc.S, "steps_timed": steps, "first_step": first, "occupancy": dc.c,
+            "cache_full_at_first_step": full, "us_per_step": us,
+            "tokens_per_s": dc.S / (us * 1e-6), "bytes_per_step": byts,
+            "gbs": byts / (us * 1e-6) / 1e9, "frac_hbm": byts / (us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+            "l2": "steps back to back (the 210 MB cache exceeds the 126 MB L2)"}
+
+
+def config_rows(S, dev, flush, peaks):
+    """The other configurations through the same kernels, one row each."""
+    rows = {}
+    rows["llama3-8b-prefill"] = attn_row(S, workloads.LLAMA3_8B_PREFILL, dev, flush, peaks,
+                                         workloads.LLAMA3_8B_PREFILL.n, False, 10)
+    torch.cuda.empty_cache()
+    lc = workloads.LONG_CONTEXT
+    rows["long-context"] = attn_row(S, lc, dev, flush, peaks, lc.n, True, 3)
+    torch.cuda.empty_cache()
+    rows["long-context-all-keep"] = attn_row(S, lc, dev, flush, peaks, lc.L, True, 2)
+    torch.cuda.empty_cache()
+    rows["sepcache-decode-stream"] = decode_loop_row(S, dev, peaks)
+    torch.cuda.empty_cache()
+    for r in rows.values():
+        r["inputs"] = "seeded, drawn on the device generator"
+    return rows
+
+
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "dram_traffic.json")
+CSRC = os.path.join(ROOT, "kv_cache_compression_sep_b200", "csrc")
+
+
+def source_digest(fname):
+    """sha256 (first 16 hex digits) of one kernel source file of the library."""
+    import hashlib
+    with open(os.path.join(CSRC, fname), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def load_traffic(name):
+    """DRAM bytes per launch of a pass (dram__bytes_read.sum + dram__bytes_write.sum) from the
+    committed ncu capture table, or None when no capture covers the pass or the kernel's source
+    file changed after the capture (the counters then describe another kernel)."""
+    if not os.path.exists(TRAFFIC_JSON):
+        return None
+    with open(TRAFFIC_JSON) as fh:
+        table = json.load(fh)
+    e = table.get("passes", {}).get(name)
+    if not e:
+        return None
+    try:
+        if source_digest(e["source"]) != e["source_sha256"]:
+            return None
+    except OSError:
+        return None
+    return int(e["bytes_per_launch"])
+
+
+def attn_pass_bytes(B, L, Hq, Hkv, d, name):
+    """Algorithmic HBM bytes of one attention pass: every input read once, every output written
+    once (bf16 tensors, fp32 LSE and Delta); scratch traffic is not counted."""
+    q = B * L * Hq * d * 2
+    kv = B * L * Hkv * d * 2
+    st = B * Hq * L * 4
+    return {"fwd_kernel": q + 2 * kv + q + st,             # Q, K, V -> O, LSE
+            "bwd_dq": 2 * q + 2 * kv + 2 * st + q,         # Q, dO, K, V, LSE, Delta -> dQ
+            "bwd_dkdv": 2 * q + 2 * kv + 2 * st + 2 * kv}[name]  # ... -> dK, dV
+
+
+def pair_slots(gather_end, L, n):
+    """Query-key pair slots the attention kernels compute per head (summed over the batch):
+    every query tile t runs whole 128 x 128 tiles over its window key tiles lo(t)..t and over
+    ceil(gather_end[t] / 128) compacted anchor chunks. Identical for the forward, the dQ pass
+    and the dK/dV pass (the latter visits the same (query tile, key unit) pairs key-major)."""
+    import numpy as np
+    ge = np.asarray(gather_end, dtype=np.int64)
+    T = ge.shape[-1]
+    t = np.arange(T)
+    lo = np.maximum(0, 128 * t - n + 1) // 128
+    tiles = (t - lo + 1)[None, :] + (ge + 127) // 128
+    return int(tiles.sum()) * 128 * 128
 
 
 def roofline_for(name, comps, step, peaks, peak_src):
@@ -347,22 +551,18 @@ def roofline_for(name, comps, step, peaks, peak_src):
     kname = {"fwd_kernel": "sep_attn_fwd_kernel", "bwd_dq": "sep_attn_bwd_dq_kernel",
              "bwd_dkdv": "sep_attn_bwd_dkv_kernel"}[name]
     ach = flops / (ms * 1e-3) / 1e12
-    return {"kernel": kname, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
-            "peak_source": peak_src, "algorithmic_flops_per_launch": flops}
-
-
-def load_traffic(name):
-    """DRAM bytes per launch from the committed ncu summary table, if a row covers this pass."""
-    p = os.path.join(ROOT, "profiles", "traffic.md")
-    if not os.path.exists(p):
-        return None
-    with open(p) as fh:
-        for ln in fh:
-            cells = [c.strip() for c in ln.strip().strip("|").split("|")]
-            if len(cells) >= 3 and cells[0] == name and cells[2].isdigit():
-                return int(cells[2])
-    return None
+    out = {"kernel": kname, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+           "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": traffic,
+           "peak_source": peak_src, "algorithmic_flops_per_launch": flops}
+    cfg = getattr(step, "cfg", None)
+    if cfg is not None:
+        byts = attn_pass_bytes(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.d, name)
+        t_min = max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9))
+        out.update({"algorithmic_bytes_per_launch": byts,
+                    "combined_frac": t_min / (ms * 1e-3),
+                    "combined_bound": "hbm" if byts / (peaks["hbm_gbs"] * 1e9) >
+                    flops / (peaks["bf16_tflops"] * 1e12) else "tensor"})
+    return out
 
 
 def e2e_run(step, args, dev, world):
@@ -692,6 +892,8 @@ def main():
                              "cache-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the Llama prefill, long-context and decode-stream rows")
     ap.add_argument("--quick", action="store_true",
                     help="timed step only: no e2e, breakdown or CPU baseline (for ncu runs)")
     args = ap.parse_args()

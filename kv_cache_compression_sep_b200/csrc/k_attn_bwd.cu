@@ -14,9 +14,9 @@
 //   2. dQ (query-major, persistent over the forward's item order and key tiles): S = Q K^T and
 //      dP = dO V^T into TMEM, dS = P (dP - Delta) written back to TMEM as bf16,
 //      dQ += dS K (A from TMEM, B = K MN-major); a storer warp writes the dQ tile.
-//   3. dK/dV (key-major, persistent, items fetched dynamically): work items are window key
-//      tiles u (query tiles t with lo(t) <= u <= t) and (anchor chunk c, segment of query tiles
-//      that gather it). Per (query tile, query head), in two 64-row query halves:
+//   3. dK/dV (key-major, persistent, items fetched dynamically, heaviest first): work items
+//      are window key tiles u (all query tiles t with lo(t) <= u <= t) and (anchor chunk c,
+//      segment of query tiles that gather it). Per (query tile, query head), in two 64-row query halves:
 //      S^T = K Q^T, dP^T = V dO^T into TMEM; P^T and dS^T back to TMEM as bf16;
 //      dV += P^T dO, dK += dS^T Q. Non-anchor keys of a window tile get their complete gradient
 //      and leave as bf16 through a storer warp's TMA store; anchor keys are summed in fp32
@@ -38,13 +38,13 @@ constexpr int kBoxBytes = 128 * 64 * 2;
 //   position i are Hq * d contiguous bf16: 16-byte chunks, D / 8 consecutive chunks per head,
 //   summed over the D / 8 lanes that hold them);
 //   row i of the compacted anchor K / V (i < roundup128(cnt));
-//   zero row i of the compact fp32 anchor partials (i < cnt, direct mode);
+//   zero row i of the compact fp32 anchor partials (i < cnt);
 //   and the four work-list counters (block 0).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const uint4* __restrict__ o, const uint4* __restrict__ dout, const uint4* __restrict__ k,
     const uint4* __restrict__ v, const int32_t* __restrict__ anchor_idx,
-    const int32_t* __restrict__ anchor_cnt, int L, int Hq, int Hkv, int zero_partials,
+    const int32_t* __restrict__ anchor_cnt, int L, int Hq, int Hkv,
     uint4* __restrict__ kc, uint4* __restrict__ vc, float4* __restrict__ dka,
     float4* __restrict__ dva, float* __restrict__ delta, int32_t* __restrict__ counters) {
   constexpr int CPH = D / 8;  // 16-byte chunks per head; divides 32
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
   const int cnt = __ldg(anchor_cnt + b);
   if (i < min(L, (cnt + 127) / 128 * 128))
     compact_anchor_row(k, v, anchor_idx, cnt, L, b, i, Hkv * D / 8, kc, vc, lane);
-  if (zero_partials && i < cnt) {
+  if (i < cnt) {
     const int pc = Hkv * D / 4;
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c = lane; c < pc; c += 32) {
@@ -528,10 +528,13 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
 
 // ------------------------------------------------------------------ dK/dV work list
 // Items of the key-major pass, one per (key unit, segment of query tiles):
-//   window item: key tile u of batch b with query tiles t_begin..t_end-1 (those whose window key
-//                tiles lo(t)..t contain u), split into segments of at most kSegT tiles;
+//   window item: key tile u of batch b with every query tile t whose window key tiles lo(t)..t
+//                contain u (t_begin = u .. t_end - 1), so that its non-anchor keys get their
+//                complete gradient in one item; at position u * B + b, so that the list runs
+//                from the largest key range (u = 0 under dense causal) to the smallest;
 //   anchor item: compacted anchor chunk c (anchors 128c..128c+127) with the query tiles that
-//                gather it (gather_end[t] > 128c), in segments of kSegT tiles.
+//                gather it (gather_end[t] > 128c), in segments of kSegT tiles (their fp32 partial
+//                sums are added atomically).
 // Every kv head processes every item. Built on the device by bwd_schedule_kernel.
 constexpr int kSegT = 16;
 
@@ -605,17 +608,17 @@ __global__ void __launch_bounds__(1024) bwd_schedule_kernel(
       }
     }
   }
-  // ---- window items: query tiles t with lo(t) <= u <= t, in segments
+  // ---- window items: query tiles t with lo(t) <= u <= t; lo is non-decreasing in t, so the
+  // last such t is found by binary search
   for (int u = tid; u < T; u += blockDim.x) {
-    int te = u + 1;
-    while (te < T && window_lo_tile(te, n) <= u) ++te;
-    const int nseg = (te - u + kSegT - 1) / kSegT;
-    const int at = atomicAdd(&counters[1], nseg);
-    for (int sg = 0; sg < nseg; ++sg) {
-      const int t0 = u + sg * kSegT;
-      window_items[at + sg] = WorkItem{b, u, t0, min(te, t0 + kSegT)};
+    int lo = u + 1, hi = T;  // first t > u with lo(t) > u
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (window_lo_tile(mid, n) > u) hi = mid; else lo = mid + 1;
     }
+    window_items[(size_t)u * gridDim.x + b] = WorkItem{b, u, u, lo};
   }
+  if (tid == 0) atomicAdd(&counters[1], T);
 }
 
 // ------------------------------------------------------------------ dK/dV kernel
@@ -626,11 +629,10 @@ __global__ void __launch_bounds__(1024) bwd_schedule_kernel(
 //   P^T = exp2(S^T c - lse2), dS^T = P^T (dP^T - Delta), written over S^T_h / dP^T_h as bf16
 //   dV += P^T_h dO_h, dK += dS^T_h Q_h             (A from TMEM, B MN-major in smem)
 // The MMA warp issues one half's S^T/dP^T while the other half's softmax runs. dV and dK stay
-// in TMEM for the whole item. Epilogue, with `direct` set (every window item covers all query
-// tiles of its key tile): non-anchor rows are final and leave as bf16 through shared memory and
-// a TMA store; anchor rows add their fp32 window part into the compact anchor partials. Anchor
-// items add into the compact partials. Without `direct` (long windows split into segments) every
-// row adds into position-indexed fp32 accumulators.
+// in TMEM for the whole item. Epilogue: every window item covers all query tiles of its key
+// tile, so its non-anchor rows are final and leave as bf16 through shared memory and a TMA
+// store; anchor rows add their fp32 window part into the compact anchor partials, and anchor
+// items add into the compact partials too.
 template <int D>
 struct DkvCfg {
   static constexpr int KB = D / 64;
@@ -689,7 +691,7 @@ template <int D>
 __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     sep_attn_bwd_dkv_kernel(const __grid_constant__ BwdParams p, const WorkItem* __restrict__ aitems,
                             const WorkItem* __restrict__ witems, int32_t* __restrict__ counters,
-                            const int32_t* __restrict__ tile_prefix, int direct) {
+                            const int32_t* __restrict__ tile_prefix) {
   using C = DkvCfg<D>;
   constexpr int NST = C::NST, KVB = C::KVB;
   const int G = p.Hq / p.Hkv;
@@ -912,7 +914,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     }
   } else if (warp == 10) {
     // ---------------------------------------------------------------- dK/dV storer
-    // Per item, once the softmax warps have staged it: the bf16 rows of a direct-mode window
+    // Per item, once the softmax warps have staged it: the bf16 rows of a window
     // item leave by TMA store from the item's K/V buffer; then the buffer is released.
     if (lane == 0) {
       for (int I = 0;; ++I) {
@@ -922,7 +924,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
         const int kb = I % KVB;
         if (!mbar_wait(&bar->staged[kb], (I / KVB) & 1, p.err, abort_flag)) break;
-        if (direct && it.window) {
+        if (it.window) {
           for (int z = 0; z < C::KB; ++z) {
             tma_store_4d(&p.tmdV, sV + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
             tma_store_4d(&p.tmdK, sK + kb * C::TILE + z * kBoxBytes, z * 64, it.kvh, it.unit * 128, it.b);
@@ -1065,28 +1067,21 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       const float mul = h ? p.scale : 1.f;
       const uint32_t col0 = h ? C::COL_DK : C::COL_DV;
       float* part = h ? p.dka : p.dva;
-      long long dst_row = -1;  // fp32 accumulator row, or -1
-      bool stage_row = false;
-      if (direct) {
-        if (it.window) {
-          stage_row = true;
-          if (fj) {
-            int before = pre_tile;
+      // compact anchor row that takes this row's fp32 sums, or -1; non-anchor rows of a window
+      // item are final and are staged for the TMA store
+      long long dst_row = -1;
+      const bool stage_row = it.window;
+      if (it.window) {
+        if (fj) {
+          int before = pre_tile;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q < (krow >> 5)) before += __popc(tile_words[q]);
-            before += __popc(tile_words[krow >> 5] & ((1u << (krow & 31)) - 1u));
-            dst_row = before;
-          }
-        } else if (r < cnt_b) {
-          dst_row = r;
+          for (int q = 0; q < 4; ++q)
+            if (q < (krow >> 5)) before += __popc(tile_words[q]);
+          before += __popc(tile_words[krow >> 5] & ((1u << (krow & 31)) - 1u));
+          dst_row = before;
         }
-      } else {
-        if (it.window) {
-          if (j < p.L) dst_row = j;
-        } else if (r < cnt_b) {
-          dst_row = p.anchor_idx[(size_t)it.b * p.L + r];
-        }
+      } else if (r < cnt_b) {
+        dst_row = r;
       }
       float* dst = dst_row >= 0 ? part + (((size_t)it.b * p.L + dst_row) * p.Hkv + it.kvh) * D : nullptr;
       uint8_t* stage = (h ? sK : sV) + kb * C::TILE;
@@ -1137,19 +1132,6 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       atomicExch(&counters[2], 0);
       atomicExch(&counters[3], 0);
     }
-  }
-}
-
-// Position-indexed fp32 accumulators to bf16 dK / dV (used when window items are segmented).
-__global__ void __launch_bounds__(256) acc_to_bf16_kernel(const float4* __restrict__ dka,
-                                                          const float4* __restrict__ dva,
-                                                          long long n4, uint2* __restrict__ dk,
-                                                          uint2* __restrict__ dv) {
-  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n4;
-       e += (long long)gridDim.x * blockDim.x) {
-    const float4 x = dka[e], y = dva[e];
-    dk[e] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
-    dv[e] = make_uint2(pack_bf16x2(y.x, y.y), pack_bf16x2(y.z, y.w));
   }
 }
 
@@ -1222,9 +1204,6 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   (void)tile_map;
   cudaError_t e = cudaSuccess;
   const int T = (s.L + 127) / 128, W = (s.L + 31) / 32;
-  // window items are single segments (direct dK/dV stores) unless windows span > kSegT tiles
-  const int win_tiles = (s.n - 1 + 127) / 128 + 1;
-  const int direct = (win_tiles <= kSegT || T <= kSegT) ? 1 : 0;
   // schedule region: counters, tile prefix counts, anchor items, window items
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t cap = (size_t)s.B * T * ((T + kSegT - 1) / kSegT);
@@ -1233,18 +1212,13 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   int32_t* tile_prefix = reinterpret_cast<int32_t*>(sw + up(4 * sizeof(int32_t)));
   WorkItem* aitems = reinterpret_cast<WorkItem*>(sw + up(4 * sizeof(int32_t)) + up((size_t)s.B * T * sizeof(int32_t)));
   WorkItem* witems = aitems + up(cap * sizeof(WorkItem)) / sizeof(WorkItem);
-  const size_t acc_bytes = (size_t)s.B * s.L * s.Hkv * s.d * sizeof(float);
 
   if (stages & kBwdPrep) {
-    if (!direct) {
-      if ((e = cudaMemsetAsync(dka, 0, acc_bytes, stream)) != cudaSuccess) return e;
-      if ((e = cudaMemsetAsync(dva, 0, acc_bytes, stream)) != cudaSuccess) return e;
-    }
     const dim3 pgrid((s.L + 7) / 8, s.B);
     auto prep = (s.d == 128) ? bwd_prep_kernel<128> : bwd_prep_kernel<64>;
     prep<<<pgrid, 256, 0, stream>>>(
         static_cast<const uint4*>(o), static_cast<const uint4*>(dout), static_cast<const uint4*>(k),
-        static_cast<const uint4*>(v), anchor_idx, anchor_cnt, s.L, s.Hq, s.Hkv, direct,
+        static_cast<const uint4*>(v), anchor_idx, anchor_cnt, s.L, s.Hq, s.Hkv,
         static_cast<uint4*>(kc), static_cast<uint4*>(vc), reinterpret_cast<float4*>(dka),
         reinterpret_cast<float4*>(dva), delta, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1296,7 +1270,7 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (stages & kBwdDkv)
       sep_attn_bwd_dkv_kernel<128><<<nsm, DkvCfg<128>::THREADS, dkv_smem_bytes<128>(), stream>>>(
-          prm, aitems, witems, counters, tile_prefix, direct);
+          prm, aitems, witems, counters, tile_prefix);
   } else {
     if ((e = set_bwd_attrs<64>()) != cudaSuccess) return e;
     if (stages & kBwdDq)
@@ -1304,21 +1278,14 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (stages & kBwdDkv)
       sep_attn_bwd_dkv_kernel<64><<<nsm, DkvCfg<64>::THREADS, dkv_smem_bytes<64>(), stream>>>(
-          prm, aitems, witems, counters, tile_prefix, direct);
+          prm, aitems, witems, counters, tile_prefix);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (stages & kBwdDkv) {
-    if (direct) {
-      dim3 grid((s.L + 7) / 8, s.B);
-      anchor_combine_kernel<<<grid, 256, 0, stream>>>(
-          anchor_idx, anchor_cnt, s.L, s.Hkv * s.d / 4, reinterpret_cast<const float4*>(dka),
-          reinterpret_cast<const float4*>(dva), static_cast<uint2*>(dk), static_cast<uint2*>(dv));
-    } else {
-      const long long n4 = (long long)s.B * s.L * s.Hkv * s.d / 4;
-      acc_to_bf16_kernel<<<nsm * 8, 256, 0, stream>>>(
-          reinterpret_cast<const float4*>(dka), reinterpret_cast<const float4*>(dva), n4,
-          static_cast<uint2*>(dk), static_cast<uint2*>(dv));
-    }
+    dim3 grid((s.L + 7) / 8, s.B);
+    anchor_combine_kernel<<<grid, 256, 0, stream>>>(
+        anchor_idx, anchor_cnt, s.L, s.Hkv * s.d / 4, reinterpret_cast<const float4*>(dka),
+        reinterpret_cast<const float4*>(dva), static_cast<uint2*>(dk), static_cast<uint2*>(dv));
   }
   return cudaGetLastError();
 }

@@ -25,7 +25,8 @@
 // rotating every key at every step. A key is rotated by RoPE(t) when it is appended and, when it
 // enters the separator FIFO, re-rotated by RoPE(A - t). Without positional shifting
 // (original_positions) keys stay at RoPE(t) and every block's query angle is its own position.
-// Angles are formed in fp64 (position x inverse frequency), rotations are rounded once to bf16.
+// Angles are formed and reduced in fp64 (position x inverse frequency), rotations are rounded to
+// bf16.
 //
 // Decode: one CTA per (sequence, KV head), all resident in one wave. Bulk copies stream the
 // retained K/V rows in rank order through a shared-memory ring; a group of D/8 lanes takes one
@@ -41,8 +42,19 @@
 namespace sep {
 
 // ------------------------------------------------------------------ RoPE of stored keys
+// (cos, sin) of the angle pos * f: the angle is formed in fp64 and reduced to [-pi, pi] by
+// subtracting the nearest multiple of 2 pi (fp64), then the fp32 sincosf of the reduced angle is
+// taken. The error (about 1e-7 absolute, from rounding the reduced angle to fp32) is far below the
+// bf16 rounding of the rotated keys, and positions up to 2^31 keep full precision.
+__device__ __forceinline__ void rope_cos_sin(long long pos, double f, float* cs, float* sn) {
+  constexpr double kTwoPi = 6.283185307179586, kInvTwoPi = 0.15915494309189535;
+  const double x = __dmul_rn((double)pos, f);
+  const double r = __fma_rn(-rint(__dmul_rn(x, kInvTwoPi)), kTwoPi, x);
+  sincosf((float)r, sn, cs);
+}
+
 // Rotate-half pairs (k, k + d/2), angle pos * freq[k], freq[k] = theta^(-2k/d) (fp64 table).
-// x holds dims k0..k0+7, y dims k0+d/2..k0+d/2+7 of one key row; fp64 arithmetic with the
+// x holds dims k0..k0+7, y dims k0+d/2..k0+d/2+7 of one key row; fp32 arithmetic with the
 // operations spelled out (no contraction choices left to the compiler), rounded to bf16, so that
 // every kernel that rotates the same row by the same angle produces the same bits.
 __device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, long long pos,
@@ -53,15 +65,15 @@ __device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, l
   for (int q = 0; q < 4; ++q) {
     const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&xs[q]);
     const __nv_bfloat162 ya = *reinterpret_cast<const __nv_bfloat162*>(&ys[q]);
-    const double xv[2] = {(double)__low2float(xa), (double)__high2float(xa)};
-    const double yv[2] = {(double)__low2float(ya), (double)__high2float(ya)};
+    const float xv[2] = {__low2float(xa), __high2float(xa)};
+    const float yv[2] = {__low2float(ya), __high2float(ya)};
     __nv_bfloat16 xo[2], yo[2];
 #pragma unroll
     for (int z = 0; z < 2; ++z) {
-      double sn, cs;
-      sincos(__dmul_rn((double)pos, __ldg(freq + k0 + 2 * q + z)), &sn, &cs);
-      xo[z] = __double2bfloat16(__fma_rn(xv[z], cs, -__dmul_rn(yv[z], sn)));
-      yo[z] = __double2bfloat16(__fma_rn(yv[z], cs, __dmul_rn(xv[z], sn)));
+      float sn, cs;
+      rope_cos_sin(pos, __ldg(freq + k0 + 2 * q + z), &cs, &sn);
+      xo[z] = __float2bfloat16_rn(__fmaf_rn(xv[z], cs, -__fmul_rn(yv[z], sn)));
+      yo[z] = __float2bfloat16_rn(__fmaf_rn(yv[z], cs, __fmul_rn(xv[z], sn)));
     }
     const __nv_bfloat162 xp = __halves2bfloat162(xo[0], xo[1]);
     const __nv_bfloat162 yp = __halves2bfloat162(yo[0], yo[1]);
@@ -467,9 +479,12 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
 
 // ------------------------------------------------------------------ decode
 // Lane groups: LPK = D / 8 lanes per key row, 8 contiguous elements per lane; NG = 128 / LPK
-// groups per CTA, each taking two rows of every KC = 2 NG row chunk.
+// groups per CTA, each taking kDecRows rows of every KC = kDecRows NG row chunk (four
+// independent rows per group and stage give each warp enough work between ring waits), in a
+// ring of three chunks.
 constexpr int kDecThreads = 128;
-constexpr int kDecStages = 4;
+constexpr int kDecStages = 3;
+constexpr int kDecRows = 4;
 constexpr int kDecWarps = kDecThreads / 32;
 
 template <int N>
@@ -526,7 +541,7 @@ template <int D, int GP>
 struct DecCfg {
   static constexpr int LPK = D / 8;
   static constexpr int NG = kDecThreads / LPK;
-  static constexpr int KC = 2 * NG;  // rows per ring stage
+  static constexpr int KC = kDecRows * NG;  // rows per ring stage
   static constexpr int RING_BYTES = kDecStages * KC * D * 2 * 2;
   static constexpr int COMB_BYTES = kDecWarps * GP * D * 4;  // per-warp V sums at the end
   static constexpr int BUF_BYTES = RING_BYTES > COMB_BYTES ? RING_BYTES : COMB_BYTES;
@@ -639,17 +654,17 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
     qpos[2] = (long long)T - 1;
     for (int e = tid; e < 3 * HALF; e += kDecThreads) {
       const int blk = e / HALF, k = e % HALF;
-      double sn, cs;
-      sincos(__dmul_rn((double)qpos[blk], __ldg(p.freq + k)), &sn, &cs);
+      float sn, cs;
+      rope_cos_sin(qpos[blk], __ldg(p.freq + k), &cs, &sn);
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float r1 = 0.f, r2 = 0.f;
         if (g < p.G) {
           const __nv_bfloat16* qh = p.q + ((size_t)seq * p.Hq + kvh * p.G + g) * D;
-          const double x1 = (double)__bfloat162float(qh[k]);
-          const double x2 = (double)__bfloat162float(qh[k + HALF]);
-          r1 = (float)(x1 * cs - x2 * sn) * p.scale_log2;
-          r2 = (float)(x2 * cs + x1 * sn) * p.scale_log2;
+          const float x1 = __bfloat162float(qh[k]);
+          const float x2 = __bfloat162float(qh[k + HALF]);
+          r1 = (x1 * cs - x2 * sn) * p.scale_log2;
+          r2 = (x2 * cs + x1 * sn) * p.scale_log2;
         }
         sm.qrot[blk][g][k] = r1;
         sm.qrot[blk][g][k + HALF] = r2;
@@ -658,7 +673,7 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
   }
   __syncthreads();
 
-  // ---- consumers: group grp takes rows grp and grp + NG of every chunk
+  // ---- consumers: group grp takes rows grp, grp + NG, ... of every chunk
   float2 qr[GP][4];   // this lane's 8 query elements (as pairs) of the current block
   float2 acc[GP][4];  // V sums of every query over this lane's 8 elements
   float m_own = -INFINITY, l_own = 0.f;  // softmax state of this lane's own query
@@ -677,7 +692,7 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
     }
     const int c0 = ch * KC;
 #pragma unroll
-    for (int sub = 0; sub < 2; ++sub) {
+    for (int sub = 0; sub < kDecRows; ++sub) {
       const int row = sub * NG + grp;
       const int r = c0 + row;
       const bool valid = r < occ;

@@ -134,6 +134,21 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
     s_oldsep = slot_sep[(size_t)seq * ns + win_base + wh];
     s_oldpos = slot_pos[(size_t)seq * ns + win_base + wh];
   }
+  // this thread's first share of the new token (K rotated at its position t, V), fetched and
+  // rotated while the step is planned: it depends on t only, not on the plan
+  const int vec = d / 8;   // 16-byte vectors per row
+  const int hv = vec / 2;  // vectors per RoPE half
+  uint4 nkx = make_uint4(0u, 0u, 0u, 0u), nky = nkx, nv = nkx;
+  {
+    const int t_new = m[SEPCACHE_META_T];
+    if (tid < Hkv * hv) {
+      const size_t src = ((size_t)seq * Hkv + tid / hv) * vec + tid % hv;
+      nkx = k_new[src];
+      nky = k_new[src + hv];
+      rope_rotate_chunks(nkx, nky, 8 * (tid % hv), t_new, freq);
+    }
+    if (tid < Hkv * vec) nv = v_new[(size_t)seq * Hkv * vec + tid];
+  }
   __syncthreads();
   if (tid == 0) {
     const int t = s_meta[SEPCACHE_META_T];
@@ -194,8 +209,6 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
   }
   __syncthreads();
   const int slot_new = plan[0], move_from = plan[1], move_to = plan[2], t = plan[3];
-  const int vec = d / 8;  // 16-byte vectors per row
-  const int hv = vec / 2; // vectors per RoPE half
   const size_t seq_rows = (size_t)seq * Hkv * ns;
   // move a row (all heads, all threads): V copied, K re-rotated by `angle` on the way
   auto move_row = [&](int from, int to, int angle) {
@@ -222,19 +235,24 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
     }
     __syncthreads();
   }
-  // the new token: K rotated at its original position t
+  // the new token: K rotated at its original position t (the first share was prepared above)
   for (int e = tid; e < Hkv * hv; e += kUpdateThreads) {
     const int hh = e / hv, q = e % hv;
     const size_t dst = (seq_rows + (size_t)hh * ns + slot_new) * vec + q;
-    const size_t src = ((size_t)seq * Hkv + hh) * vec + q;
-    uint4 x = k_new[src], y = k_new[src + hv];
-    rope_rotate_chunks(x, y, 8 * q, t, freq);
+    uint4 x = nkx, y = nky;
+    if (e != tid) {
+      const size_t src = ((size_t)seq * Hkv + hh) * vec + q;
+      x = k_new[src];
+      y = k_new[src + hv];
+      rope_rotate_chunks(x, y, 8 * q, t, freq);
+    }
     k_slots[dst] = x;
     k_slots[dst + hv] = y;
   }
   for (int e = tid; e < Hkv * vec; e += kUpdateThreads) {
     const int hh = e / vec, q = e % vec;
-    v_slots[(seq_rows + (size_t)hh * ns + slot_new) * vec + q] = v_new[((size_t)seq * Hkv + hh) * vec + q];
+    v_slots[(seq_rows + (size_t)hh * ns + slot_new) * vec + q] =
+        (e == tid) ? nv : v_new[((size_t)seq * Hkv + hh) * vec + q];
   }
   if (tid == 0) {
     slot_pos[(size_t)seq * ns + slot_new] = t;

@@ -46,6 +46,14 @@ struct FwdParams {
   float scale_log2;
 };
 
+// Every kFwdEx2FmaPeriod-th pair of scores of the softmax takes its exp2 on the FMA pipe
+// (ex2_fma2) instead of the XU pipe: 74.7 -> 71.3 us for the Pythia-160m forward with a quarter
+// moved (a third: 72.2 us, a half: 73.9 us).
+#ifndef SEP_FWD_EX2_FMA_PERIOD
+#define SEP_FWD_EX2_FMA_PERIOD 4
+#endif
+constexpr int kFwdEx2FmaPeriod = SEP_FWD_EX2_FMA_PERIOD;
+
 template <int D>
 struct FwdCfg {
   static constexpr int BM = 128, BN = 128;
@@ -451,7 +459,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int c = 0; c < 64; c += 2) {
           const float2 x = f2_fma(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
                                   sl2x2, nm2);
-          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          // every kFwdEx2FmaPeriod-th pair on the FMA pipe, the rest on the XU pipe
+          const float2 e = (kFwdEx2FmaPeriod > 0 &&
+                            (c >> 1) % (kFwdEx2FmaPeriod > 0 ? kFwdEx2FmaPeriod : 1) ==
+                                kFwdEx2FmaPeriod - 1)
+                               ? ex2_fma2(x)
+                               : make_float2(ex2(x.x), ex2(x.y));
           sum4[(c >> 1) & 3] = f2_add(sum4[(c >> 1) & 3], e);
           s[c >> 1] = pack_bf16x2(e.x, e.y);
         }

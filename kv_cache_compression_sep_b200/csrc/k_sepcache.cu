@@ -54,12 +54,21 @@ __device__ __forceinline__ void rope_cos_sin(long long pos, double f, float* cs,
 }
 
 // Rotate-half pairs (k, k + d/2), angle pos * freq[k], freq[k] = theta^(-2k/d) (fp64 table).
-// x holds dims k0..k0+7, y dims k0+d/2..k0+d/2+7 of one key row; fp32 arithmetic with the
-// operations spelled out (no contraction choices left to the compiler), rounded to bf16, so that
-// every kernel that rotates the same row by the same angle produces the same bits.
-__device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, long long pos,
-                                                   const double* __restrict__ freq) {
-  if (pos == 0) return;
+// x holds dims k0..k0+7, y dims k0+d/2..k0+d/2+7 of one key row. The (cos, sin) of the 8 pairs
+// come from rope_cos_sin (rope_chunk_cs); the rotation is fp32 arithmetic with the operations
+// spelled out (no contraction choices left to the compiler), rounded to bf16, so that every
+// kernel that rotates the same row by the same angle produces the same bits.
+struct ChunkCS {
+  float c[8], s[8];
+};
+__device__ __forceinline__ ChunkCS rope_chunk_cs(int k0, long long pos,
+                                                 const double* __restrict__ freq) {
+  ChunkCS r;
+#pragma unroll
+  for (int z = 0; z < 8; ++z) rope_cos_sin(pos, __ldg(freq + k0 + z), &r.c[z], &r.s[z]);
+  return r;
+}
+__device__ __forceinline__ void rope_apply_chunks(uint4& x, uint4& y, const ChunkCS& r) {
   uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -70,8 +79,7 @@ __device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, l
     __nv_bfloat16 xo[2], yo[2];
 #pragma unroll
     for (int z = 0; z < 2; ++z) {
-      float sn, cs;
-      rope_cos_sin(pos, __ldg(freq + k0 + 2 * q + z), &cs, &sn);
+      const float cs = r.c[2 * q + z], sn = r.s[2 * q + z];
       xo[z] = __float2bfloat16_rn(__fmaf_rn(xv[z], cs, -__fmul_rn(yv[z], sn)));
       yo[z] = __float2bfloat16_rn(__fmaf_rn(yv[z], cs, __fmul_rn(xv[z], sn)));
     }
@@ -82,6 +90,11 @@ __device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, l
   }
   x = make_uint4(xs[0], xs[1], xs[2], xs[3]);
   y = make_uint4(ys[0], ys[1], ys[2], ys[3]);
+}
+__device__ __forceinline__ void rope_rotate_chunks(uint4& x, uint4& y, int k0, long long pos,
+                                                   const double* __restrict__ freq) {
+  if (pos == 0) return;
+  rope_apply_chunks(x, y, rope_chunk_cs(k0, pos, freq));
 }
 
 // ------------------------------------------------------------------ init
@@ -335,13 +348,15 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
 //   tokens triggers a compression, so run boundaries follow the recurrence
 //   e <- e + need(sep_cnt), sep_cnt <- min(s, sep_cnt + separators in the run), as long as a
 //   run has left the window entirely; tokens [e_end, L - nwin) are the past window.
-// One CTA per (sequence, KV head): each finds e_end and the separator count (block-wide counts),
-// scans the flags to place the kept separators, copies and rotates its head's K/V rows; the
-// head-0 CTA writes the metadata and the slot maps. K/V rows of unused slots are left as they
-// are. Keys get exactly the rotations the single-token updates give them: RoPE(t) on entry
-// and, for separators with shifting, RoPE(A - t) on admission.
+// kPrefillSplit CTAs per sequence, each for a run of slots: each finds e_end and the separator
+// count (block-wide counts), scans the flags to place the kept separators, writes the slot maps
+// of its slots and copies and rotates their K/V rows of every KV head (the cos/sin of a slot's
+// pairs are formed once and applied to all heads); the first CTA writes the metadata. K/V rows
+// of unused slots are left as they are. Keys get exactly the rotations the single-token updates
+// give them: RoPE(t) on entry and, for separators with shifting, RoPE(A - t) on admission.
 constexpr int kPrefillThreads = 256;
 constexpr int kPrefillItems = 16;
+constexpr int kPrefillSplit = 8;
 
 __device__ __forceinline__ int block_count_flags(const uint8_t* flags, int lo, int hi,
                                                  int* s_warp) {
@@ -366,8 +381,10 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
   extern __shared__ int s_seppos[];  // [s]: position of the separator at each ring index
   __shared__ int s_warp[kPrefillThreads / 32];
   const int Hkv = cd.Hkv, d = cd.d, a = cd.a, s = cd.s, w = cd.w, P = cd.P;
-  const int seq = blockIdx.x, head = blockIdx.y;
+  const int seq = blockIdx.x, split = blockIdx.y;
   const int ns = a + s + P + w;
+  const int slots_per = (ns + kPrefillSplit - 1) / kPrefillSplit;
+  const int slot_lo = split * slots_per, slot_hi = min(ns, slot_lo + slots_per);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint8_t* flags = sep_in + (size_t)seq * L;
   const int ninit = min(a, L);
@@ -454,14 +471,14 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
     return -1;
   };
 
-  // ---- metadata and slot maps (once per sequence)
-  if (head == 0) {
-    for (int slot = tid; slot < ns; slot += kPrefillThreads) {
-      int A = 0;
-      const int pos = pos_of(slot, &A);
-      slot_pos[(size_t)seq * ns + slot] = pos;
-      slot_sep[(size_t)seq * ns + slot] = (pos >= 0 && flags[pos] != 0) ? 1 : 0;
-    }
+  // ---- slot maps of this CTA's slots, metadata once per sequence
+  for (int slot = slot_lo + tid; slot < slot_hi; slot += kPrefillThreads) {
+    int A = 0;
+    const int pos = pos_of(slot, &A);
+    slot_pos[(size_t)seq * ns + slot] = pos;
+    slot_sep[(size_t)seq * ns + slot] = (pos >= 0 && flags[pos] != 0) ? 1 : 0;
+  }
+  if (split == 0) {
     if (tid == 0) {
       int32_t* m = meta + (size_t)seq * SEPCACHE_META;
       m[SEPCACHE_META_T] = L;
@@ -474,24 +491,34 @@ __global__ void __launch_bounds__(kPrefillThreads) sepcache_prefill_kernel(
       m[SEPCACHE_META_SEP_ADMIT] = count;
     }
   }
-  // ---- this head's K/V rows of the occupied slots (one warp per row, 16-byte vectors)
+  // ---- K/V rows of this CTA's occupied slots, every head (one warp per slot): lane l rotates
+  // pair chunk l % hv of heads l / hv, l / hv + 32 / hv, ... with the chunk's cos/sin formed once
   const int vec = d / 8;
-  const size_t dst_base = ((size_t)seq * Hkv + head) * ns;
-  for (int slot = warp; slot < ns; slot += kPrefillThreads / 32) {
+  const int hv = vec / 2;         // pair chunks per row (8 at d = 128, 4 at d = 64)
+  const int hstep = 32 / hv;      // heads one warp pass covers
+  const int e = lane % hv;
+  for (int slot = slot_lo + warp; slot < slot_hi; slot += kPrefillThreads / 32) {
     int A = 0;
     const int pos = pos_of(slot, &A);
     if (pos < 0) continue;
-    const bool is_sep_slot = slot >= a && slot < a + s;
-    const size_t src = (((size_t)seq * L + pos) * Hkv + head) * vec;
-    const size_t dst = (dst_base + slot) * vec;
-    for (int e = lane; e < vec / 2; e += 32) {  // K: chunk e and its RoPE partner
-      uint4 x = __ldg(k_in + src + e), y = __ldg(k_in + src + e + vec / 2);
-      rope_rotate_chunks(x, y, 8 * e, pos, freq);
-      if (is_sep_slot && !cd.orig) rope_rotate_chunks(x, y, 8 * e, (long long)A - pos, freq);
+    const bool rerotate = slot >= a && slot < a + s && !cd.orig;
+    const ChunkCS cs1 = rope_chunk_cs(8 * e, pos, freq);
+    ChunkCS cs2 = cs1;
+    if (rerotate) cs2 = rope_chunk_cs(8 * e, (long long)A - pos, freq);
+    for (int head = lane / hv; head < Hkv; head += hstep) {
+      const size_t src = (((size_t)seq * L + pos) * Hkv + head) * vec;
+      const size_t dst = (((size_t)seq * Hkv + head) * ns + slot) * vec;
+      uint4 x = __ldg(k_in + src + e), y = __ldg(k_in + src + e + hv);
+      if (pos != 0) rope_apply_chunks(x, y, cs1);
+      if (rerotate && A != pos) rope_apply_chunks(x, y, cs2);
       k_slots[dst + e] = x;
-      k_slots[dst + e + vec / 2] = y;
+      k_slots[dst + e + hv] = y;
     }
-    for (int e = lane; e < vec; e += 32) v_slots[dst + e] = __ldg(v_in + src + e);
+    for (int c = lane; c < Hkv * vec; c += 32) {
+      const int head = c / vec, q = c % vec;
+      v_slots[(((size_t)seq * Hkv + head) * ns + slot) * vec + q] =
+          __ldg(v_in + (((size_t)seq * L + pos) * Hkv + head) * vec + q);
+    }
   }
 }
 
@@ -932,7 +959,7 @@ cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, cons
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  sepcache_prefill_kernel<<<dim3(st.S, st.Hkv), kPrefillThreads, smem, stream>>>(
+  sepcache_prefill_kernel<<<dim3(st.S, kPrefillSplit), kPrefillThreads, smem, stream>>>(
       L, cache_dims(st), st.rope_freq, static_cast<const uint4*>(k),
       static_cast<const uint4*>(v), sep, reinterpret_cast<uint4*>(st.k_slots),
       reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta);

@@ -273,6 +273,29 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x for a pair on the FMA pipe instead of the XU pipe (the softmax kernels run one exp2 per
+// computed score, which keeps the XU pipe the busiest; part of them move here). Cody-Waite
+// reduction x = n + f with n = rint(x) (the 1.5 * 2^23 shift leaves rint(x) in the low mantissa
+// bits of t), f in [-1/2, 1/2]; 2^f by a cubic fitted here for least maximum relative error on
+// that interval (Lawson's reweighted least squares, fp32 coefficients, max relative error
+// 8.3e-5); 2^n added to the exponent field, since (bits(t) << 23) = n << 23 modulo 2^32.
+// Inputs below -125 are clamped there (the result stays a normal float, about 2e-38, in place of
+// 0); inputs are at most 8 in these kernels.
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 shift = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, shift);
+  const float2 f = __fadd2_rn(x, __fadd2_rn(shift, make_float2(-t.x, -t.y)));
+  float2 p = __ffma2_rn(make_float2(0.055212993f, 0.055212993f), f,
+                        make_float2(0.24271414f, 0.24271414f));
+  p = __ffma2_rn(p, f, make_float2(0.69326216f, 0.69326216f));
+  p = __ffma2_rn(p, f, make_float2(0.99991959f, 0.99991959f));
+  return make_float2(
+      __uint_as_float(__float_as_uint(t.x) * 8388608u + __float_as_uint(p.x)),
+      __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(p.y)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

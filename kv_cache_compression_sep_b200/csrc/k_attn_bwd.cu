@@ -645,6 +645,16 @@ struct DkvCfg {
   static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, storer
 };
 
+// One entry of the item ring: the work item and the mask inputs every role needs, loaded once
+// from global memory by the producer and read by the other roles from shared memory.
+struct ItemSlot {
+  int x;                   // item index (>= nitems: no more items)
+  int b, unit, t_begin, t_end, window;
+  int pre_tile;            // anchors left of key tile `unit` (window items)
+  int cnt_b;               // anchors of batch b
+  uint32_t tile_words[4];  // anchor flags of key tile `unit` (window items)
+};
+
 template <int NST, int KVB>
 struct DkvBar {
   uint64_t kv_full[KVB], kv_empty[KVB];
@@ -653,10 +663,11 @@ struct DkvBar {
   uint64_t acc_full, acc_free;
   uint64_t staged[KVB];   // the item's dK/dV rows are in the K/V buffer (softmax -> storer)
   uint64_t drain;
-  uint64_t item_full[4];  // ring of fetched work-item indices (producer -> MMA, softmax)
-  int item_x[4];
+  uint64_t item_full[4];  // ring of fetched work items (producer -> MMA, softmax, storer)
+  ItemSlot item[4];
   float nlse2[NST][128];  // -log2-domain LSE of each query of the stage (-inf past L)
   float delta[NST][128];
+  int pin[NST];           // mask input of the stage's pair: tile class (window) or gather_end
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -684,6 +695,17 @@ __device__ __forceinline__ DkvItem dkv_item(const BwdParams& p, const WorkItem* 
   it.t_begin = w.t_begin;
   it.t_end = w.t_end;
   it.npairs = (w.t_end - w.t_begin) * G;
+  return it;
+}
+__device__ __forceinline__ DkvItem slot_item(const ItemSlot& sl, int Hkv, int G) {
+  DkvItem it;
+  it.kvh = sl.x % Hkv;
+  it.window = sl.window != 0;
+  it.b = sl.b;
+  it.unit = sl.unit;
+  it.t_begin = sl.t_begin;
+  it.t_end = sl.t_end;
+  it.npairs = (sl.t_end - sl.t_begin) * G;
   return it;
 }
 
@@ -755,24 +777,40 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
       int x = 0;
       if (lane == 0) {
+        // fetch the item, start its K/V loads, then load its mask inputs and publish it all
         x = min(atomicAdd(&counters[2], 1), nitems);
-        bar->item_x[I & 3] = x;
+        ItemSlot& sl = bar->item[I & 3];
+        sl.x = x;
+        if (x < nitems) {
+          const DkvItem w = dkv_item(p, aitems, witems, n_anchor, x, G);
+          mbar_arrive_expect_tx(&bar->kv_full[kb], 2 * C::TILE);
+          const int krow = w.unit * 128;
+          for (int q = 0; q < C::KB; ++q) {
+            tma_load_4d(sK + kb * C::TILE + q * kBoxBytes, w.window ? &p.tmK : &p.tmKc,
+                        &bar->kv_full[kb], q * 64, w.kvh, krow, w.b);
+            tma_load_4d(sV + kb * C::TILE + q * kBoxBytes, w.window ? &p.tmV : &p.tmVc,
+                        &bar->kv_full[kb], q * 64, w.kvh, krow, w.b);
+          }
+          nkv = I + 1;
+          sl.b = w.b;
+          sl.unit = w.unit;
+          sl.t_begin = w.t_begin;
+          sl.t_end = w.t_end;
+          sl.window = w.window ? 1 : 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            sl.tile_words[q] = (w.window && w.unit * 4 + q < p.W)
+                                   ? __ldg(p.anchor_bits + (size_t)w.b * p.W + w.unit * 4 + q)
+                                   : 0u;
+          sl.pre_tile = w.window ? __ldg(tile_prefix + (size_t)w.b * p.T + w.unit) : 0;
+          sl.cnt_b = __ldg(p.anchor_cnt + w.b);
+        }
         mbar_arrive(&bar->item_full[I & 3]);
       }
       x = __shfl_sync(0xffffffffu, x, 0);
       if (x >= nitems) break;
-      const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
-      nkv = I + 1;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar->kv_full[kb], 2 * C::TILE);
-        const int krow = it.unit * 128;
-        for (int q = 0; q < C::KB; ++q) {
-          tma_load_4d(sK + kb * C::TILE + q * kBoxBytes, it.window ? &p.tmK : &p.tmKc,
-                      &bar->kv_full[kb], q * 64, it.kvh, krow, it.b);
-          tma_load_4d(sV + kb * C::TILE + q * kBoxBytes, it.window ? &p.tmV : &p.tmVc,
-                      &bar->kv_full[kb], q * 64, it.kvh, krow, it.b);
-        }
-      }
+      __syncwarp();
+      const DkvItem it = slot_item(bar->item[I & 3], p.Hkv, G);
       for (int q = 0; q < it.npairs; ++q, ++P) {
         const int st = P % NST, r = P / NST;
         const int t = it.t_begin + q / G, h = it.kvh * G + q % G;
@@ -787,6 +825,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
             tma_load_4d(sdO + st * C::TILE + z * kBoxBytes, &p.tmdO, &bar->q_full[st], z * 64, h,
                         t * 128, it.b);
           }
+          // the pair's mask input: class of block (t, unit), or the anchors tile t gathers
+          bar->pin[st] = it.window ? (int)__ldg(p.tile_map + ((size_t)it.b * p.T + t) * p.T + it.unit)
+                                   : __ldg(p.gather_end + (size_t)it.b * p.T + t);
         }
         // per-query statistics: log2-domain lse (+inf past L: P = 0 there) and Delta
         const size_t base = ((size_t)it.b * p.Hq + h) * p.L;
@@ -828,9 +869,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       };
       auto load_item = [&](Cur& c) -> bool {  // c.I set: wait for the producer to publish it
         if (!mbar_wait(&bar->item_full[c.I & 3], (c.I >> 2) & 1, p.err, abort_flag)) return false;
-        c.x = bar->item_x[c.I & 3];
+        c.x = bar->item[c.I & 3].x;
         c.q = 0;
-        if (c.x < nitems) c.it = dkv_item(p, aitems, witems, n_anchor, c.x, G);
+        if (c.x < nitems) c.it = slot_item(bar->item[c.I & 3], p.Hkv, G);
         return true;
       };
       auto issue_S = [&](const Cur& c, int h) -> bool {
@@ -919,9 +960,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     if (lane == 0) {
       for (int I = 0;; ++I) {
         if (!mbar_wait(&bar->item_full[I & 3], (I >> 2) & 1, p.err, abort_flag)) break;
-        const int x = bar->item_x[I & 3];
+        const int x = bar->item[I & 3].x;
         if (x >= nitems) break;
-        const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+        const DkvItem it = slot_item(bar->item[I & 3], p.Hkv, G);
         const int kb = I % KVB;
         if (!mbar_wait(&bar->staged[kb], (I / KVB) & 1, p.err, abort_flag)) break;
         if (it.window) {
@@ -949,38 +990,40 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         ok = false;
         break;
       }
-      const int x = bar->item_x[I & 3];
+      const ItemSlot& sl = bar->item[I & 3];
+      const int x = sl.x;
       if (x >= nitems) break;
-      const DkvItem it = dkv_item(p, aitems, witems, n_anchor, x, G);
+      const DkvItem it = slot_item(sl, p.Hkv, G);
       const int kb = I % KVB;
       long long j = -1;  // key position (window items)
       bool fj = false;
       int r = -1;        // compact anchor row (anchor items)
-      uint32_t tile_words[4] = {0u, 0u, 0u, 0u};
+      uint32_t tile_words[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tile_words[q] = sl.tile_words[q];
       if (it.window) {
         j = (long long)it.unit * 128 + krow;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          tile_words[q] = (it.unit * 4 + q < p.W) ? __ldg(p.anchor_bits + (size_t)it.b * p.W + it.unit * 4 + q) : 0u;
         fj = j < p.L && ((tile_words[krow >> 5] >> (krow & 31)) & 1u);
       } else {
         r = it.unit * 128 + krow;
       }
-      const int* ge_row = p.gather_end + (size_t)it.b * p.T;
-      // loaded now, used at the epilogue
-      const int pre_tile = it.window ? __ldg(tile_prefix + (size_t)it.b * p.T + it.unit) : 0;
-      const int cnt_b = __ldg(p.anchor_cnt + it.b);
-      const int8_t* tm_col = p.tile_map + (size_t)it.b * p.T * p.T + it.unit;  // [t][u] at t * T
-      // per-pair mask input (tile class or gather count), loaded one pair ahead
-      int nxt = it.window ? (int)__ldg(tm_col + (size_t)it.t_begin * p.T) : __ldg(ge_row + it.t_begin);
+      // used at the epilogue
+      const int pre_tile = sl.pre_tile;
+      const int cnt_b = sl.cnt_b;
       for (int q = 0; q < it.npairs; ++q, ++P) {
         const int st = P % NST;
         const int t = it.t_begin + q / G;
-        const int cur = nxt;
-        if (q + 1 < it.npairs) {
-          const int tn = it.t_begin + (q + 1) / G;
-          nxt = it.window ? (int)__ldg(tm_col + (size_t)tn * p.T) : __ldg(ge_row + tn);
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[h], P & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
         }
+        // q_full also covers the per-query statistics and the mask input of the pair, written
+        // by the producer warp
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar->q_full[st], (P / NST) & 1, p.err, abort_flag))) {
+          ok = false;
+          break;
+        }
+        const int cur = bar->pin[st];
         // keep bits over the 64 query columns of this half
         uint32_t keep[2];
         const long long q0 = (long long)t * 128 + 64 * h;
@@ -999,15 +1042,6 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         } else {
           const uint32_t all = (r < cur) ? 0xffffffffu : 0u;
           keep[0] = keep[1] = all;
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[h], P & 1, p.err, abort_flag))) {
-          ok = false;
-          break;
-        }
-        // q_full also covers the per-query statistics written by the producer warp
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar->q_full[st], (P / NST) & 1, p.err, abort_flag))) {
-          ok = false;
-          break;
         }
         tc_fence_after();
         const uint32_t aS = tmem + lane_off + 128 * h, aP = aS + 64;

@@ -12,7 +12,8 @@ retained slot and query head in decode), summed over the step and divided by its
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
 --workload picks a single-row run instead (llama-prefill, long-context, long-context-dense,
-decode) for the other configurations.
+decode, ...) for the other configurations; llama-train adds the backward to the Llama-3-8B
+prefill shape (a small d = 128 backward case for profiler captures).
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no data-path collective);
 time is the max over ranks.
 """
@@ -851,7 +852,8 @@ def single_row(args, dev):
                     "gbs": byts / (ms * 1e-3) / 1e9,
                     "frac_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]})
         return out
-    cfg = {"llama-prefill": workloads.LLAMA3_8B_PREFILL, "long-context": workloads.LONG_CONTEXT,
+    cfg = {"llama-prefill": workloads.LLAMA3_8B_PREFILL, "llama-train": workloads.LLAMA3_8B_PREFILL,
+           "long-context": workloads.LONG_CONTEXT,
            "long-context-dense": workloads.LONG_CONTEXT,
            "pythia-train": workloads.PYTHIA160M}[args.workload]
     n = cfg.L if args.workload == "long-context-dense" else cfg.n
@@ -887,7 +889,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="train-decode",
-                    choices=["train-decode", "pythia-train", "llama-prefill", "long-context",
+                    choices=["train-decode", "pythia-train", "llama-prefill", "llama-train",
+                             "long-context",
                              "long-context-dense", "decode", "decode-past", "decode-noshift",
                              "cache-prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -36,6 +36,8 @@
 // the V rows of every query. Groups are combined through shared memory. No global scratch.
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "sep_common.cuh"
 #include "sep_launch.h"
 
@@ -603,6 +605,11 @@ struct DecSmem {
   int abort_flag;
 };
 
+// Block of logical rank r: 0 initial, 1 separator FIFO, 2 past window and window.
+__device__ __forceinline__ int rank_block(int r, int ninit, int sep_cnt) {
+  return (r < ninit) ? 0 : (r < ninit + sep_cnt) ? 1 : 2;
+}
+
 struct DecodeArgs {
   int Hq, Hkv, G, a, s, P, w;
   const __nv_bfloat16* k_slots;
@@ -728,6 +735,20 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[g][i] = make_float2(0.f, 0.f);
 
+  // this lane's 8 query elements of every query, rotated for block blk
+  auto load_q = [&](int blk) {
+    cur_blk = blk;
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&sm.qrot[blk][g][l * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sm.qrot[blk][g][l * 8 + 4]);
+      qr[g][0] = make_float2(a0.x, a0.y);
+      qr[g][1] = make_float2(a0.z, a0.w);
+      qr[g][2] = make_float2(a1.x, a1.y);
+      qr[g][3] = make_float2(a1.z, a1.w);
+    }
+  };
+
   bool ok = true;
   for (int ch = 0; ch < nchunks && ok; ++ch) {
     const int st = ch % kDecStages;
@@ -736,23 +757,17 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
       break;
     }
     const int c0 = ch * KC;
-#pragma unroll
-    for (int sub = 0; sub < kDecRows; ++sub) {
+    // one key row of the group: scores against the block's rotated queries, online softmax of
+    // this lane's query, V sums of every query; CHECKED rows test their rank (block boundary,
+    // rows past the occupancy), the others belong to a chunk that lies in one block entirely
+    auto process_row = [&](auto checked, int sub) {
+      constexpr bool CHECKED = decltype(checked)::value;
       const int row = sub * NG + grp;
       const int r = c0 + row;
-      const bool valid = r < occ;
-      const int blk = (r < ninit) ? 0 : (r < ninit + sep_cnt) ? 1 : 2;
-      if (blk != cur_blk) {
-        cur_blk = blk;
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          const float4 a0 = *reinterpret_cast<const float4*>(&sm.qrot[blk][g][l * 8]);
-          const float4 a1 = *reinterpret_cast<const float4*>(&sm.qrot[blk][g][l * 8 + 4]);
-          qr[g][0] = make_float2(a0.x, a0.y);
-          qr[g][1] = make_float2(a0.z, a0.w);
-          qr[g][2] = make_float2(a1.x, a1.y);
-          qr[g][3] = make_float2(a1.z, a1.w);
-        }
+      const bool valid = !CHECKED || r < occ;
+      if (CHECKED) {
+        const int blk = rank_block(r, ninit, sep_cnt);
+        if (blk != cur_blk) load_q(blk);
       }
       uint4 kk = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
       if (valid) {
@@ -798,6 +813,15 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[g][i] = f2_fma(pg2, v2[i], acc[g][i]);
       }
+    };
+    const int blk0 = rank_block(c0, ninit, sep_cnt);
+    if (c0 + KC <= occ && blk0 == rank_block(c0 + KC - 1, ninit, sep_cnt)) {
+      if (blk0 != cur_blk) load_q(blk0);
+#pragma unroll
+      for (int sub = 0; sub < kDecRows; ++sub) process_row(std::false_type(), sub);
+    } else {
+#pragma unroll
+      for (int sub = 0; sub < kDecRows; ++sub) process_row(std::true_type(), sub);
     }
     // the last warp done with this stage refills it (its reads all precede the atomic)
     __syncwarp();

@@ -759,7 +759,9 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
     const int c0 = ch * KC;
     // one key row of the group: scores against the block's rotated queries, online softmax of
     // this lane's query, V sums of every query; CHECKED rows test their rank (block boundary,
-    // rows past the occupancy), the others belong to a chunk that lies in one block entirely
+    // rows past the occupancy). A chunk that lies in one block entirely takes the path below
+    // without them, where the group's rows are scored independently and enter the online
+    // softmax together (one maximum and one rescale test per kDecRows rows).
     auto process_row = [&](auto checked, int sub) {
       constexpr bool CHECKED = decltype(checked)::value;
       const int row = sub * NG + grp;
@@ -817,8 +819,59 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
     const int blk0 = rank_block(c0, ninit, sep_cnt);
     if (c0 + KC <= occ && blk0 == rank_block(c0 + KC - 1, ninit, sep_cnt)) {
       if (blk0 != cur_blk) load_q(blk0);
+      // the group's rows scored independently, entering the online softmax together
+      float sc[kDecRows];
+      uint4 vv[kDecRows];
 #pragma unroll
-      for (int sub = 0; sub < kDecRows; ++sub) process_row(std::false_type(), sub);
+      for (int sub = 0; sub < kDecRows; ++sub) {
+        const int row = sub * NG + grp;
+        const uint4 kk = *reinterpret_cast<const uint4*>(ring_k(st, row) + l * 8);
+        vv[sub] = *reinterpret_cast<const uint4*>(ring_v(st, row) + l * 8);
+        const float2 k2[4] = {bf16x2_to_float2(kk.x), bf16x2_to_float2(kk.y),
+                              bf16x2_to_float2(kk.z), bf16x2_to_float2(kk.w)};
+        float part[GP];
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float2 s2 = f2_mul(qr[g][0], k2[0]);
+          s2 = f2_fma(qr[g][1], k2[1], s2);
+          s2 = f2_fma(qr[g][2], k2[2], s2);
+          s2 = f2_fma(qr[g][3], k2[3], s2);
+          part[g] = s2.x + s2.y;
+        }
+        sc[sub] = group_reduce_own<GP, LPK>(part, l);
+      }
+      float mx = sc[0];
+#pragma unroll
+      for (int sub = 1; sub < kDecRows; ++sub) mx = fmaxf(mx, sc[sub]);
+      const bool need = mx > m_own + 8.0f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2(m_own - mx) : 1.0f;
+        if (need) {
+          l_own *= alpha;
+          m_own = mx;
+        }
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float ag = __shfl_sync(0xffffffffu, alpha, lane_of_query<GP, LPK>(g), LPK);
+          const float2 ag2 = make_float2(ag, ag);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[g][i] = f2_mul(acc[g][i], ag2);
+        }
+      }
+#pragma unroll
+      for (int sub = 0; sub < kDecRows; ++sub) {
+        const float p_own = ex2(sc[sub] - m_own);
+        l_own += p_own;
+        const float2 v2[4] = {bf16x2_to_float2(vv[sub].x), bf16x2_to_float2(vv[sub].y),
+                              bf16x2_to_float2(vv[sub].z), bf16x2_to_float2(vv[sub].w)};
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const float pg = __shfl_sync(0xffffffffu, p_own, lane_of_query<GP, LPK>(g), LPK);
+          const float2 pg2 = make_float2(pg, pg);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[g][i] = f2_fma(pg2, v2[i], acc[g][i]);
+        }
+      }
     } else {
 #pragma unroll
       for (int sub = 0; sub < kDecRows; ++sub) process_row(std::true_type(), sub);

@@ -329,11 +329,11 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         const int st = gg % NST;
         if (!mbar_wait(&bar->ds_ready, gg & 1, p.err, abort_flag)) return false;
         tc_fence_after();
+        const uint32_t klo = sdesc_lo(sKa + st * C::TILE, kBoxBytes);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
           mma_ts(tmem + C::COL_DQ, tmem + C::COL_DS + kk * 8,
-                 make_sdesc_sw128(sKa + st * C::TILE + kk * 2048, kBoxBytes, 1024), idQ,
-                 (!first || kk > 0) ? 1u : 0u);
+                 sdesc_join(klo + kk * (2048 >> 4), kDescHi), idQ, (!first || kk > 0) ? 1u : 0u);
         tc_commit(&bar->dq_done);
         tc_commit(&bar->k_empty[st]);
         return true;
@@ -355,17 +355,19 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
             break;
           }
           tc_fence_after();
+          const uint32_t qlo = sdesc_lo(sQb, 16), klo = sdesc_lo(sKa + st * C::TILE, 16);
+          const uint32_t dlo = sdesc_lo(sdOb, 16), vlo = sdesc_lo(sVa + st * C::TILE, 16);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::COL_S, make_sdesc_sw128(sQb + off, 16, 1024),
-                   make_sdesc_sw128(sKa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + C::COL_S, sdesc_join(qlo + off, kDescHi), sdesc_join(klo + off, kDescHi),
+                   idS, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            mma_ss(tmem + C::COL_DP, make_sdesc_sw128(sdOb + off, 16, 1024),
-                   make_sdesc_sw128(sVa + st * C::TILE + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + C::COL_DP, sdesc_join(dlo + off, kDescHi),
+                   sdesc_join(vlo + off, kDescHi), idS, kk > 0 ? 1u : 0u);
           }
           tc_commit(&bar->s_full);
           tc_commit(&bar->v_empty[st]);
@@ -640,8 +642,18 @@ struct DkvCfg {
   static constexpr int KVB = (D == 128) ? 1 : 2;  // K/V buffers (items in flight)
   static constexpr int NST = (D == 128) ? 2 : 3;  // Q/dO stages (pairs in flight)
   static constexpr int SMEM_TILES = TILE * (2 * KVB + 2 * NST);
-  // TMEM columns: half h holds S^T at 128h and dP^T at 128h + 64
-  static constexpr int COL_DV = 256, COL_DK = 256 + D;
+  // d = 64 ("wide"): S^T and dP^T of a whole pair (128 keys x 128 queries, N = 128 products),
+  // P^T and dS^T as bf16 in columns of their own, so that the next pair's S^T / dP^T may be
+  // issued as soon as the softmax warps have read these; both softmax warpgroups work on the
+  // same pair (query columns 64 wg ..). TMEM: S^T 0, dP^T 128, P^T 256, dS^T 320, dV 384, dK 448.
+  // d = 128: the accumulators take 256 columns, so S^T / dP^T are formed per 64-query half in
+  // two buffers (half-pair k = 2 P + h uses buffer k % 2: S^T at 128 b, dP^T at 128 b + 64, then
+  // P^T / dS^T written over them).
+  static constexpr bool WIDE = (D == 64);
+  static constexpr int NB = 2;
+  static constexpr int COL_S = 0, COL_DPW = 128, COL_P = 256, COL_DS = 320;
+  static constexpr int COL_DV = WIDE ? 384 : 256, COL_DK = COL_DV + D;
+  static_assert(COL_DK + D <= 512, "TMEM columns");
   static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, storer
 };
 
@@ -655,11 +667,13 @@ struct ItemSlot {
   uint32_t tile_words[4];  // anchor flags of key tile `unit` (window items)
 };
 
-template <int NST, int KVB>
+template <int NST, int KVB, int NB>
 struct DkvBar {
   uint64_t kv_full[KVB], kv_empty[KVB];
   uint64_t q_full[NST], q_empty[NST];
-  uint64_t s_full[2], pds_ready[2], mm_done[2];
+  // per S^T / dP^T buffer (wide: index 0 only): S^T / dP^T ready, P^T / dS^T written, products
+  // done; wide: S^T / dP^T read by both warpgroups (s_free)
+  uint64_t s_full[NB], pds_ready[NB], mm_done[NB], s_free;
   uint64_t acc_full, acc_free;
   uint64_t staged[KVB];   // the item's dK/dV rows are in the K/V buffer (softmax -> storer)
   uint64_t drain;
@@ -674,7 +688,8 @@ struct DkvBar {
 
 template <int D>
 constexpr size_t dkv_smem_bytes() {
-  return 1024 + DkvCfg<D>::SMEM_TILES + sizeof(DkvBar<DkvCfg<D>::NST, DkvCfg<D>::KVB>);
+  return 1024 + DkvCfg<D>::SMEM_TILES +
+         sizeof(DkvBar<DkvCfg<D>::NST, DkvCfg<D>::KVB, DkvCfg<D>::NB>);
 }
 
 struct DkvItem {
@@ -715,7 +730,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
                             const WorkItem* __restrict__ witems, int32_t* __restrict__ counters,
                             const int32_t* __restrict__ tile_prefix) {
   using C = DkvCfg<D>;
-  constexpr int NST = C::NST, KVB = C::KVB;
+  constexpr int NST = C::NST, KVB = C::KVB, NB = C::NB;
   const int G = p.Hq / p.Hkv;
   const int n_anchor = counters[0];
   const int nitems = (n_anchor + counters[1]) * p.Hkv;
@@ -727,7 +742,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
   uint8_t* sV = sK + KVB * C::TILE;         // KVB buffers
   uint8_t* sQ = sV + KVB * C::TILE;         // NST stages
   uint8_t* sdO = sQ + NST * C::TILE;        // NST stages
-  DkvBar<NST, KVB>* bar = reinterpret_cast<DkvBar<NST, KVB>*>(sdO + NST * C::TILE);
+  DkvBar<NST, KVB, NB>* bar = reinterpret_cast<DkvBar<NST, KVB, NB>*>(sdO + NST * C::TILE);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &bar->abort_flag;
 
@@ -740,11 +755,12 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       mbar_init(&bar->q_full[s], 1 + 32);
       mbar_init(&bar->q_empty[s], 1);
     }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&bar->s_full[h], 1);
-      mbar_init(&bar->pds_ready[h], 128);
-      mbar_init(&bar->mm_done[h], 1);
+    for (int bb = 0; bb < NB; ++bb) {
+      mbar_init(&bar->s_full[bb], 1);
+      mbar_init(&bar->pds_ready[bb], C::WIDE ? 256 : 128);
+      mbar_init(&bar->mm_done[bb], 1);
     }
+    mbar_init(&bar->s_free, 256);
     mbar_init(&bar->acc_full, 1);
     mbar_init(&bar->acc_free, 256);
     for (int s = 0; s < KVB; ++s) mbar_init(&bar->staged[s], 256);
@@ -851,20 +867,21 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
-    // Order over the flattened pair stream: G(P, A), S(P+1, A), G(P, B), S(P+1, B), where S
-    // issues S^T/dP^T of a half and G its dV/dK products; half A's next softmax can then run
-    // while half B's is still working. At an item boundary with a single K/V buffer, both G
-    // of the last pair come first (the next item's K/V needs this item's epilogue).
+    // Over the flattened sequence of half-pairs k = 2 P + h (pair P, query half h): S^T/dP^T of
+    // the first NB half-pairs, then for every k its dV/dK products G(k) followed by S(k + NB),
+    // which reuses the buffer of k once G(k) has read it. With one K/V buffer the next item is
+    // published only after this item's epilogue, so every G of the item goes out before its
+    // first S.
     if (lane == 0) {
       constexpr uint32_t idS = make_idesc_bf16(128, 64, false, false);
       constexpr uint32_t idG = make_idesc_bf16(128, D, false, true);
       const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV);
       const uint32_t sQa = smem_u32(sQ), sdOa = smem_u32(sdO);
       bool ok = true;
-      // cursor over (item, pair): local item count I, its index x, pair q within it, and the
-      // CTA-wide pair count P
+      // cursor over (item, pair): local item count I, its index x, pair q within it, the
+      // CTA-wide pair count P, and the query half h
       struct Cur {
-        int I, x, q, P;
+        int I, x, q, P, h;
         DkvItem it;
       };
       auto load_item = [&](Cur& c) -> bool {  // c.I set: wait for the producer to publish it
@@ -874,82 +891,193 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         if (c.x < nitems) c.it = slot_item(bar->item[c.I & 3], p.Hkv, G);
         return true;
       };
-      auto issue_S = [&](const Cur& c, int h) -> bool {
+      auto issue_S = [&](const Cur& c) -> bool {
+        const int h = c.h, k = 2 * c.P + h, bb = k % NB;
         const int kb = c.I % KVB, st = c.P % NST;
         if (h == 0) {
           if (c.q == 0 && !mbar_wait(&bar->kv_full[kb], (c.I / KVB) & 1, p.err, abort_flag)) return false;
           if (!mbar_wait(&bar->q_full[st], (c.P / NST) & 1, p.err, abort_flag)) return false;
         }
-        // the half's buffers hold the previous pair's P^T / dS^T until its products are done
-        if (c.P > 0 && !mbar_wait(&bar->mm_done[h], (c.P - 1) & 1, p.err, abort_flag)) return false;
+        // the buffer holds the P^T / dS^T of half-pair k - NB until its products are done
+        if (k >= NB && !mbar_wait(&bar->mm_done[bb], ((k / NB) - 1) & 1, p.err, abort_flag))
+          return false;
         tc_fence_after();
         const uint32_t kA = sKa + kb * C::TILE, vA = sVa + kb * C::TILE;
         const uint32_t qA = sQa + st * C::TILE, dA = sdOa + st * C::TILE;
-        const uint32_t cS = tmem + 128 * h, cP = cS + 64;
+        const uint32_t cS = tmem + 128 * bb, cP = cS + 64;
+        const uint32_t klo = sdesc_lo(kA, 16), vlo = sdesc_lo(vA, 16);
+        const uint32_t qlo = sdesc_lo(qA + h * 64 * 128, 16), dlo = sdesc_lo(dA + h * 64 * 128, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          const uint32_t qoff = (kk >> 2) * kBoxBytes + h * 64 * 128 + (kk & 3) * 32;
-          mma_ss(cS, make_sdesc_sw128(kA + off, 16, 1024), make_sdesc_sw128(qA + qoff, 16, 1024),
-                 idS, kk > 0 ? 1u : 0u);
-          mma_ss(cP, make_sdesc_sw128(vA + off, 16, 1024), make_sdesc_sw128(dA + qoff, 16, 1024),
-                 idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss(cS, sdesc_join(klo + off, kDescHi), sdesc_join(qlo + off, kDescHi), idS,
+                 kk > 0 ? 1u : 0u);
+          mma_ss(cP, sdesc_join(vlo + off, kDescHi), sdesc_join(dlo + off, kDescHi), idS,
+                 kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bar->s_full[h]);
+        tc_commit(&bar->s_full[bb]);
         return true;
       };
-      auto issue_G = [&](const Cur& c, int h) -> bool {
+      auto issue_G = [&](const Cur& c) -> bool {
+        const int h = c.h, k = 2 * c.P + h, bb = k % NB;
         const int st = c.P % NST;
         // the first dV/dK product of an item overwrites the accumulators: the previous item's
         // epilogue must have read them
         if (h == 0 && c.q == 0 && c.I > 0 &&
             !mbar_wait(&bar->acc_free, (c.I - 1) & 1, p.err, abort_flag))
           return false;
-        if (!mbar_wait(&bar->pds_ready[h], c.P & 1, p.err, abort_flag)) return false;
+        if (!mbar_wait(&bar->pds_ready[bb], (k / NB) & 1, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint32_t qA = sQa + st * C::TILE, dA = sdOa + st * C::TILE;
-        const uint32_t cS = tmem + 128 * h, cP = cS + 64;
+        const uint32_t cS = tmem + 128 * bb, cP = cS + 64;
+        const uint32_t dlo = sdesc_lo(dA + h * 64 * 128, kBoxBytes);
+        const uint32_t qlo = sdesc_lo(qA + h * 64 * 128, kBoxBytes);
 #pragma unroll
         for (int kk = 0; kk < 64 / 16; ++kk) {
-          const uint32_t roff = (h * 64 + kk * 16) * 128;
+          const uint32_t roff = (kk * 16 * 128) >> 4;
           const uint32_t acc = (c.q > 0 || h > 0 || kk > 0) ? 1u : 0u;
-          mma_ts(tmem + C::COL_DV, cS + kk * 8, make_sdesc_sw128(dA + roff, kBoxBytes, 1024), idG,
-                 acc);
-          mma_ts(tmem + C::COL_DK, cP + kk * 8, make_sdesc_sw128(qA + roff, kBoxBytes, 1024), idG,
-                 acc);
+          mma_ts(tmem + C::COL_DV, cS + kk * 8, sdesc_join(dlo + roff, kDescHi), idG, acc);
+          mma_ts(tmem + C::COL_DK, cP + kk * 8, sdesc_join(qlo + roff, kDescHi), idG, acc);
         }
-        tc_commit(&bar->mm_done[h]);
+        tc_commit(&bar->mm_done[bb]);
         if (h == 1) {
           tc_commit(&bar->q_empty[st]);
           if (c.q == c.it.npairs - 1) tc_commit(&bar->acc_full);
         }
         return true;
       };
-      Cur c;
-      c.I = 0;
-      c.P = 0;
-      ok = load_item(c);
-      if (ok && c.x < nitems) ok = issue_S(c, 0) && issue_S(c, 1);
-      while (ok && c.x < nitems) {
-        Cur n = c;
-        ++n.P;
-        if (c.q + 1 < c.it.npairs) {
-          ++n.q;
-          ok = issue_G(c, 0) && issue_S(n, 0) && issue_G(c, 1) && issue_S(n, 1);
-        } else if (KVB == 1) {
-          // the next item is published only after this item's epilogue (one K/V buffer)
-          ++n.I;
-          ok = issue_G(c, 0) && issue_G(c, 1) && load_item(n);
-          if (ok && n.x < nitems) ok = issue_S(n, 0) && issue_S(n, 1);
-        } else {
-          ++n.I;
-          ok = load_item(n);
-          const bool more = ok && n.x < nitems;
-          ok = ok && issue_G(c, 0) && (!more || issue_S(n, 0)) && issue_G(c, 1) &&
-               (!more || issue_S(n, 1));
+      if constexpr (C::WIDE) {
+        // S^T / dP^T of the whole pair (N = 128), then, once the softmax warps have read them,
+        // the next pair's; dV / dK products of a pair once its P^T / dS^T are in TMEM
+        constexpr uint32_t idSW = make_idesc_bf16(128, 128, false, false);
+        auto issue_SW = [&](const Cur& c) -> bool {
+          const int kb = c.I % KVB, st = c.P % NST;
+          if (c.q == 0 && !mbar_wait(&bar->kv_full[kb], (c.I / KVB) & 1, p.err, abort_flag)) return false;
+          if (!mbar_wait(&bar->q_full[st], (c.P / NST) & 1, p.err, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t klo = sdesc_lo(sKa + kb * C::TILE, 16), vlo = sdesc_lo(sVa + kb * C::TILE, 16);
+          const uint32_t qlo = sdesc_lo(sQa + st * C::TILE, 16), dlo = sdesc_lo(sdOa + st * C::TILE, 16);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + C::COL_S, sdesc_join(klo + off, kDescHi), sdesc_join(qlo + off, kDescHi),
+                   idSW, kk > 0 ? 1u : 0u);
+            mma_ss(tmem + C::COL_DPW, sdesc_join(vlo + off, kDescHi),
+                   sdesc_join(dlo + off, kDescHi), idSW, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bar->s_full[0]);
+          return true;
+        };
+        auto issue_GW = [&](const Cur& c) -> bool {
+          const int st = c.P % NST;
+          if (c.q == 0 && c.I > 0 && !mbar_wait(&bar->acc_free, (c.I - 1) & 1, p.err, abort_flag))
+            return false;
+          if (!mbar_wait(&bar->pds_ready[0], c.P & 1, p.err, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t dlo = sdesc_lo(sdOa + st * C::TILE, kBoxBytes);
+          const uint32_t qlo = sdesc_lo(sQa + st * C::TILE, kBoxBytes);
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk) {
+            const uint32_t roff = (kk * 16 * 128) >> 4;
+            const uint32_t acc = (c.q > 0 || kk > 0) ? 1u : 0u;
+            mma_ts(tmem + C::COL_DV, tmem + C::COL_P + kk * 8, sdesc_join(dlo + roff, kDescHi),
+                   idG, acc);
+            mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + kk * 8, sdesc_join(qlo + roff, kDescHi),
+                   idG, acc);
+          }
+          tc_commit(&bar->mm_done[0]);
+          tc_commit(&bar->q_empty[st]);
+          if (c.q == c.it.npairs - 1) tc_commit(&bar->acc_full);
+          return true;
+        };
+        Cur c;
+        c.I = 0;
+        c.P = 0;
+        c.h = 0;
+        ok = load_item(c);
+        if (ok && c.x < nitems) ok = issue_SW(c);
+        while (ok && c.x < nitems) {
+          Cur n = c;
+          ++n.P;
+          bool more = true;
+          if (++n.q >= n.it.npairs) {
+            // the next item: published once the epilogue of item I + 1 - KVB has freed its K/V
+            // buffer, which needs no product of this item
+            ++n.I;
+            ok = load_item(n);
+            more = ok && n.x < nitems;
+          }
+          if (!ok) break;
+          if (more) {
+            if (!mbar_wait(&bar->s_free, c.P & 1, p.err, abort_flag)) { ok = false; break; }
+            ok = issue_SW(n);
+            if (!ok) break;
+          }
+          ok = issue_GW(c);
+          c = n;
         }
-        c = n;
+      } else {
+      // S cursor cs (at most NB half-pairs ahead) and G cursor cg; nS / nG half-pairs issued.
+      // The item a cursor moves into is read from the item ring: the S cursor waits for it to be
+      // published, which needs the epilogue of item I - KVB (its K/V buffer), so it does so only
+      // once every G of that item has been issued (s_end[I & 1]: half-pairs up to its end).
+      Cur cs, cg;
+      int nS = 0, nG = 0;
+      int s_end[2] = {0, 0};
+      bool s_pending = false;  // cs entered item cs.I, not yet loaded
+      bool g_pending = false;  // cg entered item cg.I, header not yet read
+      cs.I = 0;
+      cs.P = 0;
+      cs.h = 0;
+      ok = load_item(cs);
+      cg = cs;
+      for (;;) {
+        // S as far ahead as the buffers allow
+        while (ok && nS < nG + NB) {
+          if (s_pending) {
+            if (cs.I >= KVB && nG < s_end[(cs.I - KVB) & 1]) break;
+            ok = load_item(cs);
+            s_pending = false;
+            if (!ok) break;
+          }
+          if (cs.x >= nitems) break;
+          ok = issue_S(cs);
+          ++nS;
+          if (!ok) break;
+          if (cs.h == 0) {
+            cs.h = 1;
+          } else {
+            cs.h = 0;
+            ++cs.P;
+            if (++cs.q >= cs.it.npairs) {
+              s_end[cs.I & 1] = nS;
+              ++cs.I;
+              s_pending = true;
+            }
+          }
+        }
+        if (!ok || nG >= nS) break;
+        if (g_pending) {
+          cg.x = bar->item[cg.I & 3].x;  // published: the S cursor has waited for it
+          cg.q = 0;
+          cg.it = slot_item(bar->item[cg.I & 3], p.Hkv, G);
+          g_pending = false;
+        }
+        ok = issue_G(cg);
+        ++nG;
+        if (!ok) break;
+        if (cg.h == 0) {
+          cg.h = 1;
+        } else {
+          cg.h = 0;
+          ++cg.P;
+          if (++cg.q >= cg.it.npairs) {
+            ++cg.I;
+            g_pending = true;
+          }
+        }
       }
+      }  // half-pair path
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }
@@ -1013,7 +1141,11 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       for (int q = 0; q < it.npairs; ++q, ++P) {
         const int st = P % NST;
         const int t = it.t_begin + q / G;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar->s_full[h], P & 1, p.err, abort_flag))) {
+        // half-pair index and its S^T / dP^T buffer (wide: the pair, buffer 0)
+        const int kk2 = C::WIDE ? P : 2 * P + h, bb = C::WIDE ? 0 : kk2 % NB;
+        const int sbuf_use = C::WIDE ? P : kk2 / NB;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bar->s_full[bb], sbuf_use & 1, p.err, abort_flag))) {
           ok = false;
           break;
         }
@@ -1044,19 +1176,12 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
           keep[0] = keep[1] = all;
         }
         tc_fence_after();
-        const uint32_t aS = tmem + lane_off + 128 * h, aP = aS + 64;
         const float* nlse2 = &bar->nlse2[st][64 * h];
         const float* dl = &bar->delta[st][64 * h];
-        // two 32-column chunks; packed chunk c lands in columns 16c..16c+15, already read
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t sv[32], dp[32];
-          tmem_ld32(aS + 32 * ch, sv);
-          tmem_ld32(aP + 32 * ch, dp);
-          tmem_ld_wait();
-          uint32_t pk[16], dk16[16];
-          // two queries per packed fp32x2 instruction: x = S * scale*log2(e) - lse2,
-          // P = exp2(x) on kept pairs, dS = P (dP - Delta)
+        // one 32-column chunk: x = S * scale*log2(e) - lse2 (two queries per packed fp32x2
+        // instruction), P = exp2(x) on kept pairs, dS = P (dP - Delta), both packed to bf16
+        auto pds_chunk = [&](int ch, const uint32_t(&sv)[32], const uint32_t(&dp)[32],
+                             uint32_t(&pk)[16], uint32_t(&dk16)[16]) {
           const float2 sl2x2 = make_float2(sl2, sl2);
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
@@ -1071,24 +1196,54 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
             pk[c >> 1] = pack_bf16x2(p0, p1);
             dk16[c >> 1] = pack_bf16x2(ds.x, ds.y);
           }
-          asm volatile(
-              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-              "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aS + 16 * ch),
-              "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
-              "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]),
-              "r"(pk[13]), "r"(pk[14]), "r"(pk[15])
-              : "memory");
-          asm volatile(
-              "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-              "%10, %11, %12, %13, %14, %15, %16};" ::"r"(aP + 16 * ch),
-              "r"(dk16[0]), "r"(dk16[1]), "r"(dk16[2]), "r"(dk16[3]), "r"(dk16[4]), "r"(dk16[5]),
-              "r"(dk16[6]), "r"(dk16[7]), "r"(dk16[8]), "r"(dk16[9]), "r"(dk16[10]),
-              "r"(dk16[11]), "r"(dk16[12]), "r"(dk16[13]), "r"(dk16[14]), "r"(dk16[15])
-              : "memory");
+        };
+        if constexpr (C::WIDE) {
+          // this warpgroup's 64 query columns of the pair's S^T / dP^T; P^T / dS^T go to their
+          // own columns once the previous pair's products have read them
+          const uint32_t aS = tmem + lane_off + C::COL_S + 64 * h;
+          const uint32_t aD = tmem + lane_off + C::COL_DPW + 64 * h;
+          uint32_t pk[2][16], dk16[2][16];
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t sv[32], dp[32];
+            tmem_ld32(aS + 32 * ch, sv);
+            tmem_ld32(aD + 32 * ch, dp);
+            tmem_ld_wait();
+            if (ch == 1) {
+              tc_fence_before();
+              mbar_arrive(&bar->s_free);  // the next pair's S^T / dP^T may overwrite them
+            }
+            pds_chunk(ch, sv, dp, pk[ch], dk16[ch]);
+          }
+          if (P > 0 && !__all_sync(0xffffffffu,
+                                   mbar_wait(&bar->mm_done[0], (P - 1) & 1, p.err, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            tmem_st16(tmem + lane_off + C::COL_P + 32 * h + 16 * ch, pk[ch]);
+            tmem_st16(tmem + lane_off + C::COL_DS + 32 * h + 16 * ch, dk16[ch]);
+          }
+        } else {
+          // two 32-column chunks; packed chunk c lands in columns 16c..16c+15, already read
+          const uint32_t aS = tmem + lane_off + 128 * bb, aP = aS + 64;
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t sv[32], dp[32];
+            tmem_ld32(aS + 32 * ch, sv);
+            tmem_ld32(aP + 32 * ch, dp);
+            tmem_ld_wait();
+            uint32_t pk[16], dk16[16];
+            pds_chunk(ch, sv, dp, pk, dk16);
+            tmem_st16(aS + 16 * ch, pk);
+            tmem_st16(aP + 16 * ch, dk16);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bar->pds_ready[h]);
+        mbar_arrive(&bar->pds_ready[bb]);
       }
       if (!ok) break;
       // ---------------------------------------------------------------- item epilogue

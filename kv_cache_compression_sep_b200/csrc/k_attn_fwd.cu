@@ -259,12 +259,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         if (!mbar_wait(&bar->v_full[st], (gg / NST) & 1, p.err, abort_flag, p.wait_ns)) return false;
         tc_fence_after();
         const uint32_t aP = tmem + C::COL_P;
+        const uint32_t vlo = sdesc_lo(sVa + st * C::TILE_BYTES, C::BOX_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t bd =
-              make_sdesc_sw128(sVa + st * C::TILE_BYTES + kk * 2048, C::BOX_BYTES, 1024);
-          mma_ts(tmem + C::COL_O, aP + kk * 8, bd, idO, (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + C::COL_O, aP + kk * 8, sdesc_join(vlo + kk * (2048 >> 4), kDescHi), idO,
+                 (!first || kk > 0) ? 1u : 0u);
         tc_commit(&bar->pv_done);
         tc_commit(&bar->v_empty[st]);
         return true;
@@ -291,12 +290,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             break;
           }
           tc_fence_after();
+          const uint32_t qlo = sdesc_lo(sQb, 16), klo = sdesc_lo(sKa + st * C::TILE_BYTES, 16);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-            const uint64_t ad = make_sdesc_sw128(sQb + off, 16, 1024);
-            const uint64_t bd = make_sdesc_sw128(sKa + st * C::TILE_BYTES + off, 16, 1024);
-            mma_ss(tmem + C::COL_S, ad, bd, idS, kk > 0 ? 1u : 0u);
+            const uint32_t off = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+            mma_ss(tmem + C::COL_S, sdesc_join(qlo + off, kDescHi), sdesc_join(klo + off, kDescHi),
+                   idS, kk > 0 ? 1u : 0u);
           }
           tc_commit(&bar->s_full);
           tc_commit(&bar->k_empty[st]);

@@ -207,6 +207,24 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool a_mn_m
 //  K-major tiles: rows of 128 B (64 bf16), 8-row groups 1024 B apart (SBO), LBO unused (1).
 //  MN-major tiles: 64 MN-elements (128 B) contiguous per K-row, 8 K-rows per 1024 B group
 //  (SBO = 1024), and LBO = distance between 64-element MN groups.
+// The same descriptor in two 32-bit words: the address word (start address and LBO) and the
+// constant high word (SBO, version, swizzle). The MMA loops keep the high word fixed and step
+// the address word with 32-bit adds (the address field holds smem byte address / 16 < 2^14, so
+// offsets inside shared memory never carry into the LBO field): rebuilding the 64-bit descriptor
+// for every instruction costs the issuing thread about 190 cycles per tcgen05.mma, against about
+// 50 this way (measured on B200; an M128 N64 K16 product takes 32 cycles of tensor time).
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t smem_addr, uint32_t lbo_bytes) {
+  return ((smem_addr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t sdesc_hi_sw128(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) /*version*/ | (2u << 29) /*SWIZZLE_128B*/;
+}
+__device__ __forceinline__ uint64_t sdesc_join(uint32_t lo, uint32_t hi) {
+  return ((uint64_t)hi << 32) | lo;
+}
+// High word of every descriptor in these kernels: 8-row groups 1024 bytes apart, 128-byte swizzle.
+constexpr uint32_t kDescHi = sdesc_hi_sw128(1024);
+
 __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t smem_addr, uint32_t lbo_bytes,
                                                      uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -242,6 +260,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+      "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() {

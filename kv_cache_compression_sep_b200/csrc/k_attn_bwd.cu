@@ -1008,12 +1008,19 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
             more = ok && n.x < nitems;
           }
           if (!ok) break;
+          // at the last pair of an item its products go first, so that the epilogue (which
+          // runs before the next item's first softmax) starts as early as possible
+          const bool gfirst = n.q == 0;
+          if (gfirst) {
+            ok = issue_GW(c);
+            if (!ok) break;
+          }
           if (more) {
             if (!mbar_wait(&bar->s_free, c.P & 1, p.err, abort_flag)) { ok = false; break; }
             ok = issue_SW(n);
             if (!ok) break;
           }
-          ok = issue_GW(c);
+          if (!gfirst) ok = issue_GW(c);
           c = n;
         }
       } else {
@@ -1274,11 +1281,14 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       }
       float* dst = dst_row >= 0 ? part + (((size_t)it.b * p.L + dst_row) * p.Hkv + it.kvh) * D : nullptr;
       uint8_t* stage = (h ? sK : sV) + kb * C::TILE;
-#pragma unroll 1
+      // every accumulator column of the row in one round trip, then the writes
+      uint32_t accs[D / 32][32];
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lane_off + col0 + cc * 32, accs[cc]);
+      tmem_ld_wait();
+#pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t acc[32];
-        tmem_ld32(tmem + lane_off + col0 + cc * 32, acc);
-        tmem_ld_wait();
+        const uint32_t(&acc)[32] = accs[cc];
         if (dst) {
 #pragma unroll
           for (int z = 0; z < 8; ++z)

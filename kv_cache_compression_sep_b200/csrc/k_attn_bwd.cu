@@ -347,6 +347,12 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         const uint32_t sQb = sQa + qb * C::TILE, sdOb = sdOa + db * C::TILE;
         for (int j = 0; j < it.N; ++j, ++g) {
           const int st = g % NST;
+          // at an item boundary the previous item's last dQ product goes first: the next item's
+          // S waits for its Q / dO tiles, and that item's epilogue waits for this product
+          if (j == 0 && pend >= 0) {
+            if (!issue_dQ(pend, pend_first)) { ok = false; break; }
+            pend = -1;
+          }
           if (!mbar_wait(&bar->k_full[st], (g / NST) & 1, p.err, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&bar->v_full[st], (g / NST) & 1, p.err, abort_flag)) { ok = false; break; }
           if (g > 0 && !mbar_wait(&bar->s_free, (g - 1) & 1, p.err, abort_flag)) { ok = false; break; }

@@ -62,10 +62,13 @@ struct FwdCfg {
   static constexpr int TILE_BYTES = KB * BOX_BYTES; // one [128][D] tile
   static constexpr int NST = (D == 128) ? 2 : 4;    // K/V pipeline stages
   static constexpr int SMEM_TILES = TILE_BYTES * (2 + 2 * NST);  // Q x2, NST x (K, V)
-  static constexpr int COL_S = 0;        // S: 128 fp32 columns
-  static constexpr int COL_O = 128;      // O: D fp32 columns
-  static constexpr int COL_P = 128 + D;  // P: 64 columns (bf16 pairs)
-  static constexpr int TMEM_COLS = (COL_P + 64 <= 256) ? 256 : 512;
+  static constexpr int COL_S = 0;  // S: 128 fp32 columns
+  // O in two accumulators, one per key half (softmax warpgroup): O_wg = sum over the tile's keys
+  // 64 wg .. 64 wg + 63 of P V, each scaled by its own warpgroup's running row max
+  static constexpr int COL_O0 = 128, COL_O1 = 128 + D;
+  static constexpr int COL_P = 128 + 2 * D;  // P: 64 columns (bf16 pairs)
+  static constexpr int TMEM_COLS = 512;
+  static_assert(COL_P + 64 <= TMEM_COLS, "TMEM columns");
   static constexpr int THREADS = 352;  // 8 softmax warps, producer, MMA issuer, O storer
 };
 
@@ -75,9 +78,9 @@ struct FwdBar {
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
   uint64_t s_full, s_free, p_ready, pv_done;
   uint64_t drain;
-  uint64_t pair[4];      // exchange barrier of softmax warps w and w + 4 (64 arrivals)
-  float xch[2][2][128];  // row-max halves exchanged by the two softmax warpgroups (by tile parity)
-  float xl[2][128];      // row-sum halves, exchanged once per item
+  uint64_t pair[4];  // exchange barrier of softmax warps w and w + 4 (64 arrivals)
+  float xm[2][128];  // running row max of each warpgroup's key half, exchanged once per item
+  float xl[2][128];  // and its row sum
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -262,8 +265,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const uint32_t vlo = sdesc_lo(sVa + st * C::TILE_BYTES, C::BOX_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::COL_O, aP + kk * 8, sdesc_join(vlo + kk * (2048 >> 4), kDescHi), idO,
-                 (!first || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + (kk < 4 ? C::COL_O0 : C::COL_O1), aP + kk * 8,
+                 sdesc_join(vlo + kk * (2048 >> 4), kDescHi), idO,
+                 (!first || (kk & 3) > 0) ? 1u : 0u);
         tc_commit(&bar->pv_done);
         tc_commit(&bar->v_empty[st]);
         return true;
@@ -407,31 +411,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             for (int w = 0; w < 2; ++w) keep[w] = range_word(0, rem - 1, 2 * wg + w);
           }
         }
-        // ---- row max of the half (8 independent chains), exchanged with the other half
-        float mx8[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) mx8[q] = -INFINITY;
+        // ---- row max of this warpgroup's 64 key columns (three-input max, 4 chains); the two
+        // halves keep separate running statistics and accumulators until the item's epilogue
         if (masked) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float v = ((keep[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(s[c]) : -INFINITY;
-            s[c] = __float_as_uint(v);
-            mx8[c & 7] = fmaxf(mx8[c & 7], v);
-          }
-        } else {
+          for (int c = 0; c < 64; ++c)
+            if (!((keep[c >> 5] >> (c & 31)) & 1u)) s[c] = __float_as_uint(-INFINITY);
+        }
+        float mx4[4];
 #pragma unroll
-          for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(s[c]));
-        }
-        const float mh = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        bar->xch[g & 1][wg][row] = mh;
-        if (!pair_sync()) {
-          ok = false;
-          break;
-        }
-        const float mx = fmaxf(mh, bar->xch[g & 1][wg ^ 1][row]);
-        // ---- online max with lazy rescale (only when the max grows by more than 2^8); both
-        // halves of a row take the same decision from the same values
+        for (int q = 0; q < 4; ++q) mx4[q] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; c += 2)
+          mx4[(c >> 1) & 3] =
+              fmax3(mx4[(c >> 1) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        // ---- online max with lazy rescale (only when the max grows by more than 2^8)
         const float m_tile = mx * sl2;
         float alpha = 1.0f;
         bool any_rescale = false;
@@ -479,9 +474,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         tc_fence_after();
         if (any_rescale) {
 #pragma unroll 1
-          for (int cc = 0; cc < D / 64; ++cc) {
+          for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t ov[32];
-            const uint32_t ao = tmem + lane_off + C::COL_O + wg * (D / 2) + cc * 32;
+            const uint32_t ao = tmem + lane_off + (wg ? C::COL_O1 : C::COL_O0) + cc * 32;
             tmem_ld32(ao, ov);
             tmem_ld_wait();
 #pragma unroll
@@ -495,16 +490,24 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         mbar_arrive(&bar->p_ready);
       }
       if (!ok) break;
-      // ---- epilogue of this item: row sum of both halves, O / l, LSE (O is reused by the next
-      // item's first P V, which the MMA warp issues only after this thread's next p_ready)
-      // (its own slot: the next item's first row-max exchange may start before the other half
-      // has read this value; the next write here is an item later, after further pair barriers)
+      // ---- epilogue of this item: the two halves' running max and row sum are exchanged and
+      // combined, O = (O0 2^(m0-m) + O1 2^(m1-m)) / (l0 2^(m0-m) + l1 2^(m1-m)), LSE (O0 / O1
+      // are reused by the next item's first P V, which the MMA warp issues only after this
+      // thread's next p_ready; the other half reads these slots before its next p_ready, so
+      // they are not rewritten before being read)
+      bar->xm[wg][row] = m_run;
       bar->xl[wg][row] = l_run;
       if (!pair_sync()) {
         ok = false;
         break;
       }
-      const float l_tot = l_run + bar->xl[wg ^ 1][row];
+      const float m_o = bar->xm[wg ^ 1][row], l_o = bar->xl[wg ^ 1][row];
+      const float m0 = wg ? m_o : m_run, m1 = wg ? m_run : m_o;
+      const float l0 = wg ? l_o : l_run, l1 = wg ? l_run : l_o;
+      const float m_max = fmaxf(m0, m1);
+      const float m_row = (m_max == -INFINITY) ? 0.f : m_max;
+      const float a0 = ex2(m0 - m_row), a1 = ex2(m1 - m_row);
+      const float l_tot = l0 * a0 + l1 * a1;
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&bar->pv_done, (g - 1) & 1, p.err, abort_flag, p.wait_ns))) {
         ok = false;
@@ -512,20 +515,23 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       }
       tc_fence_after();
       const float inv_l = 1.0f / l_tot;
+      const float c0 = a0 * inv_l, c1 = a1 * inv_l;
       const bool valid = i < p.L;
       // O / l as bf16 into the item's Q buffer (every S MMA of the item has completed, so Q is
       // no longer read), in the swizzled box layout, then one TMA store of the whole tile
       uint8_t* stage = sQ + (k_item & 1) * C::TILE_BYTES;
 #pragma unroll 1
       for (int cc = 0; cc < D / 64; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(tmem + lane_off + C::COL_O + wg * (D / 2) + cc * 32, ov);
+        uint32_t ov0[32], ov1[32];
+        tmem_ld32(tmem + lane_off + C::COL_O0 + wg * (D / 2) + cc * 32, ov0);
+        tmem_ld32(tmem + lane_off + C::COL_O1 + wg * (D / 2) + cc * 32, ov1);
         tmem_ld_wait();
         uint32_t pkd[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q)
-          pkd[q] = pack_bf16x2(__uint_as_float(ov[2 * q]) * inv_l,
-                               __uint_as_float(ov[2 * q + 1]) * inv_l);
+          pkd[q] = pack_bf16x2(
+              fmaf(__uint_as_float(ov0[2 * q]), c0, __uint_as_float(ov1[2 * q]) * c1),
+              fmaf(__uint_as_float(ov0[2 * q + 1]), c0, __uint_as_float(ov1[2 * q + 1]) * c1));
         const int col0 = wg * (D / 2) + cc * 32;  // first column of these 32
         uint8_t* box = stage + (col0 >> 6) * C::BOX_BYTES;
 #pragma unroll
@@ -539,7 +545,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       mbar_arrive(&bar->o_staged[k_item & 1]);  // the storer warp writes the tile out
       if (valid && wg == 0)
         p.lse[((size_t)it.b * p.Hq + it.h) * p.L + i] =
-            (m_run + __log2f(l_tot)) * 0.69314718055994531f;
+            (m_row + __log2f(l_tot)) * 0.69314718055994531f;
       ++k_item;
     }
     tc_fence_before();

@@ -324,6 +324,13 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x) {
       __uint_as_float(__float_as_uint(t.y) * 8388608u + __float_as_uint(p.y)));
 }
 
+// Largest of three (the three-input max.f32 of sm_100; a NaN operand is ignored, as in fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -330,15 +330,18 @@ def train_components(step, comps, peaks, peak_src):
     fractions, and the pair slots the kernels compute per kept pair."""
     cfg = step.cfg
     slots = pair_slots(step.mask.gather_end.cpu(), cfg.L, cfg.n)
+    slots_fwd = pair_slots(step.mask.gather_end.cpu(), cfg.L, cfg.n,
+                           step.mask.anchor_bits.cpu().numpy())
     computed_over_kept = slots / step.kept
     rows = {}
-    for name, flops in (("fwd_kernel", step.flops_fwd), ("bwd_dq", 1.5 * step.flops_fwd),
-                        ("bwd_dkdv", 2.0 * step.flops_fwd)):
+    for name, flops, sl in (("fwd_kernel", step.flops_fwd, slots_fwd),
+                            ("bwd_dq", 1.5 * step.flops_fwd, slots),
+                            ("bwd_dkdv", 2.0 * step.flops_fwd, slots)):
         r = roofline_for(name, comps, step, peaks, peak_src)
         rows[name] = {"us": comps[name] * 1e3, "tflops": r["achieved"], "frac_bf16_peak": r["frac"],
                       "algorithmic_flops": flops, "algorithmic_bytes": r["algorithmic_bytes_per_launch"],
                       "combined_frac": r["combined_frac"], "combined_bound": r["combined_bound"],
-                      "computed_pairs_over_kept": computed_over_kept}
+                      "computed_pairs_over_kept": sl / step.kept}
     bwd_ms = comps["bwd_prep"] + comps["bwd_dq"] + comps["bwd_dkdv"]
     dec = roofline_for("decode_attention", comps, step, peaks, peak_src)
     return {
@@ -389,7 +392,7 @@ def attn_row(S, cfg, dev, flush, peaks, n, bwd, iters):
     torch.cuda.synchronize()
     kept = int(mask.kept.sum())
     fl = 4.0 * cfg.d * kept * cfg.Hq
-    slots = pair_slots(mask.gather_end.cpu(), cfg.L, n)
+    slots = pair_slots(mask.gather_end.cpu(), cfg.L, n, mask.anchor_bits.cpu().numpy())
     ws = torch.empty(S.sep_attn_fwd_workspace_size(cfg.B, cfg.L, cfg.Hkv, cfg.d),
                      dtype=torch.uint8, device=dev)
     g = capture(lambda: S.sep_attn_fwd(d["q"], d["k"], d["v"], mask, out=o, lse=lse,
@@ -400,7 +403,7 @@ def attn_row(S, cfg, dev, flush, peaks, n, bwd, iters):
     t_f = max(fl / (peaks["bf16_tflops"] * 1e12), fb / (peaks["hbm_gbs"] * 1e9))
     row = {"B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "L": cfg.L, "d": cfg.d, "a": cfg.a, "n": n,
            "kept_pairs": kept, "kept_over_dense_causal": kept / (cfg.B * cfg.L * (cfg.L + 1) / 2),
-           "computed_pairs_over_kept": slots / kept,
+           "fwd_computed_pairs_over_kept": slots / kept,
            "fwd_ms": ms, "fwd_tflops": fl / (ms * 1e-3) / 1e12,
            "fwd_frac_bf16_peak": fl / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
            "fwd_combined_frac": t_f / (ms * 1e-3)}
@@ -524,17 +527,34 @@ def attn_pass_bytes(B, L, Hq, Hkv, d, name):
             "bwd_dkdv": 2 * q + 2 * kv + 2 * st + 2 * kv}[name]  # ... -> dK, dV
 
 
-def pair_slots(gather_end, L, n):
+def pair_slots(gather_end, L, n, anchor_bits=None):
     """Query-key pair slots the attention kernels compute per head (summed over the batch):
     every query tile t runs whole 128 x 128 tiles over its window key tiles lo(t)..t and over
-    ceil(gather_end[t] / 128) compacted anchor chunks. Identical for the forward, the dQ pass
-    and the dK/dV pass (the latter visits the same (query tile, key unit) pairs key-major)."""
+    ceil(gather_end[t] / 128) compacted anchor chunks (the dQ and dK/dV passes; the latter
+    visits the same (query tile, key unit) pairs key-major).
+    With anchor_bits ([B, W] anchor flags), the forward's count: a query tile whose oldest
+    window tile's lower 64 keys lie outside every row's band (128 t - n + 1 >= 128 lo + 64)
+    gathers their anchors too (G = gather_end + their count), and the first 64 gathered anchors
+    fill that half of the tile, so ceil(max(0, G - 64) / 128) chunks follow."""
     import numpy as np
     ge = np.asarray(gather_end, dtype=np.int64)
     T = ge.shape[-1]
     t = np.arange(T)
     lo = np.maximum(0, 128 * t - n + 1) // 128
-    tiles = (t - lo + 1)[None, :] + (ge + 127) // 128
+    chunks = (ge + 127) // 128
+    if anchor_bits is not None:
+        half = (lo < t) & (128 * t - n + 1 >= 128 * lo + 64)
+        bits = np.asarray(anchor_bits).astype(np.int64) & 0xFFFFFFFF
+        w0 = np.minimum(4 * lo, bits.shape[-1] - 1)
+        w1 = np.minimum(4 * lo + 1, bits.shape[-1] - 1)
+
+        def popc(x):
+            return np.array([[bin(int(v)).count("1") for v in row] for row in x], dtype=np.int64)
+
+        extra = popc(bits[:, w0]) + popc(bits[:, w1])
+        g = ge + extra * half[None, :]
+        chunks = np.where(half[None, :], (np.maximum(0, g - 64) + 127) // 128, chunks)
+    tiles = (t - lo + 1)[None, :] + chunks
     return int(tiles.sum()) * 128 * 128
 
 

@@ -39,14 +39,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [B, L, H, d] bf16 token-major tensor as a 4-D map {d, H, L, B}; box {64, 1, 128, 1} with the
-// 128-byte swizzle (one 128-byte row of 64 bf16 per key/query, 128 rows per box).
-bool encode_map(CUtensorMap* m, const void* base, int B, int L, int H, int d) {
+// [B, L, H, d] bf16 token-major tensor as a 4-D map {d, H, L, B}; box {64, 1, rows, 1} with the
+// 128-byte swizzle (one 128-byte row of 64 bf16 per key/query, 128 or 64 rows per box).
+bool encode_map(CUtensorMap* m, const void* base, int B, int L, int H, int d, int rows = 128) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)L, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)L * H * d * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -147,7 +147,10 @@ static int attn_fwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const
     std::memset(&maps, 0, sizeof(maps));
     if (!encode_map(&maps.q, q, B, L, Hq, d) || !encode_map(&maps.k, k, B, L, Hkv, d) ||
         !encode_map(&maps.v, v, B, L, Hkv, d) || !encode_map(&maps.kc, kc, B, L, Hkv, d) ||
-        !encode_map(&maps.vc, vc, B, L, Hkv, d) || !encode_map(&maps.o, o, B, L, Hq, d))
+        !encode_map(&maps.vc, vc, B, L, Hkv, d) || !encode_map(&maps.o, o, B, L, Hq, d) ||
+        !encode_map(&maps.k64, k, B, L, Hkv, d, 64) || !encode_map(&maps.v64, v, B, L, Hkv, d, 64) ||
+        !encode_map(&maps.kc64, kc, B, L, Hkv, d, 64) ||
+        !encode_map(&maps.vc64, vc, B, L, Hkv, d, 64))
       return SEP_ERR_CUDA;
     AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
     return cuda_status(

@@ -35,6 +35,7 @@ namespace sep {
 
 struct FwdParams {
   CUtensorMap tmQ, tmK, tmV, tmKc, tmVc, tmO;
+  CUtensorMap tmK64, tmV64, tmKc64, tmVc64;  // 64-row boxes: the two halves of a merged tile
   const uint32_t* anchor_bits;  // [B, W] packed anchor flags
   const int32_t* gather_end;
   const int8_t* tile_map;
@@ -91,8 +92,16 @@ constexpr size_t fwd_smem_bytes() {
 }
 
 // Work item x (heaviest query tiles first): query tile t, head h, batch b, and its key tiles.
+// Half window: when the lower 64 keys of the oldest window tile lo lie outside every row's band
+// (128 t - n + 1 >= 128 lo + 64, e.g. any n <= 64), every row keeps exactly the anchors among
+// them, like the anchors left of tile lo; they join the gathered anchors (ge counts both), and
+// the oldest window tile becomes a merged tile: its lower half holds compacted anchors 0..63,
+// its upper half the keys 128 lo + 64 .. 128 lo + 127. The remaining anchors follow in chunks of
+// 128 from compacted row arow0 = 64. This saves the key tile that anchors up to 64 would
+// otherwise take, and half of the padding of the gathered part.
 struct FwdItem {
-  int t, h, b, nwin, ge, N;
+  int t, h, b, nwin, ge, N, arow0;
+  bool half;
 };
 __device__ __forceinline__ FwdItem fwd_item_base(const FwdParams& p, int x) {
   FwdItem it;
@@ -101,19 +110,29 @@ __device__ __forceinline__ FwdItem fwd_item_base(const FwdParams& p, int x) {
   const int rem = x % per_t;
   it.h = rem % p.Hq;
   it.b = rem / p.Hq;
-  it.nwin = it.t - window_lo_tile(it.t, p.n) + 1;
+  const int lo = window_lo_tile(it.t, p.n);
+  it.nwin = it.t - lo + 1;
+  it.half = lo < it.t && (long long)it.t * 128 - p.n + 1 >= (long long)lo * 128 + 64;
+  it.arow0 = it.half ? 64 : 0;
   it.ge = 0;
   it.N = it.nwin;
   return it;
 }
+// Gathered anchors of item x: gather_end (anchors left of tile lo), plus those in the lower half
+// of tile lo for a half-window item.
 __device__ __forceinline__ int fwd_item_ge(const FwdParams& p, int x) {
   const FwdItem it = fwd_item_base(p, x);
-  return p.gather_end[(size_t)it.b * p.T + it.t];
+  int ge = p.gather_end[(size_t)it.b * p.T + it.t];
+  if (it.half) {
+    const uint32_t* w = p.anchor_bits + (size_t)it.b * p.W + (size_t)(it.t - it.nwin + 1) * 4;
+    ge += __popc(__ldg(w)) + __popc(__ldg(w + 1));
+  }
+  return ge;
 }
 __device__ __forceinline__ FwdItem fwd_item_with(const FwdParams& p, int x, int ge) {
   FwdItem it = fwd_item_base(p, x);
   it.ge = ge;
-  it.N = it.nwin + (ge + 127) / 128;
+  it.N = it.nwin + (max(0, ge - it.arow0) + 127) / 128;
   return it;
 }
 
@@ -191,6 +210,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&p.tmV);
       tma_prefetch_desc(&p.tmKc);
       tma_prefetch_desc(&p.tmVc);
+      tma_prefetch_desc(&p.tmK64);
+      tma_prefetch_desc(&p.tmV64);
+      tma_prefetch_desc(&p.tmKc64);
+      tma_prefetch_desc(&p.tmVc64);
       int g = 0;
       int kq = 0;  // items whose Q load was issued
       bool ok = true;
@@ -213,26 +236,39 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int j = 0; j < it.N; ++j, ++g) {
           const int st = g % NST, r = g / NST;
           const bool win = j < it.nwin;
+          const bool merged = it.half && j == it.nwin - 1;
           const CUtensorMap* mk = win ? &p.tmK : &p.tmKc;
           const CUtensorMap* mv = win ? &p.tmV : &p.tmVc;
-          const int row0 = win ? (it.t - j) * C::BN : (j - it.nwin) * C::BN;
+          const int row0 = win ? (it.t - j) * C::BN : it.arow0 + (j - it.nwin) * C::BN;
           if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&bar->k_full[st], C::TILE_BYTES);
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_4d(sK + st * C::TILE_BYTES + kb * C::BOX_BYTES, mk, &bar->k_full[st],
-                        kb * 64, kvh, row0, it.b);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            uint8_t* dst = sK + st * C::TILE_BYTES + kb * C::BOX_BYTES;
+            if (merged) {  // compacted anchors 0..63, then keys 128 lo + 64 ..
+              tma_load_4d(dst, &p.tmKc64, &bar->k_full[st], kb * 64, kvh, 0, it.b);
+              tma_load_4d(dst + 64 * 128, &p.tmK64, &bar->k_full[st], kb * 64, kvh, row0 + 64, it.b);
+            } else {
+              tma_load_4d(dst, mk, &bar->k_full[st], kb * 64, kvh, row0, it.b);
+            }
+          }
           if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag, p.wait_ns)) {
             mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&bar->v_full[st], C::TILE_BYTES);
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_4d(sV + st * C::TILE_BYTES + kb * C::BOX_BYTES, mv, &bar->v_full[st],
-                        kb * 64, kvh, row0, it.b);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            uint8_t* dst = sV + st * C::TILE_BYTES + kb * C::BOX_BYTES;
+            if (merged) {
+              tma_load_4d(dst, &p.tmVc64, &bar->v_full[st], kb * 64, kvh, 0, it.b);
+              tma_load_4d(dst + 64 * 128, &p.tmV64, &bar->v_full[st], kb * 64, kvh, row0 + 64, it.b);
+            } else {
+              tma_load_4d(dst, mv, &bar->v_full[st], kb * 64, kvh, row0, it.b);
+            }
+          }
         }
       }
       if (!ok) {
@@ -390,7 +426,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         // ---- mask of this thread's 64 columns (words 2wg, 2wg+1 of the tile)
         uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
         bool masked = false;
-        if (j < it.nwin) {
+        if (it.half && j == it.nwin - 1 && wg == 0) {
+          // lower half of the merged tile: gathered anchors 0..63, kept by every row
+          const int cnt = min(it.ge, 64);
+          if (cnt < 64) {
+            masked = true;
+#pragma unroll
+            for (int w = 0; w < 2; ++w) keep[w] = range_word(0, cnt - 1, w);
+          }
+        } else if (j < it.nwin) {
           const int u = it.t - j;
           const long long k0 = (long long)u * C::BN;
           if (raw.cls != SEP_TILE_FULL) {
@@ -404,7 +448,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             for (int w = 0; w < 2; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, 2 * wg + w);
           }
         } else {
-          const int rem = it.ge - (j - it.nwin) * C::BN;  // valid anchors in this chunk
+          const int rem = it.ge - it.arow0 - (j - it.nwin) * C::BN;  // valid anchors in this chunk
           if (rem < C::BN) {
             masked = true;
 #pragma unroll
@@ -559,9 +603,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 }
 
 // ------------------------------------------------------------------ anchor compaction
-// Row r < anchor_cnt[b] of kc/vc receives the K/V row of anchor r; rows from anchor_cnt[b] up to
-// the next multiple of 128 are zeroed so that the last (partly valid) anchor chunk holds finite
-// values (masked scores still multiply V in the P*V product).
+// Row r < anchor_cnt[b] of kc/vc receives the K/V row of anchor r; the 128 rows after the last
+// anchor are zeroed, so that the last (partly valid) anchor chunk holds finite values wherever
+// it starts (at a multiple of 128, or at 64 + a multiple of 128 after a merged tile): masked
+// scores still multiply V in the P*V product.
 // One warp per compacted row (8 rows per CTA); CTAs past the last anchor tile exit at once.
 __global__ void __launch_bounds__(256) compact_anchors_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, const int32_t* __restrict__ anchor_idx,
@@ -569,7 +614,7 @@ __global__ void __launch_bounds__(256) compact_anchors_kernel(
     uint4* __restrict__ vc) {
   const int b = blockIdx.y;
   const int cnt = __ldg(anchor_cnt + b);
-  const int pad_end = min(L, (cnt + 127) / 128 * 128);
+  const int pad_end = min(L, cnt + 128);
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (i >= pad_end) return;
   compact_anchor_row(k, v, anchor_idx, cnt, L, b, i, kv_ch, kc, vc, threadIdx.x & 31);
@@ -629,6 +674,10 @@ cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.tmKc = maps.kc;
   prm.tmVc = maps.vc;
   prm.tmO = maps.o;
+  prm.tmK64 = maps.k64;
+  prm.tmV64 = maps.v64;
+  prm.tmKc64 = maps.kc64;
+  prm.tmVc64 = maps.vc64;
   prm.anchor_bits = anchor_bits;
   prm.gather_end = gather_end;
   prm.tile_map = tile_map;

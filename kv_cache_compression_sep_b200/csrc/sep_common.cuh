@@ -69,20 +69,19 @@ __device__ __forceinline__ void record_failure(unsigned* err, volatile int* abor
 
 // Bounded wait for the phase of `parity` to complete. Returns false on timeout (after
 // `limit_ns` of %globaltimer) or when the CTA abort flag is already raised (another role gave
-// up).
+// up). try_wait suspends the thread for a while when the phase is not complete, so a wait takes
+// few passes: both conditions are checked on every pass after the first.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err,
                                           volatile int* abort_flag,
                                           unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  unsigned long long t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        record_failure(err, abort_flag, SEP_ERR_TIMEOUT);
-        return false;
-      }
+    if (abort_flag && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      record_failure(err, abort_flag, SEP_ERR_TIMEOUT);
+      return false;
     }
   }
 }

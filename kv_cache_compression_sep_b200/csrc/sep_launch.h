@@ -36,6 +36,7 @@ cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* 
 struct AttnMaps {
   CUtensorMap q, k, v, kc, vc;  // 4-D {d, H, L, B}, box {64, 1, 128, 1}, 128-byte swizzle
   CUtensorMap o, dout, dq, dk, dv;  // O store (forward); dO load, dQ/dK/dV stores (backward)
+  CUtensorMap k64, v64, kc64, vc64;  // the same tensors with 64-row boxes (forward half tiles)
 };
 
 struct AttnShape {

@@ -11,8 +11,8 @@
 namespace sep {
 
 // Row i of batch b of the compacted anchor K / V (one warp; kv_ch = 16-byte chunks per row):
-// the K / V row of the i-th anchor when i < cnt, zeros up to the end of the anchors' last
-// 128-row tile. The caller takes rows i < min(L, roundup128(cnt)).
+// the K / V row of the i-th anchor when i < cnt, zeros for the padding rows after the last
+// anchor (how many is the caller's choice).
 __device__ __forceinline__ void compact_anchor_row(const uint4* __restrict__ k,
                                                    const uint4* __restrict__ v,
                                                    const int32_t* __restrict__ anchor_idx,

@@ -58,6 +58,28 @@ def test_pair_slots_counts_whole_tiles():
     assert bench.pair_slots(np.zeros((1, 4), dtype=int), 512, 512) == (1 + 2 + 3 + 4) * 128 * 128
 
 
+def test_pair_slots_forward_half_window():
+    import numpy as np
+    # L = 512, n = 64: query tiles 1..3 have half windows (lower half of tile t-1 outside the
+    # band). Anchors: 10 in the lower half of tile 0, 3 in the lower half of tile 1, 7 in the
+    # lower half of tile 2 (words 4lo and 4lo + 1 of each tile).
+    bits = np.zeros((1, 16), dtype=np.int64)
+    bits[0, 0] = (1 << 10) - 1
+    bits[0, 4] = 0b111
+    bits[0, 9] = (1 << 7) - 1
+    # gather_end (anchors left of tile lo): t = 2 sees the 10 of tile 0 plus more in its upper
+    # half (say 40 in all), t = 3 sees 170
+    ge = np.array([[0, 0, 40, 170]])
+    slots = bench.pair_slots(ge, 512, 64, bits)
+    # t=0: 1 tile; t=1: G = 0 + 10 <= 64 -> 2 window tiles, no chunk; t=2: G = 43 -> 2;
+    # t=3: G = 177 -> 2 + ceil(113 / 128) = 3
+    assert slots == (1 + 2 + 2 + 3) * 128 * 128
+    # without the bits (dQ, dK/dV): whole chunks of gather_end
+    assert bench.pair_slots(ge, 512, 64) == (1 + 2 + 3 + 4) * 128 * 128
+    # n = 128: no half windows (the band reaches the lower half), same as without bits
+    assert bench.pair_slots(ge, 512, 128, bits) == bench.pair_slots(ge, 512, 128)
+
+
 def test_roofline_tensor_pass():
     step = types.SimpleNamespace(flops_fwd=8.0e9, bytes_dec=2.0e8)
     peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6500.0}

@@ -335,7 +335,7 @@ def train_components(step, comps, peaks, peak_src):
     computed_over_kept = slots / step.kept
     rows = {}
     for name, flops, sl in (("fwd_kernel", step.flops_fwd, slots_fwd),
-                            ("bwd_dq", 1.5 * step.flops_fwd, slots),
+                            ("bwd_dq", 1.5 * step.flops_fwd, slots_fwd),
                             ("bwd_dkdv", 2.0 * step.flops_fwd, slots)):
         r = roofline_for(name, comps, step, peaks, peak_src)
         rows[name] = {"us": comps[name] * 1e3, "tflops": r["achieved"], "frac_bf16_peak": r["frac"],
@@ -530,9 +530,10 @@ def attn_pass_bytes(B, L, Hq, Hkv, d, name):
 def pair_slots(gather_end, L, n, anchor_bits=None):
     """Query-key pair slots the attention kernels compute per head (summed over the batch):
     every query tile t runs whole 128 x 128 tiles over its window key tiles lo(t)..t and over
-    ceil(gather_end[t] / 128) compacted anchor chunks (the dQ and dK/dV passes; the latter
-    visits the same (query tile, key unit) pairs key-major).
-    With anchor_bits ([B, W] anchor flags), the forward's count: a query tile whose oldest
+    ceil(gather_end[t] / 128) compacted anchor chunks (the dK/dV pass, which visits these
+    (query tile, key unit) pairs key-major).
+    With anchor_bits ([B, W] anchor flags), the count of the forward and dQ passes: a query
+    tile whose oldest
     window tile's lower 64 keys lie outside every row's band (128 t - n + 1 >= 128 lo + 64)
     gathers their anchors too (G = gather_end + their count), and the first 64 gathered anchors
     fill that half of the tile, so ceil(max(0, G - 64) / 128) chunks follow."""

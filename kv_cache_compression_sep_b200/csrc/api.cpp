@@ -204,7 +204,10 @@ static int attn_bwd_impl(int stages, const sep_bf16* q, const sep_bf16* k, const
       !encode_map(&maps.v, v, B, L, Hkv, d) || !encode_map(&maps.kc, kc, B, L, Hkv, d) ||
       !encode_map(&maps.vc, vc, B, L, Hkv, d) || !encode_map(&maps.o, o, B, L, Hq, d) ||
       !encode_map(&maps.dout, dout, B, L, Hq, d) || !encode_map(&maps.dq, dq, B, L, Hq, d) ||
-      !encode_map(&maps.dk, dk, B, L, Hkv, d) || !encode_map(&maps.dv, dv, B, L, Hkv, d))
+      !encode_map(&maps.dk, dk, B, L, Hkv, d) || !encode_map(&maps.dv, dv, B, L, Hkv, d) ||
+      !encode_map(&maps.k64, k, B, L, Hkv, d, 64) || !encode_map(&maps.v64, v, B, L, Hkv, d, 64) ||
+      !encode_map(&maps.kc64, kc, B, L, Hkv, d, 64) ||
+      !encode_map(&maps.vc64, vc, B, L, Hkv, d, 64))
     return SEP_ERR_CUDA;
   AttnShape sh{B, L, Hq, Hkv, d, a, n, scale};
   return cuda_status(sep::launch_attn_bwd(

@@ -37,7 +37,8 @@ constexpr int kBoxBytes = 128 * 64 * 2;
 //   Delta[b][h][i] = sum_c dO[b,i,h,c] * O[b,i,h,c] for every query head h (the O and dO rows of
 //   position i are Hq * d contiguous bf16: 16-byte chunks, D / 8 consecutive chunks per head,
 //   summed over the D / 8 lanes that hold them);
-//   row i of the compacted anchor K / V (i < roundup128(cnt));
+//   row i of the compacted anchor K / V (i < cnt + 128: the 128 rows after the last anchor are
+//   zeros, for the anchor chunks of the dQ pass that start at 64 + a multiple of 128);
 //   zero row i of the compact fp32 anchor partials (i < cnt);
 //   and the four work-list counters (block 0).
 template <int D>
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     }
   }
   const int cnt = __ldg(anchor_cnt + b);
-  if (i < min(L, (cnt + 127) / 128 * 128))
+  if (i < min(L, cnt + 128))
     compact_anchor_row(k, v, anchor_idx, cnt, L, b, i, Hkv * D / 8, kc, vc, lane);
   if (i < cnt) {
     const int pc = Hkv * D / 4;
@@ -107,6 +108,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
 // ------------------------------------------------------------------ shared parameter block
 struct BwdParams {
   CUtensorMap tmQ, tmK, tmV, tmKc, tmVc, tmdO, tmdQ, tmdK, tmdV;
+  CUtensorMap tmK64, tmV64, tmKc64, tmVc64;  // 64-row boxes: the halves of a merged tile (dQ)
   const uint32_t* anchor_bits;  // [B, W] packed anchor flags
   const int32_t* anchor_idx;
   const int32_t* anchor_cnt;
@@ -156,8 +158,14 @@ constexpr size_t dq_smem_bytes() {
   return 1024 + DqCfg<D>::SMEM_TILES + sizeof(DqBar<DqCfg<D>::NST, DqCfg<D>::DOB>);
 }
 
+// Items of the dQ pass, with the forward's half-window rule: when the lower 64 keys of the
+// oldest window tile lo lie outside every row's band (128 t - n + 1 >= 128 lo + 64), their
+// anchors join the gathered ones (ge counts both), the oldest window tile is merged (lower half:
+// compacted anchors 0..63; upper half: keys 128 lo + 64 ..) and the anchor chunks start at
+// compacted row arow0 = 64.
 struct BwdItem {
-  int t, h, b, nwin, ge, N;
+  int t, h, b, nwin, ge, N, arow0;
+  bool half;
 };
 __device__ __forceinline__ BwdItem bwd_item_base(const BwdParams& p, int x) {
   BwdItem it;
@@ -166,19 +174,27 @@ __device__ __forceinline__ BwdItem bwd_item_base(const BwdParams& p, int x) {
   const int rem = x % per_t;
   it.h = rem % p.Hq;
   it.b = rem / p.Hq;
-  it.nwin = it.t - window_lo_tile(it.t, p.n) + 1;
+  const int lo = window_lo_tile(it.t, p.n);
+  it.nwin = it.t - lo + 1;
+  it.half = lo < it.t && (long long)it.t * 128 - p.n + 1 >= (long long)lo * 128 + 64;
+  it.arow0 = it.half ? 64 : 0;
   it.ge = 0;
   it.N = it.nwin;
   return it;
 }
 __device__ __forceinline__ int bwd_item_ge(const BwdParams& p, int x) {
   const BwdItem it = bwd_item_base(p, x);
-  return p.gather_end[(size_t)it.b * p.T + it.t];
+  int ge = p.gather_end[(size_t)it.b * p.T + it.t];
+  if (it.half) {
+    const uint32_t* w = p.anchor_bits + (size_t)it.b * p.W + (size_t)(it.t - it.nwin + 1) * 4;
+    ge += __popc(__ldg(w)) + __popc(__ldg(w + 1));
+  }
+  return ge;
 }
 __device__ __forceinline__ BwdItem bwd_item_with(const BwdParams& p, int x, int ge) {
   BwdItem it = bwd_item_base(p, x);
   it.ge = ge;
-  it.N = it.nwin + (ge + 127) / 128;
+  it.N = it.nwin + (max(0, ge - it.arow0) + 127) / 128;
   return it;
 }
 struct BwdTileRaw {
@@ -283,24 +299,37 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
           }
           const int st = g % NST, r = g / NST;
           const bool win = j < it.nwin;
-          const int row0 = win ? (it.t - j) * 128 : (j - it.nwin) * 128;
+          const bool merged = it.half && j == it.nwin - 1;
+          const int row0 = win ? (it.t - j) * 128 : it.arow0 + (j - it.nwin) * 128;
           if (r > 0 && !mbar_wait(&bar->k_empty[st], (r - 1) & 1, p.err, abort_flag)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&bar->k_full[st], C::TILE);
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_4d(sK + st * C::TILE + kb * kBoxBytes, win ? &p.tmK : &p.tmKc,
-                        &bar->k_full[st], kb * 64, kvh, row0, it.b);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            uint8_t* dst = sK + st * C::TILE + kb * kBoxBytes;
+            if (merged) {  // compacted anchors 0..63, then keys 128 lo + 64 ..
+              tma_load_4d(dst, &p.tmKc64, &bar->k_full[st], kb * 64, kvh, 0, it.b);
+              tma_load_4d(dst + 64 * 128, &p.tmK64, &bar->k_full[st], kb * 64, kvh, row0 + 64, it.b);
+            } else {
+              tma_load_4d(dst, win ? &p.tmK : &p.tmKc, &bar->k_full[st], kb * 64, kvh, row0, it.b);
+            }
+          }
           if (r > 0 && !mbar_wait(&bar->v_empty[st], (r - 1) & 1, p.err, abort_flag)) {
             mbar_wait(&bar->k_full[st], r & 1, nullptr, nullptr);
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&bar->v_full[st], C::TILE);
-          for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_4d(sV + st * C::TILE + kb * kBoxBytes, win ? &p.tmV : &p.tmVc,
-                        &bar->v_full[st], kb * 64, kvh, row0, it.b);
+          for (int kb = 0; kb < C::KB; ++kb) {
+            uint8_t* dst = sV + st * C::TILE + kb * kBoxBytes;
+            if (merged) {
+              tma_load_4d(dst, &p.tmVc64, &bar->v_full[st], kb * 64, kvh, 0, it.b);
+              tma_load_4d(dst + 64 * 128, &p.tmV64, &bar->v_full[st], kb * 64, kvh, row0 + 64, it.b);
+            } else {
+              tma_load_4d(dst, win ? &p.tmV : &p.tmVc, &bar->v_full[st], kb * 64, kvh, row0, it.b);
+            }
+          }
         }
       }
       if (!ok) {
@@ -438,7 +467,12 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
           cur = bwd_tile_raw(p, fn.b, fn.t, fn.t);
         }
         uint32_t keep[2] = {0xffffffffu, 0xffffffffu};
-        if (j < it.nwin) {
+        if (it.half && j == it.nwin - 1 && wg == 0) {
+          // lower half of the merged tile: gathered anchors 0..63, kept by every row
+          const int cnt = min(it.ge, 64);
+#pragma unroll
+          for (int w = 0; w < 2; ++w) keep[w] = range_word(0, cnt - 1, w);
+        } else if (j < it.nwin) {
           const int u = it.t - j;
           const long long k0 = (long long)u * 128;
           if (raw.cls != SEP_TILE_FULL) {
@@ -450,7 +484,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
             for (int w = 0; w < 2; ++w) keep[w] = range_word(0, (long long)p.L - 1 - k0, 2 * wg + w);
           }
         } else {
-          const int rem = it.ge - (j - it.nwin) * 128;
+          const int rem = it.ge - it.arow0 - (j - it.nwin) * 128;
           if (rem < 128) {
 #pragma unroll
             for (int w = 0; w < 2; ++w) keep[w] = range_word(0, rem - 1, 2 * wg + w);
@@ -1439,6 +1473,10 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   prm.tmKc = maps.kc;
   prm.tmVc = maps.vc;
   prm.tmdO = maps.dout;
+  prm.tmK64 = maps.k64;
+  prm.tmV64 = maps.v64;
+  prm.tmKc64 = maps.kc64;
+  prm.tmVc64 = maps.vc64;
   prm.tmdQ = maps.dq;
   prm.tmdK = maps.dk;
   prm.tmdV = maps.dv;

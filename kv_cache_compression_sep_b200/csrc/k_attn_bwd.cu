@@ -1064,67 +1064,37 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
           c = n;
         }
       } else {
-      // S cursor cs (at most NB half-pairs ahead) and G cursor cg; nS / nG half-pairs issued.
-      // The item a cursor moves into is read from the item ring: the S cursor waits for it to be
-      // published, which needs the epilogue of item I - KVB (its K/V buffer), so it does so only
-      // once every G of that item has been issued (s_end[I & 1]: half-pairs up to its end).
-      Cur cs, cg;
-      int nS = 0, nG = 0;
-      int s_end[2] = {0, 0};
-      bool s_pending = false;  // cs entered item cs.I, not yet loaded
-      bool g_pending = false;  // cg entered item cg.I, header not yet read
-      cs.I = 0;
-      cs.P = 0;
-      cs.h = 0;
-      ok = load_item(cs);
-      cg = cs;
-      for (;;) {
-        // S as far ahead as the buffers allow
-        while (ok && nS < nG + NB) {
-          if (s_pending) {
-            if (cs.I >= KVB && nG < s_end[(cs.I - KVB) & 1]) break;
-            ok = load_item(cs);
-            s_pending = false;
-            if (!ok) break;
-          }
-          if (cs.x >= nitems) break;
-          ok = issue_S(cs);
-          ++nS;
-          if (!ok) break;
-          if (cs.h == 0) {
-            cs.h = 1;
+        // per 64-query half h: G(P, A), S(P+1, A), G(P, B), S(P+1, B), so that half A's next
+        // softmax can run while half B's is still working; with one K/V buffer the next item
+        // is published only after this item's epilogue, so both G of an item's last pair come
+        // before the next item's S
+        auto S_h = [&](Cur c, int h) { c.h = h; return issue_S(c); };
+        auto G_h = [&](Cur c, int h) { c.h = h; return issue_G(c); };
+        Cur c;
+        c.I = 0;
+        c.P = 0;
+        c.h = 0;
+        ok = load_item(c);
+        if (ok && c.x < nitems) ok = S_h(c, 0) && S_h(c, 1);
+        while (ok && c.x < nitems) {
+          Cur n = c;
+          ++n.P;
+          if (c.q + 1 < c.it.npairs) {
+            ++n.q;
+            ok = G_h(c, 0) && S_h(n, 0) && G_h(c, 1) && S_h(n, 1);
+          } else if (KVB == 1) {
+            ++n.I;
+            ok = G_h(c, 0) && G_h(c, 1) && load_item(n);
+            if (ok && n.x < nitems) ok = S_h(n, 0) && S_h(n, 1);
           } else {
-            cs.h = 0;
-            ++cs.P;
-            if (++cs.q >= cs.it.npairs) {
-              s_end[cs.I & 1] = nS;
-              ++cs.I;
-              s_pending = true;
-            }
+            ++n.I;
+            ok = load_item(n);
+            const bool more = ok && n.x < nitems;
+            ok = ok && G_h(c, 0) && (!more || S_h(n, 0)) && G_h(c, 1) && (!more || S_h(n, 1));
           }
-        }
-        if (!ok || nG >= nS) break;
-        if (g_pending) {
-          cg.x = bar->item[cg.I & 3].x;  // published: the S cursor has waited for it
-          cg.q = 0;
-          cg.it = slot_item(bar->item[cg.I & 3], p.Hkv, G);
-          g_pending = false;
-        }
-        ok = issue_G(cg);
-        ++nG;
-        if (!ok) break;
-        if (cg.h == 0) {
-          cg.h = 1;
-        } else {
-          cg.h = 0;
-          ++cg.P;
-          if (++cg.q >= cg.it.npairs) {
-            ++cg.I;
-            g_pending = true;
-          }
+          c = n;
         }
       }
-      }  // half-pair path
       tc_commit(&bar->drain);
       mbar_wait(&bar->drain, 0, nullptr, nullptr);
     }

@@ -23,6 +23,7 @@
 //      (window part + every gathered part) in a compact [B, anchors, Hkv, d] buffer.
 //   4. combine: anchor partials to bf16 dK/dV at the anchors' positions.
 #include <cuda_runtime.h>
+#include <cstddef>
 
 #include "sep_common.cuh"
 #include "sep_launch.h"
@@ -719,13 +720,20 @@ struct DkvBar {
   uint64_t drain;
   uint64_t item_full[4];  // ring of fetched work items (producer -> MMA, softmax, storer)
   ItemSlot item[4];
-  float nlse2[NST][128];  // -log2-domain LSE of each query of the stage (-inf past L)
-  float delta[NST][128];
+  alignas(16) float nlse2[NST][128];  // -log2-domain LSE of each query of the stage (-inf past L)
+  alignas(16) float delta[NST][128];
   int pin[NST];           // mask input of the stage's pair: tile class (window) or gather_end
   uint32_t tmem_base;
   int abort_flag;
 };
 
+// the softmax reads the per-query statistics four at a time (16-byte shared-memory loads)
+using DkvBar128 = DkvBar<DkvCfg<128>::NST, DkvCfg<128>::KVB, DkvCfg<128>::NB>;
+using DkvBar64 = DkvBar<DkvCfg<64>::NST, DkvCfg<64>::KVB, DkvCfg<64>::NB>;
+static_assert(offsetof(DkvBar128, nlse2) % 16 == 0 && offsetof(DkvBar128, delta) % 16 == 0,
+              "16-byte aligned statistics");
+static_assert(offsetof(DkvBar64, nlse2) % 16 == 0 && offsetof(DkvBar64, delta) % 16 == 0,
+              "16-byte aligned statistics");
 template <int D>
 constexpr size_t dkv_smem_bytes() {
   return 1024 + DkvCfg<D>::SMEM_TILES +
@@ -1200,13 +1208,19 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         auto pds_chunk = [&](int ch, const uint32_t(&sv)[32], const uint32_t(&dp)[32],
                              uint32_t(&pk)[16], uint32_t(&dk16)[16]) {
           const float2 sl2x2 = make_float2(sl2, sl2);
+          float4 nl4 = make_float4(0.f, 0.f, 0.f, 0.f), dl4 = nl4;
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const int col = 32 * ch + c;
+            if ((c & 3) == 0) {
+              nl4 = *reinterpret_cast<const float4*>(nlse2 + col);
+              dl4 = *reinterpret_cast<const float4*>(dl + col);
+            }
+            const float2 nlp = (c & 3) ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+            const float2 dlp = (c & 3) ? make_float2(dl4.z, dl4.w) : make_float2(dl4.x, dl4.y);
             const float2 x = f2_fma(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
-                                    sl2x2, *reinterpret_cast<const float2*>(nlse2 + col));
-            const float2 dd = f2_sub(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
-                                     *reinterpret_cast<const float2*>(dl + col));
+                                    sl2x2, nlp);
+            const float2 dd = f2_sub(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), dlp);
             const float p0 = ((keep[ch] >> c) & 1u) ? ex2(x.x) : 0.f;
             const float p1 = ((keep[ch] >> (c + 1)) & 1u) ? ex2(x.y) : 0.f;
             const float2 ds = f2_mul(make_float2(p0, p1), dd);

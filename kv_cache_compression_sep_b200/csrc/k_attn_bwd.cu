@@ -24,6 +24,7 @@
 //   4. combine: anchor partials to bf16 dK/dV at the anchors' positions.
 #include <cuda_runtime.h>
 #include <cstddef>
+#include <type_traits>
 
 #include "sep_common.cuh"
 #include "sep_launch.h"
@@ -509,15 +510,19 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         tc_fence_before();
         mbar_arrive(&bar->s_free);  // S and dP may be overwritten by the next tile's MMAs
 #pragma unroll
+        // two columns per packed fp32x2 instruction: x = S * scale*log2(e) - lse2, P = exp2(x)
+        // on kept pairs, dS = P (dP - Delta)
+        const float2 sl2x2 = make_float2(sl2, sl2), nl2 = make_float2(-lse2, -lse2);
+        const float2 ndl2 = make_float2(-dlt, -dlt);
         for (int c = 0; c < 64; c += 2) {
-          float v[2];
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const bool kp = (keep[(c + q) >> 5] >> ((c + q) & 31)) & 1u;
-            const float pr = kp ? ex2(fmaf(__uint_as_float(sv[c + q]), sl2, -lse2)) : 0.f;
-            v[q] = pr * (__uint_as_float(dp[c + q]) - dlt);
-          }
-          sv[c >> 1] = pack_bf16x2(v[0], v[1]);
+          const float2 x = f2_fma(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
+                                  sl2x2, nl2);
+          const float2 dd = f2_add(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                   ndl2);
+          const float p0 = ((keep[c >> 5] >> (c & 31)) & 1u) ? ex2(x.x) : 0.f;
+          const float p1 = ((keep[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u) ? ex2(x.y) : 0.f;
+          const float2 v = f2_mul(make_float2(p0, p1), dd);
+          sv[c >> 1] = pack_bf16x2(v.x, v.y);
         }
         // dS has one buffer: the previous tile's dQ MMA must have read it
         if (g > 0 &&
@@ -1205,8 +1210,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
         const float* dl = &bar->delta[st][64 * h];
         // one 32-column chunk: x = S * scale*log2(e) - lse2 (two queries per packed fp32x2
         // instruction), P = exp2(x) on kept pairs, dS = P (dP - Delta), both packed to bf16
-        auto pds_chunk = [&](int ch, const uint32_t(&sv)[32], const uint32_t(&dp)[32],
-                             uint32_t(&pk)[16], uint32_t(&dk16)[16]) {
+        auto pds_chunk = [&](auto all_kept, int ch, const uint32_t(&sv)[32],
+                             const uint32_t(&dp)[32], uint32_t(&pk)[16], uint32_t(&dk16)[16]) {
+          constexpr bool kAll = decltype(all_kept)::value;
           const float2 sl2x2 = make_float2(sl2, sl2);
           float4 nl4 = make_float4(0.f, 0.f, 0.f, 0.f), dl4 = nl4;
 #pragma unroll
@@ -1221,8 +1227,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
             const float2 x = f2_fma(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
                                     sl2x2, nlp);
             const float2 dd = f2_sub(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), dlp);
-            const float p0 = ((keep[ch] >> c) & 1u) ? ex2(x.x) : 0.f;
-            const float p1 = ((keep[ch] >> (c + 1)) & 1u) ? ex2(x.y) : 0.f;
+            const float p0 = (kAll || ((keep[ch] >> c) & 1u)) ? ex2(x.x) : 0.f;
+            const float p1 = (kAll || ((keep[ch] >> (c + 1)) & 1u)) ? ex2(x.y) : 0.f;
             const float2 ds = f2_mul(make_float2(p0, p1), dd);
             pk[c >> 1] = pack_bf16x2(p0, p1);
             dk16[c >> 1] = pack_bf16x2(ds.x, ds.y);
@@ -1234,6 +1240,8 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
           const uint32_t aS = tmem + lane_off + C::COL_S + 64 * h;
           const uint32_t aD = tmem + lane_off + C::COL_DPW + 64 * h;
           uint32_t pk[2][16], dk16[2][16];
+          // every row of the warp keeps all 64 query columns (e.g. anchor items): no selects
+          const bool all_kept = __all_sync(0xffffffffu, (keep[0] & keep[1]) == 0xffffffffu);
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             uint32_t sv[32], dp[32];
@@ -1244,7 +1252,10 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
               tc_fence_before();
               mbar_arrive(&bar->s_free);  // the next pair's S^T / dP^T may overwrite them
             }
-            pds_chunk(ch, sv, dp, pk[ch], dk16[ch]);
+            if (all_kept)
+              pds_chunk(std::true_type{}, ch, sv, dp, pk[ch], dk16[ch]);
+            else
+              pds_chunk(std::false_type{}, ch, sv, dp, pk[ch], dk16[ch]);
           }
           if (P > 0 && !__all_sync(0xffffffffu,
                                    mbar_wait(&bar->mm_done[0], (P - 1) & 1, p.err, abort_flag))) {
@@ -1267,7 +1278,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
             tmem_ld32(aP + 32 * ch, dp);
             tmem_ld_wait();
             uint32_t pk[16], dk16[16];
-            pds_chunk(ch, sv, dp, pk, dk16);
+            pds_chunk(std::false_type{}, ch, sv, dp, pk, dk16);
             tmem_st16(aS + 16 * ch, pk);
             tmem_st16(aP + 16 * ch, dk16);
           }

@@ -509,11 +509,11 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
         }
         tc_fence_before();
         mbar_arrive(&bar->s_free);  // S and dP may be overwritten by the next tile's MMAs
-#pragma unroll
         // two columns per packed fp32x2 instruction: x = S * scale*log2(e) - lse2, P = exp2(x)
         // on kept pairs, dS = P (dP - Delta)
         const float2 sl2x2 = make_float2(sl2, sl2), nl2 = make_float2(-lse2, -lse2);
         const float2 ndl2 = make_float2(-dlt, -dlt);
+#pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float2 x = f2_fma(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])),
                                   sl2x2, nl2);

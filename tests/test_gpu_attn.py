@@ -56,6 +56,8 @@ SMALL = [
     (1, 700, 4, 1, 128, 3, 1000, 0.1),
     (1, 1030, 2, 1, 64, 4, 64, 0.3),
     (1, 333, 8, 8, 128, 0, 5, 0.0),
+    (1, 520, 4, 2, 64, 2, 65, 0.15),    # the widest band with half-window pairs at d = 64
+    (1, 300, 2, 1, 64, 1, 5, 0.2),      # a narrow band: half-window pairs, few kept per row
 ]
 
 

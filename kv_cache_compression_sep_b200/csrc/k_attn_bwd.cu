@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(
     const int32_t* __restrict__ anchor_cnt, int L, int Hq, int Hkv,
     uint4* __restrict__ kc, uint4* __restrict__ vc, float4* __restrict__ dka,
     float4* __restrict__ dva, float* __restrict__ delta, int32_t* __restrict__ counters) {
+  grid_dep_wait();
+  grid_dep_launch_next();
   constexpr int CPH = D / 8;  // 16-byte chunks per head; divides 32
   const int b = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -261,6 +263,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  grid_dep_wait();
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -567,6 +570,7 @@ __global__ void __launch_bounds__(DqCfg<D>::THREADS, 1)
     }
     tc_fence_before();
   }
+  grid_dep_launch_next();  // the next kernel of the stream may start its prologue
   __syncthreads();
   if (warp == 9) {
     tc_fence_after();
@@ -596,6 +600,8 @@ __global__ void __launch_bounds__(1024) bwd_schedule_kernel(
     const uint32_t* __restrict__ anchor_bits, int L, int n, int T, int W, int32_t* __restrict__ tile_prefix,
     WorkItem* __restrict__ anchor_items, WorkItem* __restrict__ window_items,
     int32_t* __restrict__ counters /* [0] anchor items, [1] window items; [2], [3] dK/dV pass */) {
+  grid_dep_wait();
+  grid_dep_launch_next();
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   __shared__ int s_warp[32];
@@ -785,8 +791,6 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
   using C = DkvCfg<D>;
   constexpr int NST = C::NST, KVB = C::KVB, NB = C::NB;
   const int G = p.Hq / p.Hkv;
-  const int n_anchor = counters[0];
-  const int nitems = (n_anchor + counters[1]) * p.Hkv;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -830,6 +834,9 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  grid_dep_wait();
+  const int n_anchor = counters[0];
+  const int nitems = (n_anchor + counters[1]) * p.Hkv;
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer (whole warp)
@@ -1353,6 +1360,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     }
     tc_fence_before();
   }
+  grid_dep_launch_next();  // the next kernel of the stream may start its prologue
   __syncthreads();
   if (warp == 9) {
     tc_fence_after();
@@ -1376,6 +1384,8 @@ __global__ void __launch_bounds__(256) anchor_combine_kernel(
     const int32_t* __restrict__ anchor_idx, const int32_t* __restrict__ anchor_cnt, int L, int q4,
     const float4* __restrict__ dka, const float4* __restrict__ dva, uint2* __restrict__ dk,
     uint2* __restrict__ dv) {
+  grid_dep_wait();
+  grid_dep_launch_next();
   const int b = blockIdx.y;
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= __ldg(anchor_cnt + b)) return;
@@ -1450,15 +1460,17 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   if (stages & kBwdPrep) {
     const dim3 pgrid((s.L + 7) / 8, s.B);
     auto prep = (s.d == 128) ? bwd_prep_kernel<128> : bwd_prep_kernel<64>;
-    prep<<<pgrid, 256, 0, stream>>>(
-        static_cast<const uint4*>(o), static_cast<const uint4*>(dout), static_cast<const uint4*>(k),
-        static_cast<const uint4*>(v), anchor_idx, anchor_cnt, s.L, s.Hq, s.Hkv,
-        static_cast<uint4*>(kc), static_cast<uint4*>(vc), reinterpret_cast<float4*>(dka),
-        reinterpret_cast<float4*>(dva), delta, counters);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_schedule_kernel<<<s.B, 1024, 0, stream>>>(anchor_cnt, gather_end, anchor_bits, s.L, s.n,
-                                                  T, W, tile_prefix, aitems, witems, counters);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_chained(prep, pgrid, dim3(256), 0, stream, static_cast<const uint4*>(o),
+                       static_cast<const uint4*>(dout), static_cast<const uint4*>(k),
+                       static_cast<const uint4*>(v), anchor_idx, anchor_cnt, s.L, s.Hq, s.Hkv,
+                       static_cast<uint4*>(kc), static_cast<uint4*>(vc),
+                       reinterpret_cast<float4*>(dka), reinterpret_cast<float4*>(dva), delta,
+                       counters);
+    if (e != cudaSuccess) return e;
+    e = launch_chained(bwd_schedule_kernel, dim3(s.B), dim3(1024), 0, stream, anchor_cnt,
+                       gather_end, anchor_bits, s.L, s.n, T, W, tile_prefix, aitems, witems,
+                       counters);
+    if (e != cudaSuccess) return e;
   }
   if (!(stages & (kBwdDq | kBwdDkv))) return cudaSuccess;
   BwdParams prm;
@@ -1503,29 +1515,35 @@ cudaError_t launch_attn_bwd(const AttnMaps& maps, const AttnShape& s, const uint
   const int grid_q = dq_items < nsm ? dq_items : nsm;
   if (s.d == 128) {
     if ((e = set_bwd_attrs<128>()) != cudaSuccess) return e;
-    if (stages & kBwdDq)
-      sep_attn_bwd_dq_kernel<128><<<grid_q, DqCfg<128>::THREADS, dq_smem_bytes<128>(), stream>>>(prm, dq_items);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (stages & kBwdDkv)
-      sep_attn_bwd_dkv_kernel<128><<<nsm, DkvCfg<128>::THREADS, dkv_smem_bytes<128>(), stream>>>(
-          prm, aitems, witems, counters, tile_prefix);
+    if ((stages & kBwdDq) &&
+        (e = launch_chained(sep_attn_bwd_dq_kernel<128>, dim3(grid_q), dim3(DqCfg<128>::THREADS),
+                            dq_smem_bytes<128>(), stream, prm, dq_items)) != cudaSuccess)
+      return e;
+    if ((stages & kBwdDkv) &&
+        (e = launch_chained(sep_attn_bwd_dkv_kernel<128>, dim3(nsm), dim3(DkvCfg<128>::THREADS),
+                            dkv_smem_bytes<128>(), stream, prm, aitems, witems, counters,
+                            tile_prefix)) != cudaSuccess)
+      return e;
   } else {
     if ((e = set_bwd_attrs<64>()) != cudaSuccess) return e;
-    if (stages & kBwdDq)
-      sep_attn_bwd_dq_kernel<64><<<grid_q, DqCfg<64>::THREADS, dq_smem_bytes<64>(), stream>>>(prm, dq_items);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (stages & kBwdDkv)
-      sep_attn_bwd_dkv_kernel<64><<<nsm, DkvCfg<64>::THREADS, dkv_smem_bytes<64>(), stream>>>(
-          prm, aitems, witems, counters, tile_prefix);
+    if ((stages & kBwdDq) &&
+        (e = launch_chained(sep_attn_bwd_dq_kernel<64>, dim3(grid_q), dim3(DqCfg<64>::THREADS),
+                            dq_smem_bytes<64>(), stream, prm, dq_items)) != cudaSuccess)
+      return e;
+    if ((stages & kBwdDkv) &&
+        (e = launch_chained(sep_attn_bwd_dkv_kernel<64>, dim3(nsm), dim3(DkvCfg<64>::THREADS),
+                            dkv_smem_bytes<64>(), stream, prm, aitems, witems, counters,
+                            tile_prefix)) != cudaSuccess)
+      return e;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (stages & kBwdDkv) {
     dim3 grid((s.L + 7) / 8, s.B);
-    anchor_combine_kernel<<<grid, 256, 0, stream>>>(
-        anchor_idx, anchor_cnt, s.L, s.Hkv * s.d / 4, reinterpret_cast<const float4*>(dka),
-        reinterpret_cast<const float4*>(dva), static_cast<uint2*>(dk), static_cast<uint2*>(dv));
+    return launch_chained(anchor_combine_kernel, grid, dim3(256), 0, stream, anchor_idx,
+                          anchor_cnt, s.L, s.Hkv * s.d / 4, reinterpret_cast<const float4*>(dka),
+                          reinterpret_cast<const float4*>(dva), static_cast<uint2*>(dk),
+                          static_cast<uint2*>(dv));
   }
-  return cudaGetLastError();
+  return cudaSuccess;
 }
 
 }  // namespace sep

@@ -201,6 +201,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  grid_dep_wait();
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -595,6 +596,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     tc_fence_before();
   }
 
+  grid_dep_launch_next();  // the next kernel of the stream may start its prologue
   __syncthreads();
   if (warp == 9) {
     tc_fence_after();
@@ -612,6 +614,8 @@ __global__ void __launch_bounds__(256) compact_anchors_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, const int32_t* __restrict__ anchor_idx,
     const int32_t* __restrict__ anchor_cnt, int L, int kv_ch, uint4* __restrict__ kc,
     uint4* __restrict__ vc) {
+  grid_dep_wait();
+  grid_dep_launch_next();
   const int b = blockIdx.y;
   const int cnt = __ldg(anchor_cnt + b);
   const int pad_end = min(L, cnt + 128);
@@ -625,10 +629,9 @@ cudaError_t launch_compact_anchors(const void* k, const void* v, const int32_t* 
                                    void* kc, void* vc, cudaStream_t stream) {
   const int kv_ch = Hkv * d * 2 / 16;
   dim3 grid((L + 7) / 8, B);
-  compact_anchors_kernel<<<grid, 256, 0, stream>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), anchor_idx, anchor_cnt, L,
-      kv_ch, static_cast<uint4*>(kc), static_cast<uint4*>(vc));
-  return cudaGetLastError();
+  return launch_chained(compact_anchors_kernel, grid, dim3(256), 0, stream,
+                        static_cast<const uint4*>(k), static_cast<const uint4*>(v), anchor_idx,
+                        anchor_cnt, L, kv_ch, static_cast<uint4*>(kc), static_cast<uint4*>(vc));
 }
 
 static int sm_count() {
@@ -660,8 +663,8 @@ static cudaError_t launch_fwd_t(const FwdParams& prm, int T, int Hq, int B, cuda
   }
   const int nitems = T * Hq * B;
   const int grid = std::min(nitems, sm_count());
-  sep_attn_fwd_kernel<D><<<grid, FwdCfg<D>::THREADS, smem, stream>>>(prm, nitems);
-  return cudaGetLastError();
+  return launch_chained(sep_attn_fwd_kernel<D>, dim3(grid), dim3(FwdCfg<D>::THREADS), smem, stream,
+                        prm, nitems);
 }
 
 cudaError_t launch_attn_fwd(const AttnMaps& maps, const AttnShape& s, const uint32_t* anchor_bits,

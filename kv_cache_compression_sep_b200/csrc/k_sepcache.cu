@@ -130,6 +130,8 @@ __global__ void __launch_bounds__(kUpdateThreads) sepcache_update_kernel(
     uint4* __restrict__ v_slots, int32_t* __restrict__ slot_pos, uint8_t* __restrict__ slot_sep,
     int32_t* __restrict__ meta, const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
     const uint8_t* __restrict__ sep_new) {
+  grid_dep_wait();
+  grid_dep_launch_next();
   extern __shared__ int2 s_moves[];  // compression: (past slot, separator slot), min(s, P) at most
   const int Hkv = cd.Hkv, d = cd.d, a = cd.a, s = cd.s, w = cd.w, P = cd.P;
   const int seq = blockIdx.x;
@@ -629,6 +631,7 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
   using C = DecCfg<D, GP>;
   constexpr int LPK = C::LPK, NG = C::NG, KC = C::KC;
   constexpr int HALF = D / 2;
+  grid_dep_wait();
   const int kvh = blockIdx.x, seq = blockIdx.y;
   const int ns = p.a + p.s + p.P + p.w;
   const int tid = threadIdx.x, warp = tid >> 5, grp = tid / LPK, l = tid % LPK;
@@ -898,6 +901,7 @@ __global__ void __launch_bounds__(kDecThreads, (GP >= 8) ? 2 : 4)
         mbar_wait(&sm.full[ch % kDecStages], (ch / kDecStages) & 1, nullptr, nullptr);
     }
   }
+  grid_dep_launch_next();  // the cache is read: the next kernel of the stream may start
 
   // ---- every query's softmax state from the lanes that own it
   float mrun[GP], lrun[GP];
@@ -1021,11 +1025,11 @@ cudaError_t launch_sepcache_update(const SepCacheState& st, const void* k_new, c
                                    const uint8_t* sep_new, cudaStream_t stream) {
   const int P = past_slots(st);
   const size_t smem = (size_t)max(1, min(st.s, P)) * sizeof(int2);  // compression moves
-  sepcache_update_kernel<<<st.S, kUpdateThreads, smem, stream>>>(
-      cache_dims(st), st.rope_freq, reinterpret_cast<uint4*>(st.k_slots),
-      reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta,
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), sep_new);
-  return cudaGetLastError();
+  return launch_chained(sepcache_update_kernel, dim3(st.S), dim3(kUpdateThreads), smem, stream,
+                        cache_dims(st), st.rope_freq, reinterpret_cast<uint4*>(st.k_slots),
+                        reinterpret_cast<uint4*>(st.v_slots), st.slot_pos, st.slot_sep, st.meta,
+                        static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+                        sep_new);
 }
 
 cudaError_t launch_sepcache_prefill(const SepCacheState& st, const void* k, const void* v,
@@ -1075,8 +1079,8 @@ static cudaError_t launch_decode_t(const SepCacheState& st, const void* q, void*
   a.scale_log2 = scale * 1.4426950408889634f;
   a.err = device_error_word();
   dim3 grid(st.Hkv, st.S);
-  sepcache_decode_kernel<D, GP, ORIG><<<grid, kDecThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+  return launch_chained(sepcache_decode_kernel<D, GP, ORIG>, grid, dim3(kDecThreads), smem, stream,
+                        a);
 }
 
 template <int D, int GP>

@@ -60,6 +60,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Programmatic dependent launch (kernels started by launch_chained): the kernel may begin while
+// the previous kernel of its stream is still running. grid_dep_wait() returns once that grid has
+// completed and its memory writes are visible; every kernel calls it before its first access to
+// global memory. grid_dep_launch_next() lets the next kernel of the stream start its own prologue
+// (its CTAs take SMs as this grid's CTAs leave them).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Records a device-side failure: sticky error word (first code wins) and the CTA abort flag.
 __device__ __forceinline__ void record_failure(unsigned* err, volatile int* abort_flag,
                                                unsigned code) {

@@ -11,6 +11,26 @@
 
 namespace sep {
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous kernel
+// of the stream finishes (it waits for it in grid_dep_wait before touching global memory), so
+// that its launch and prologue overlap the other's tail. Every kernel of the library's training
+// and decode steps is started this way.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Device address of the sticky error word on the current device (nullptr on failure).
 unsigned* device_error_word();
 // Wall-clock limit of each pipeline wait of the attention forward kernel (sep_set_wait_limit_ns);

@@ -102,3 +102,25 @@ def test_long_context_sampled(S, n):
     tiles += [(int(t), int(u)) for t, u in zip(rng.integers(0, T, 60), rng.integers(0, T, 60))]
     for t, u in tiles:
         assert got["tile_map"][0, t, u] == R.tile_class(sep[0], cfg.a, n, 128, 128, t, u), (t, u)
+
+
+def test_tile_map_both_count_paths():
+    """Tile classes from the staged flag words (L <= 192000) and from the binary search over the
+    anchor list (longer sequences): the same gather ends and classes as the oracle, sampled."""
+    import torch
+    from kv_cache_compression_sep_b200 import sepattn as S
+    for L in (192000, 196608 + 77):  # 6000 flag words (staged), 6147 (binary search)
+        rng = np.random.default_rng(L)
+        sep = (rng.random((1, L)) < 0.08).astype(np.uint8)
+        n, a = 200, 3
+        got = _run(S, sep, a, n, 128, 128)
+        f = R.anchor_flags(sep[0], a)
+        pos = np.nonzero(f)[0]
+        T = -(-L // 128)
+        lo = np.maximum(0, np.arange(T) * 128 - n + 1) // 128 * 128
+        np.testing.assert_array_equal(got["gather_end"][0], np.searchsorted(pos, lo, side="left"))
+        tiles = [(0, 0), (T - 1, T - 1), (T - 1, 0), (T - 1, T - 2), (T - 1, T - 3), (700, 698)]
+        tiles += [(int(t), int(u)) for t, u in zip(rng.integers(0, T, 40), rng.integers(0, T, 40))]
+        for t, u in tiles:
+            assert got["tile_map"][0, t, u] == R.tile_class(sep[0], a, n, 128, 128, t, u), (L, t, u)
+    torch.cuda.synchronize()

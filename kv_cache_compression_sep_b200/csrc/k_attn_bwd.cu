@@ -727,6 +727,7 @@ struct DkvBar {
   // done; wide: S^T / dP^T read by both warpgroups (s_free)
   uint64_t s_full[NB], pds_ready[NB], mm_done[NB], s_free;
   uint64_t acc_full, acc_free;
+  uint64_t acc_dv;        // wide: the item's dV products are done (its dK products may still run)
   uint64_t staged[KVB];   // the item's dK/dV rows are in the K/V buffer (softmax -> storer)
   uint64_t drain;
   uint64_t item_full[4];  // ring of fetched work items (producer -> MMA, softmax, storer)
@@ -819,6 +820,7 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
     }
     mbar_init(&bar->s_free, 256);
     mbar_init(&bar->acc_full, 1);
+    mbar_init(&bar->acc_dv, 1);
     mbar_init(&bar->acc_free, 256);
     for (int s = 0; s < KVB; ++s) mbar_init(&bar->staged[s], 256);
     mbar_init(&bar->drain, 1);
@@ -1036,14 +1038,30 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
           tc_fence_after();
           const uint32_t dlo = sdesc_lo(sdOa + st * C::TILE, kBoxBytes);
           const uint32_t qlo = sdesc_lo(sQa + st * C::TILE, kBoxBytes);
+          if (c.q < c.it.npairs - 1) {
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            const uint32_t roff = (kk * 16 * 128) >> 4;
-            const uint32_t acc = (c.q > 0 || kk > 0) ? 1u : 0u;
-            mma_ts(tmem + C::COL_DV, tmem + C::COL_P + kk * 8, sdesc_join(dlo + roff, kDescHi),
-                   idG, acc);
-            mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + kk * 8, sdesc_join(qlo + roff, kDescHi),
-                   idG, acc);
+            for (int kk = 0; kk < 128 / 16; ++kk) {
+              const uint32_t roff = (kk * 16 * 128) >> 4;
+              const uint32_t acc = (c.q > 0 || kk > 0) ? 1u : 0u;
+              mma_ts(tmem + C::COL_DV, tmem + C::COL_P + kk * 8, sdesc_join(dlo + roff, kDescHi),
+                     idG, acc);
+              mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + kk * 8, sdesc_join(qlo + roff, kDescHi),
+                     idG, acc);
+            }
+          } else {
+            // the item's last pair: every dV product, then every dK product, so that the
+            // epilogue's dV half starts while the dK products run
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              mma_ts(tmem + C::COL_DV, tmem + C::COL_P + kk * 8,
+                     sdesc_join(dlo + ((kk * 16 * 128) >> 4), kDescHi), idG,
+                     (c.q > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&bar->acc_dv);
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              mma_ts(tmem + C::COL_DK, tmem + C::COL_DS + kk * 8,
+                     sdesc_join(qlo + ((kk * 16 * 128) >> 4), kDescHi), idG,
+                     (c.q > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&bar->mm_done[0]);
           tc_commit(&bar->q_empty[st]);
@@ -1296,6 +1314,65 @@ __global__ void __launch_bounds__(DkvCfg<D>::THREADS, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------------- item epilogue
+      if constexpr (C::WIDE) {
+        // warpgroup h finishes columns 32 h .. 32 h + 31 of dV (once the item's dV products are
+        // done), then the same columns of dK (row krow of the key unit)
+        long long dst_row = -1;
+        const bool stage_row = it.window;
+        if (it.window) {
+          if (fj) {
+            int before = pre_tile;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q < (krow >> 5)) before += __popc(tile_words[q]);
+            before += __popc(tile_words[krow >> 5] & ((1u << (krow & 31)) - 1u));
+            dst_row = before;
+          }
+        } else if (r < cnt_b) {
+          dst_row = r;
+        }
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {  // 0: dV, 1: dK
+          if (!__all_sync(0xffffffffu, mbar_wait(m ? &bar->acc_full : &bar->acc_dv, I & 1, p.err,
+                                                 abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t acc[32];
+          tmem_ld32(tmem + lane_off + (m ? C::COL_DK : C::COL_DV) + 32 * h, acc);
+          tmem_ld_wait();
+          const float mul = m ? p.scale : 1.f;
+          if (dst_row >= 0) {
+            float* dst = (m ? p.dka : p.dva) +
+                         (((size_t)it.b * p.L + dst_row) * p.Hkv + it.kvh) * D + 32 * h;
+#pragma unroll
+            for (int z = 0; z < 8; ++z)
+              atomicAdd(reinterpret_cast<float4*>(dst) + z,
+                        make_float4(__uint_as_float(acc[4 * z]) * mul, __uint_as_float(acc[4 * z + 1]) * mul,
+                                    __uint_as_float(acc[4 * z + 2]) * mul, __uint_as_float(acc[4 * z + 3]) * mul));
+          }
+          if (stage_row) {
+            // bf16 into this item's K (dK) or V (dV) buffer, swizzled box layout
+            uint8_t* stage = (m ? sK : sV) + kb * C::TILE;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v4 = make_uint4(
+                  pack_bf16x2(__uint_as_float(acc[8 * q]) * mul, __uint_as_float(acc[8 * q + 1]) * mul),
+                  pack_bf16x2(__uint_as_float(acc[8 * q + 2]) * mul, __uint_as_float(acc[8 * q + 3]) * mul),
+                  pack_bf16x2(__uint_as_float(acc[8 * q + 4]) * mul, __uint_as_float(acc[8 * q + 5]) * mul),
+                  pack_bf16x2(__uint_as_float(acc[8 * q + 6]) * mul, __uint_as_float(acc[8 * q + 7]) * mul));
+              *reinterpret_cast<uint4*>(stage + sw128_offset(krow, 4 * h + q)) = v4;
+            }
+          }
+        }
+        if (!ok) break;
+        tc_fence_before();
+        mbar_arrive(&bar->acc_free);  // the next item may overwrite dV / dK
+        if (stage_row) fence_proxy_async_smem();
+        mbar_arrive(&bar->staged[kb]);  // the storer writes the rows out and frees the buffer
+        continue;
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&bar->acc_full, I & 1, p.err, abort_flag))) {
         ok = false;
         break;
